@@ -1,0 +1,452 @@
+"""Benchmark: block-sparse attention for diffusion-LLM denoising steps on B200.
+
+Workload: one bidirectional attention layer over the 8K / 256-step / 90 %-sparse
+denoising schedule of the Step-dLLM abstract (B=1, H=32, L=8192, d=128,
+64-token blocks, anchor every 32 steps), synthetic seeded bf16 inputs
+regenerated from the seed at every step.
+
+A step is one denoising step of that schedule: at anchor steps the block
+scores and the mask are rebuilt (sdl_block_scores + sdl_select_mask), then
+block-sparse attention runs (sdl_sparse_attn).  ``--steps K`` times steps
+0..K-1 (K=256 is the whole schedule); every step has its own inputs (192 MiB,
+larger than L2), all resident in HBM before the timed region starts.
+
+``value`` is the algorithmic sparse-attention throughput of the whole step
+loop: 4 * block^2 * d FLOP per kept block, times the kept blocks, over the
+device time of the K steps (anchor work included).  The JSON line also carries
+the kernel-only rate against the bf16 tensor peak, per-step latency, the dense
+baseline and the sparse/dense speedup, the end-to-end figure through host
+buffers, and the oracle's CPU time.
+
+Multi-GPU (torchrun): each rank runs its own independent sequence (weak
+scaling, no collective on the data path); the time is the max over ranks.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "bf16-L8192-H32-s90"
+METRIC = "sparse attn TFLOPS (% bf16 peak) + per-step latency & speedup vs dense at 8K/90%"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=256)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="sdl", choices=["sdl", "reference"])
+    p.add_argument("--workload", default=WORKLOAD)
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int):
+        self.ok = False
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            pass
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [k for k, v in self.REASONS.items() if self.reasons & v]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+    def rejected(self):
+        bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+        return bool(bad & set(self.summary()["reasons"]))
+
+
+# ------------------------------------------------------------------- steps
+
+
+class Runner:
+    """The library's step loop over per-step device inputs, with per-launch events."""
+
+    def __init__(self, w, seed, device):
+        import block_sparse_attention_sdl_b200 as sdl
+        from block_sparse_attention_sdl_b200.runtime import StepSparseAttention
+        self.sdl, self.w = sdl, w
+        self.att = StepSparseAttention(w.B, w.H, w.H_kv, w.L, w.d, w.bs, w.sparsity,
+                                       w.anchor_every, device=device)
+        self.out = torch.empty((w.B, w.L, w.H, w.d), dtype=torch.bfloat16, device=device)
+        self.seed = seed
+
+    def make_inputs(self, steps):
+        import synth
+        return [synth.device_inputs(self.w, s, self.seed) for s in steps]
+
+    def step(self, x, s, ev=None):
+        att, w = self.att, self.w
+        if s % w.anchor_every == 0 or att.mask_step is None:
+            if ev is not None:
+                ev["a0"].append(torch.cuda.Event(enable_timing=True))
+                ev["a0"][-1].record()
+            att.refresh(x["q"], x["k"], s)
+            if ev is not None:
+                ev["a1"].append(torch.cuda.Event(enable_timing=True))
+                ev["a1"][-1].record()
+        if ev is not None:
+            ev["s0"].append(torch.cuda.Event(enable_timing=True))
+            ev["s0"][-1].record()
+        self.sdl.sparse_attn(x["q"], x["k"], x["v"], att.row_ptr, att.col_idx, w.bs, out=self.out)
+        if ev is not None:
+            ev["s1"].append(torch.cuda.Event(enable_timing=True))
+            ev["s1"][-1].record()
+
+
+def barrier(dist_on):
+    if dist_on:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, dist_on, device):
+    if not dist_on:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(runner, inputs, steps, dist_on, device, with_events=True):
+    ev = {"a0": [], "a1": [], "s0": [], "s1": []} if with_events else None
+    runner.att.mask_step = None
+    barrier(dist_on)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for x, s in zip(inputs, steps):
+        runner.step(x, s, ev)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dist_on)
+    ms = e0.elapsed_time(e1)
+    return ms, ev
+
+
+def launches_per_anchor():
+    # pool, score; select: zero, 3 histogram passes, count, scan, write
+    return 2 + 7
+
+
+def e2e_measure(runner, inputs, steps, device):
+    """Same step loop with the inputs copied from pinned host memory and the
+    output copied back, every step, inside the timed region."""
+    ring = min(len(inputs), 8)
+    host_in = []
+    for x in inputs[:ring]:
+        host_in.append({k: v.cpu().pin_memory() for k, v in x.items()})
+    host_out = [torch.empty_like(runner.out, device="cpu").pin_memory() for _ in range(2)]
+    dev_in = {k: torch.empty_like(v) for k, v in inputs[0].items()}
+    bytes_in = sum(v.numel() * v.element_size() for v in dev_in.values())
+    bytes_out = runner.out.numel() * runner.out.element_size()
+
+    def loop(n):
+        runner.att.mask_step = None
+        for i in range(n):
+            h = host_in[i % ring]
+            for k in dev_in:
+                dev_in[k].copy_(h[k], non_blocking=True)
+            runner.step(dev_in, steps[i])
+            host_out[i % 2].copy_(runner.out, non_blocking=True)
+
+    loop(min(3, len(steps)))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    loop(len(steps))
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1), bytes_in, bytes_out
+
+
+def traffic_record():
+    """Per-launch DRAM bytes of the sparse kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "sparse_attn_traffic.json")
+    src = os.path.join(ROOT, "block_sparse_attention_sdl_b200", "csrc", "attn_tc.cu")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    if rec.get("attn_tc_sha256") != digest:
+        return None
+    return rec.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------- cpu oracle
+
+
+def cpu_oracle_sample(w, seed, target_s=8.0):
+    """Times the fp64 oracle's block-sparse attention on a bounded sample of the
+    workload's query rows (all heads, evenly spaced query blocks) of step 0 with
+    its anchor mask; returns (TFLOP/s, cores, description)."""
+    import oracle
+    import synth
+    host = synth.host_inputs(w, 0, seed)
+    P = oracle.block_scores(host["q"], host["k"], w.bs)
+    mask, _, _ = oracle.select(P, w.sparsity)
+    cores = os.cpu_count() or 1
+    nb = w.nb
+
+    def rows_for(nblk):
+        blocks = np.linspace(0, nb - 1, nblk).round().astype(int)
+        r = [(0, h, i * w.bs + t) for h in range(w.H) for i in blocks for t in range(w.bs)]
+        return np.array(r, dtype=np.int64)
+
+    def flops(rows):
+        kept = mask[rows[:, 0], rows[:, 1], rows[:, 2] // w.bs].sum(-1) * w.bs
+        return float((kept * 4 * w.d).sum())
+
+    rows = rows_for(1)
+    t0 = time.perf_counter()
+    oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=mask, rows=rows, nthreads=cores)
+    dt = time.perf_counter() - t0
+    nblk = int(min(nb, max(1, target_s / max(dt, 1e-3))))
+    rows = rows_for(nblk)
+    t0 = time.perf_counter()
+    oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=mask, rows=rows, nthreads=cores)
+    dt = time.perf_counter() - t0
+    desc = (f"block-sparse attention of {len(rows)} query rows ({nblk} of {nb} query blocks x "
+            f"{w.H} heads, step 0 with its anchor mask), fp64, {cores} threads")
+    return flops(rows) / dt / 1e12, cores, desc, dt
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle, timed per step on a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    per_step_target = max(0.5, 60.0 / max(1, args.steps + args.warmup))
+    vals, tot = [], 0.0
+    for i in range(args.warmup + args.steps):
+        v, cores, desc, dt = cpu_oracle_sample(w, args.seed, target_s=per_step_target)
+        if i >= args.warmup:
+            vals.append(v)
+            tot += dt
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox, see synth/)",
+        "config": {"workload": args.workload, "global_batch": w.B, "seq_len": w.L,
+                   "heads": w.H, "kv_heads": w.H_kv, "head_dim": w.d, "block": w.bs,
+                   "sparsity": w.sparsity, "parallelism": "cpu oracle"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import synth
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if dist_on:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = synth.WORKLOADS[args.workload]
+    seed = args.seed + rank  # each rank: its own independent sequence
+    runner = Runner(w, seed, device)
+    steps = list(range(args.steps))
+    inputs = runner.make_inputs(steps)
+    warm = [inputs[i % len(inputs)] for i in range(args.warmup)]
+    for x, s in zip(warm, range(args.warmup)):
+        runner.step(x, s)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    for attempt in range(2):
+        with sampler:
+            ms, ev = time_steps(runner, inputs, steps, dist_on, device)
+        if not sampler.rejected():
+            break
+        sampler = ClockSampler(local)
+    ms_max = max_over_ranks(ms, dist_on, device)
+
+    pk, pk_kind = peaks()
+    budget = runner.att.budget
+    flop_step = 4.0 * w.bs * w.bs * w.d * budget
+    value = flop_step * len(steps) * world / (ms_max * 1e-3) / 1e12
+    sparse_ms = [a.elapsed_time(b) for a, b in zip(ev["s0"], ev["s1"])]
+    anchor_ms = [a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])]
+    sp_avg = statistics.mean(sparse_ms)
+    kernel_tflops = flop_step / (sp_avg * 1e-3) / 1e12
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+
+    # anchor-step kernels, timed apart: scoring bandwidth and selection latency
+    sdl = runner.sdl
+    x0 = inputs[0]
+
+    def ev_time(fn, n=10):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    att = runner.att
+    sc_ms = ev_time(lambda: sdl.block_scores(x0["q"], x0["k"], w.bs, scores=att.scores,
+                                             workspace=att.ws_scores))
+    se_ms = ev_time(lambda: sdl.select_mask(att.scores, w.sparsity, w.bs, w.L,
+                                            row_ptr=att.row_ptr, col_idx=att.col_idx,
+                                            workspace=att.ws_select))
+    score_bytes = 2 * w.B * w.L * (w.H + w.H_kv) * w.d + 4 * w.B * w.H * w.nb * w.nb
+    # dense baseline on distinct inputs per launch (larger than L2 in total)
+    de = []
+    for i in range(min(6, len(inputs))):
+        x = inputs[i]
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        sdl.dense_attn(x["q"], x["k"], x["v"], out=runner.out)
+        b.record()
+        de.append((a, b))
+    torch.cuda.synchronize()
+    dense_ms = statistics.median([a.elapsed_time(b) for a, b in de[1:]] or
+                                 [de[0][0].elapsed_time(de[0][1])])
+    dense_flop = 4.0 * w.B * w.H * w.L * w.L * w.d
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, bi, bo = e2e_measure(runner, inputs, steps, device)
+        e_ms = max_over_ranks(e_ms, dist_on, device)
+        e2e = {"value": flop_step * len(steps) * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e_ms / len(steps)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, desc, _ = cpu_oracle_sample(w, seed)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    n_anchor = len(anchor_ms)
+    traffic = traffic_record()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": len(steps), "warmup": args.warmup, "ms_per_step": ms_max / len(steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Philox inputs shaped like the 8K/90% workload, regenerated "
+                "per step)",
+        "config": {"workload": args.workload, "global_batch": w.B * world, "seq_len": w.L,
+                   "heads": w.H, "kv_heads": w.H_kv, "head_dim": w.d, "block": w.bs,
+                   "sparsity": w.sparsity, "anchor_every": w.anchor_every,
+                   "parallelism": f"independent sequences x{world}",
+                   "l2": "inputs larger than L2 (192 MiB per step, distinct per step)"},
+        "sparse_attn_ms": sp_avg, "sparse_attn_tflops": kernel_tflops,
+        "pct_bf16_peak": kernel_tflops / peak,
+        "dense_attn_ms": dense_ms, "dense_attn_tflops": dense_flop / (dense_ms * 1e-3) / 1e12,
+        "speedup_vs_dense": dense_ms / sp_avg,
+        "speedup_vs_dense_amortized": dense_ms / (ms_max / len(steps)),
+        "anchor_ms": statistics.mean(anchor_ms) if anchor_ms else None,
+        "block_scores_ms": sc_ms, "block_scores_gbs": score_bytes / (sc_ms * 1e-3) / 1e9,
+        "select_mask_ms": se_ms, "mask_blocks": budget,
+        "tokens_steps_per_s": w.B * world * w.L * len(steps) / (ms_max * 1e-3),
+        "roofline": {"bound": "tensor", "achieved": kernel_tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": kernel_tflops / peak,
+                     "peak_source": f"bf16_tflops burst, {pk_kind}",
+                     "traffic": traffic},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": len(steps) + n_anchor * launches_per_anchor(),
+        "clocks": sampler.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if dist_on:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

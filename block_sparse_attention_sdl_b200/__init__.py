@@ -1,0 +1,227 @@
+"""Python binding of libsdl: block-sparse attention for diffusion-LLM denoising on B200.
+
+Argument marshalling only.  Every step runs in the CUDA kernels of ``libsdl.so``
+(built in-tree by :mod:`block_sparse_attention_sdl_b200.build`); PyTorch supplies
+device memory and streams.  There is no CPU fallback: importing this package on a
+machine without the built library raises.
+
+Tensors are laid out [B, L, heads, d] with the head dimension contiguous (any
+strides on the other axes).  The calls mirror ``include/sdl.h``:
+
+* :func:`block_scores`  pooled block scores with a row softmax (anchor steps)
+* :func:`select_mask`   head-adaptive global top-k block mask as CSR (anchor steps)
+* :func:`sparse_attn`   block-sparse attention over the kept blocks (every step)
+* :func:`dense_attn`    dense bidirectional attention (the baseline)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsdl.so")
+
+SDL_OK, SDL_ERR_INVALID_ARG, SDL_ERR_UNSUPPORTED, SDL_ERR_CAPACITY = 0, 1, 2, 3
+SDL_ERR_WORKSPACE, SDL_ERR_CUDA, SDL_ERR_TIMEOUT, SDL_ERR_BAD_MASK = 4, 5, 6, 7
+SDL_BF16, SDL_FP32 = 0, 1
+
+EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspace_bytes",
+           "sdl_block_scores", "sdl_select_mask", "sdl_sparse_attn", "sdl_dense_attn",
+           "sdl_last_device_status", "sdl_last_cuda_error", "sdl_status_string")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("H_kv", ctypes.c_int32),
+                ("L", ctypes.c_int32), ("d", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("q_strides", ctypes.c_int64 * 3), ("k_strides", ctypes.c_int64 * 3),
+                ("v_strides", ctypes.c_int64 * 3), ("o_strides", ctypes.c_int64 * 3)]
+
+
+class SdlError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = _lib().sdl_status_string(status).decode()
+        if status == SDL_ERR_CUDA:
+            msg += f" (cudaError {_lib().sdl_last_cuda_error()})"
+        super().__init__(f"{what}: {msg}")
+
+
+_L = None
+
+
+def _lib():
+    global _L
+    if _L is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m block_sparse_attention_sdl_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, SZ, D, F = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_double,
+                            ctypes.c_float)
+        SP = ctypes.POINTER(Shape)
+        L.sdl_mask_budget.argtypes = [SP, D]
+        L.sdl_mask_budget.restype = I64
+        L.sdl_scores_workspace_bytes.argtypes = [SP]
+        L.sdl_scores_workspace_bytes.restype = SZ
+        L.sdl_select_workspace_bytes.argtypes = [SP]
+        L.sdl_select_workspace_bytes.restype = SZ
+        L.sdl_block_scores.argtypes = [P, P, SP, F, P, P, SZ, P]
+        L.sdl_select_mask.argtypes = [P, SP, D, P, P, I64, P, P, SZ, P]
+        L.sdl_sparse_attn.argtypes = [P, P, P, SP, P, P, F, P, P, P]
+        L.sdl_dense_attn.argtypes = [P, P, P, SP, F, P, P, P]
+        L.sdl_last_device_status.argtypes = [P]
+        L.sdl_last_cuda_error.argtypes = []
+        L.sdl_status_string.argtypes = [ctypes.c_int]
+        L.sdl_status_string.restype = ctypes.c_char_p
+        for f in ("sdl_block_scores", "sdl_select_mask", "sdl_sparse_attn", "sdl_dense_attn",
+                  "sdl_last_device_status", "sdl_last_cuda_error"):
+            getattr(L, f).restype = ctypes.c_int
+        _L = L
+    return _L
+
+
+def lib():
+    """The loaded ``libsdl.so`` (ctypes handle)."""
+    return _lib()
+
+
+def _check(rc: int, what: str):
+    if rc != SDL_OK:
+        raise SdlError(rc, what)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return SDL_BF16
+    if t.dtype == torch.float32:
+        return SDL_FP32
+    raise TypeError(f"libsdl takes bf16 or fp32 tensors, got {t.dtype}")
+
+
+def _strides(t):
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("tensors are [B, L, heads, d] with a contiguous head dimension")
+    return (t.stride(0), t.stride(1), t.stride(2))
+
+
+def make_shape(q, k, block: int, v=None, o=None) -> Shape:
+    """sdl_shape for Q [B,L,H,d] and K/V [B,L,H_kv,d] tensors."""
+    B, L, H, d = q.shape
+    s = Shape()
+    s.B, s.H, s.H_kv, s.L, s.d, s.block = B, H, k.shape[2], L, d, block
+    s.dtype = _dtype_code(q)
+    s.q_strides[:] = _strides(q)
+    s.k_strides[:] = _strides(k)
+    s.v_strides[:] = _strides(v if v is not None else k)
+    s.o_strides[:] = _strides(o if o is not None else q)
+    return s
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def mask_budget(shape: Shape, sparsity: float) -> int:
+    return int(_lib().sdl_mask_budget(ctypes.byref(shape), float(sparsity)))
+
+
+def scores_workspace_bytes(shape: Shape) -> int:
+    return int(_lib().sdl_scores_workspace_bytes(ctypes.byref(shape)))
+
+
+def select_workspace_bytes(shape: Shape) -> int:
+    return int(_lib().sdl_select_workspace_bytes(ctypes.byref(shape)))
+
+
+def _workspace(nbytes, device, ws):
+    import torch
+    if ws is None:
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    return ws
+
+
+def block_scores(q, k, block: int, scale: float = 0.0, scores=None, workspace=None, stream=None):
+    """fp32 [B, H, nb, nb] block scores (see ``sdl_block_scores``)."""
+    import torch
+    s = make_shape(q, k, block)
+    nb = s.L // block
+    if scores is None:
+        scores = torch.empty((s.B, s.H, nb, nb), dtype=torch.float32, device=q.device)
+    need = scores_workspace_bytes(s)
+    workspace = _workspace(need, q.device, workspace)
+    _check(_lib().sdl_block_scores(q.data_ptr(), k.data_ptr(), ctypes.byref(s), float(scale),
+                                   scores.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                   _stream(stream)), "sdl_block_scores")
+    return scores
+
+
+def select_mask(scores, sparsity: float, block: int, L: int, row_ptr=None, col_idx=None,
+                mask=None, want_mask: bool = False, workspace=None, stream=None):
+    """(row_ptr int32 [B*H*nb+1], col_idx int32 [budget], mask uint8 or None)."""
+    import torch
+    B, H, nb, _ = scores.shape
+    s = Shape()
+    s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, H, L, 64, block, SDL_FP32
+    if nb != L // block:
+        raise ValueError("scores shape does not match L / block")
+    total = mask_budget(s, sparsity)
+    if total < 0:
+        raise SdlError(SDL_ERR_INVALID_ARG, "sdl_mask_budget")
+    dev = scores.device
+    if row_ptr is None:
+        row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty(total, dtype=torch.int32, device=dev)
+    if mask is None and want_mask:
+        mask = torch.empty((B, H, nb, nb), dtype=torch.uint8, device=dev)
+    workspace = _workspace(select_workspace_bytes(s), dev, workspace)
+    _check(_lib().sdl_select_mask(scores.data_ptr(), ctypes.byref(s), float(sparsity),
+                                  row_ptr.data_ptr(), col_idx.data_ptr(), col_idx.numel(),
+                                  None if mask is None else mask.data_ptr(),
+                                  workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "sdl_select_mask")
+    return row_ptr, col_idx, mask
+
+
+def sparse_attn(q, k, v, row_ptr, col_idx, block: int, scale: float = 0.0, out=None, lse=None,
+                want_lse: bool = False, stream=None):
+    """O like q (and LSE fp32 [B,H,L] when asked) over the kept blocks."""
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    s = make_shape(q, k, block, v, out)
+    if lse is None and want_lse:
+        lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
+    _check(_lib().sdl_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(s),
+                                  row_ptr.data_ptr(), col_idx.data_ptr(), float(scale),
+                                  out.data_ptr(), None if lse is None else lse.data_ptr(),
+                                  _stream(stream)), "sdl_sparse_attn")
+    return (out, lse) if want_lse or lse is not None else out
+
+
+def dense_attn(q, k, v, block: int = 64, scale: float = 0.0, out=None, lse=None,
+               want_lse: bool = False, stream=None):
+    """Dense bidirectional attention (the baseline)."""
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    s = make_shape(q, k, block, v, out)
+    if lse is None and want_lse:
+        lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
+    _check(_lib().sdl_dense_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(s),
+                                 float(scale), out.data_ptr(),
+                                 None if lse is None else lse.data_ptr(), _stream(stream)),
+           "sdl_dense_attn")
+    return (out, lse) if want_lse or lse is not None else out
+
+
+def last_device_status(stream=None) -> int:
+    """Synchronizes the stream and returns (and clears) the kernels' status code."""
+    return int(_lib().sdl_last_device_status(_stream(stream)))

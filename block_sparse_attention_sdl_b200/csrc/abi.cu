@@ -1,0 +1,286 @@
+// extern "C" entry points of libsdl: argument validation, budget arithmetic,
+// TMA descriptor encoding, launches and the device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "internal.cuh"
+
+namespace sdl {
+
+__device__ int g_device_status;
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+sdl_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = (int)e;
+  return SDL_ERR_CUDA;
+}
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+std::mutex g_mu;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by every call.  Returns SDL_OK or the error to report.
+sdl_status check_shape(const sdl_shape* s) {
+  if (!s) return SDL_ERR_INVALID_ARG;
+  if (s->B <= 0 || s->H <= 0 || s->H_kv <= 0 || s->L <= 0 || s->d <= 0 || s->block <= 0)
+    return SDL_ERR_INVALID_ARG;
+  if (s->H % s->H_kv) return SDL_ERR_INVALID_ARG;
+  if (s->dtype != SDL_BF16 && s->dtype != SDL_FP32) return SDL_ERR_INVALID_ARG;
+  if (s->block != 64 && s->block != 128) return SDL_ERR_UNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return SDL_ERR_UNSUPPORTED;
+  if (s->L % s->block) return SDL_ERR_UNSUPPORTED;
+  if (s->L > 65536) return SDL_ERR_UNSUPPORTED;
+  if ((int64_t)s->B * s->H * (s->L / s->block) * (s->L / s->block) >= (int64_t)1 << 31)
+    return SDL_ERR_UNSUPPORTED;
+  return SDL_OK;
+}
+
+sdl_status check_strides(const int64_t* st, int dtype) {
+  const int64_t q = dtype == SDL_BF16 ? 8 : 4;  // elements per 16 bytes
+  for (int i = 0; i < 3; ++i)
+    if (st[i] < 0 || st[i] % q) return SDL_ERR_INVALID_ARG;
+  return SDL_OK;
+}
+
+float resolve_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / sqrtf((float)d); }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4-D map over a [B, L, heads, d] bf16 tensor: dims (d, t, h, b), box of
+// 64 d-columns x 64 tokens, 128-byte swizzle, zero fill out of range.
+bool encode_bf16_map(CUtensorMap* map, const void* base, const sdl_shape& s, int heads,
+                     const int64_t* st) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)s.L, (cuuint64_t)heads, (cuuint64_t)s.B};
+  cuuint64_t strides[3] = {(cuuint64_t)st[1] * 2, (cuuint64_t)st[2] * 2, (cuuint64_t)st[0] * 2};
+  // a zero stride (broadcast) is not expressible: use the dimension's natural size
+  for (int i = 0; i < 3; ++i)
+    if (strides[i] == 0) strides[i] = 16;
+  cuuint32_t box[4] = {64, 64, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_shape* shape,
+                       const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
+                       float* lse, void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  const sdl_shape& s = *shape;
+  if (!q || !k || !v || !o) return SDL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return SDL_ERR_INVALID_ARG;
+  if ((e = check_strides(s.q_strides, s.dtype)) || (e = check_strides(s.k_strides, s.dtype)) ||
+      (e = check_strides(s.v_strides, s.dtype)) || (e = check_strides(s.o_strides, s.dtype)))
+    return e;
+  int* status = device_status_ptr();
+  if (!status) return SDL_ERR_CUDA;
+  AttnArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.B = s.B;
+  a.H = s.H;
+  a.Hkv = s.H_kv;
+  a.L = s.L;
+  a.d = s.d;
+  a.block = s.block;
+  a.nb = s.L / s.block;
+  for (int i = 0; i < 3; ++i) {
+    a.qs[i] = s.q_strides[i];
+    a.ks[i] = s.k_strides[i];
+    a.vs[i] = s.v_strides[i];
+    a.os[i] = s.o_strides[i];
+  }
+  a.scale = resolve_scale(scale, s.d);
+  a.scale_log2 = a.scale * 1.4426950408889634f;
+  a.status = status;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t ce;
+  if (s.dtype == SDL_BF16) {
+    CUtensorMap tq, tk, tv;
+    if (!encode_bf16_map(&tq, q, s, s.H, s.q_strides) ||
+        !encode_bf16_map(&tk, k, s, s.H_kv, s.k_strides) ||
+        !encode_bf16_map(&tv, v, s, s.H_kv, s.v_strides))
+      return cuda_fail(cudaErrorInvalidValue);
+    ce = launch_attn_tc(a, &tq, &tk, &tv, st);
+  } else {
+    ce = launch_attn_simt(a, st);
+  }
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+}  // namespace
+
+int* device_status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+}  // namespace sdl
+
+using namespace sdl;
+
+extern "C" {
+
+int64_t sdl_mask_budget(const sdl_shape* shape, double sparsity) {
+  if (check_shape(shape) != SDL_OK) return -1;
+  if (!(sparsity >= 0.0 && sparsity < 1.0)) return -1;
+  const int64_t nb = shape->L / shape->block;
+  const double per = (double)shape->H * (double)nb * (double)nb;
+  const int64_t kb = (int64_t)floor((1.0 - sparsity) * per + 0.5);
+  if (kb < (int64_t)shape->H * nb) return -1;
+  return kb * shape->B;
+}
+
+size_t sdl_scores_workspace_bytes(const sdl_shape* shape) {
+  if (check_shape(shape) != SDL_OK) return 0;
+  const size_t nb = shape->L / shape->block;
+  return align256(sizeof(float) * shape->B * shape->H * nb * shape->d) +
+         align256(sizeof(float) * shape->B * shape->H_kv * nb * shape->d);
+}
+
+size_t sdl_select_workspace_bytes(const sdl_shape* shape) {
+  if (check_shape(shape) != SDL_OK) return 0;
+  return select_workspace_bytes(shape->B, shape->H, shape->L / shape->block);
+}
+
+sdl_status sdl_block_scores(const void* q, const void* k, const sdl_shape* shape, float scale,
+                            float* scores, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  const sdl_shape& s = *shape;
+  if (!q || !k || !scores) return SDL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(scores)) return SDL_ERR_INVALID_ARG;
+  if ((e = check_strides(s.q_strides, s.dtype)) || (e = check_strides(s.k_strides, s.dtype)))
+    return e;
+  const size_t need = sdl_scores_workspace_bytes(shape);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SDL_ERR_WORKSPACE;
+  const size_t nb = s.L / s.block;
+  float* qbar = static_cast<float*>(workspace);
+  float* kbar = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         align256(sizeof(float) * s.B * s.H * nb * s.d));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t ce = launch_pool(q, k, s, qbar, kbar, st);
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  ce = launch_scores(qbar, kbar, s, resolve_scale(scale, s.d), scores, st);
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_select_mask(const float* scores, const sdl_shape* shape, double sparsity,
+                           int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                           uint8_t* mask_u8, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  if (!scores || !row_ptr || !col_idx) return SDL_ERR_INVALID_ARG;
+  if (!aligned16(scores)) return SDL_ERR_INVALID_ARG;
+  const int64_t total = sdl_mask_budget(shape, sparsity);
+  if (total < 0) return SDL_ERR_INVALID_ARG;
+  if (col_capacity < total) return SDL_ERR_CAPACITY;
+  const size_t need = sdl_select_workspace_bytes(shape);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SDL_ERR_WORKSPACE;
+  const int nb = shape->L / shape->block;
+  cudaError_t ce = launch_select(scores, shape->B, shape->H, nb, total / shape->B, row_ptr,
+                                 col_idx, mask_u8, workspace, static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_sparse_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,
+                           const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
+                           float* lse, void* stream) {
+  if (!row_ptr || !col_idx) return SDL_ERR_INVALID_ARG;
+  return attn_common(q, k, v, shape, row_ptr, col_idx, scale, o, lse, stream);
+}
+
+sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,
+                          float scale, void* o, float* lse, void* stream) {
+  return attn_common(q, k, v, shape, nullptr, nullptr, scale, o, lse, stream);
+}
+
+sdl_status sdl_last_device_status(void* stream) {
+  cudaError_t ce = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  int v = 0;
+  ce = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  const int zero = 0;
+  ce = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  if (v & kDevTimeout) return SDL_ERR_TIMEOUT;
+  if (v & kDevBadMask) return SDL_ERR_BAD_MASK;
+  return SDL_OK;
+}
+
+int sdl_last_cuda_error(void) { return t_last_cuda_error; }
+
+const char* sdl_status_string(sdl_status status) {
+  switch (status) {
+    case SDL_OK:
+      return "ok";
+    case SDL_ERR_INVALID_ARG:
+      return "invalid argument";
+    case SDL_ERR_UNSUPPORTED:
+      return "unsupported shape (d, block or L)";
+    case SDL_ERR_CAPACITY:
+      return "col_idx capacity below the mask budget";
+    case SDL_ERR_WORKSPACE:
+      return "workspace missing or too small";
+    case SDL_ERR_CUDA:
+      return "CUDA error (see sdl_last_cuda_error)";
+    case SDL_ERR_TIMEOUT:
+      return "a kernel's bounded wait timed out";
+    case SDL_ERR_BAD_MASK:
+      return "mask list entry out of range or out of order";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

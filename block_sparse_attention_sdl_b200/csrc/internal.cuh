@@ -1,0 +1,51 @@
+// Declarations shared by the translation units of libsdl.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sdl.h"
+
+namespace sdl {
+
+// Device status word bits (set by kernels, read by sdl_last_device_status).
+enum : int { kDevTimeout = 1, kDevBadMask = 2 };
+
+// Wall-time bound for every spin wait inside a kernel.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+int* device_status_ptr();  // address of the library's device status word
+
+// List entries handed to the attention kernels: 64-token key sub-block index
+// in the low 16 bits, and in bits 16..17 which halves (query rows 0..63,
+// 64..127) of a 128-row query tile keep it.
+constexpr int kSubBlock = 64;
+
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  const int32_t* row_ptr;  // null: dense
+  const int32_t* col_idx;
+  int B, H, Hkv, L, d, block, nb;
+  int64_t qs[3], ks[3], vs[3], os[3];
+  float scale_log2;  // scale * log2(e)
+  float scale;
+  int* status;
+};
+
+cudaError_t launch_pool(const void* q, const void* k, const sdl_shape& s, float* qbar, float* kbar,
+                        cudaStream_t st);
+cudaError_t launch_scores(const float* qbar, const float* kbar, const sdl_shape& s, float scale,
+                          float* scores, cudaStream_t st);
+cudaError_t launch_select(const float* scores, int B, int H, int nb, int64_t kb, int32_t* row_ptr,
+                          int32_t* col_idx, uint8_t* mask, void* ws, cudaStream_t st);
+size_t select_workspace_bytes(int B, int H, int nb);
+cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
+                           const CUtensorMap* tv, cudaStream_t st);
+cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t st);
+
+}  // namespace sdl

@@ -1,0 +1,140 @@
+/*
+ * sdl.h -- C ABI of libsdl, block-sparse attention for diffusion-LLM
+ * denoising steps on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow "Step-dLLM: Adaptive Step-aware Sparse Attention for
+ * Efficient Diffusion LLM Inference" (mlinfo.pages.dev, abstract): at anchor
+ * steps of the denoising trajectory a block-sparse mask is rebuilt under one
+ * head-adaptive global budget, it is reused until the next anchor, and a
+ * fused block-sparse attention kernel evaluates bidirectional attention on
+ * the kept blocks only; dense FlashAttention is the baseline.  The abstract
+ * does not define the block score or the selection rule; the readings this
+ * library implements are stated at each call.
+ *
+ * Conventions for every call:
+ *   - All pointers named q, k, v, o, lse, scores, row_ptr, col_idx, mask_u8
+ *     and workspace are DEVICE pointers owned by the caller.  The library
+ *     allocates no device memory per call.  It keeps one device status word
+ *     and, per device, a small cache of TMA descriptors.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream).  Argument errors are returned
+ *     before anything is launched; a launch failure returns SDL_ERR_CUDA and
+ *     sdl_last_cuda_error() gives the cudaError_t.
+ *   - Q is [B, L, H, d], K and V are [B, L, H_kv, d] and O is [B, L, H, d],
+ *     each addressed through element strides (b, t, h) with d contiguous.
+ *   - bf16 tensors must start on 16-byte boundaries and have strides that are
+ *     multiples of 8 elements (the tensor-memory-access unit's rule).
+ *   - No exception or abort crosses the ABI.
+ */
+#ifndef SDL_H
+#define SDL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SDL_OK = 0,
+  SDL_ERR_INVALID_ARG = 1, /* null pointer, bad size or stride, bad sparsity */
+  SDL_ERR_UNSUPPORTED = 2, /* valid but not implemented: d, block, L % block */
+  SDL_ERR_CAPACITY = 3,    /* col_capacity below the budget */
+  SDL_ERR_WORKSPACE = 4,   /* workspace null or smaller than required */
+  SDL_ERR_CUDA = 5,        /* a CUDA call failed; see sdl_last_cuda_error() */
+  SDL_ERR_TIMEOUT = 6,     /* a kernel's bounded wait ran out (device status) */
+  SDL_ERR_BAD_MASK = 7     /* a col_idx entry out of range or out of order */
+} sdl_status;
+
+typedef enum { SDL_BF16 = 0, SDL_FP32 = 1 } sdl_dtype;
+
+typedef struct {
+  int32_t B;     /* batch (independent sequences) */
+  int32_t H;     /* query heads */
+  int32_t H_kv;  /* key/value heads; H % H_kv == 0, query head h reads KV head h / (H / H_kv) */
+  int32_t L;     /* tokens per sequence; L % block == 0 */
+  int32_t d;     /* head dimension: 64 or 128 */
+  int32_t block; /* block size in tokens: 64 or 128 */
+  int32_t dtype; /* sdl_dtype of q, k, v, o */
+  int32_t reserved;
+  int64_t q_strides[3]; /* element strides of the (b, t, h) axes */
+  int64_t k_strides[3];
+  int64_t v_strides[3];
+  int64_t o_strides[3];
+} sdl_shape;
+
+/* Blocks kept for the whole call: B * floor((1 - sparsity) * H * nb^2 + 0.5),
+ * nb = L / block.  The budget is per batch element (each sequence is its own
+ * problem) and counts the H * nb diagonal blocks that are always kept.
+ * Returns -1 for a bad shape, sparsity outside [0, 1), or a per-sequence
+ * budget below H * nb.  Host-only; launches nothing. */
+int64_t sdl_mask_budget(const sdl_shape* shape, double sparsity);
+
+/* Workspace bytes that sdl_block_scores / sdl_select_mask need (0 on a bad shape). */
+size_t sdl_scores_workspace_bytes(const sdl_shape* shape);
+size_t sdl_select_workspace_bytes(const sdl_shape* shape);
+
+/* Block scores (anchor steps).  The Step-dLLM abstract refreshes the mask at
+ * anchor steps but leaves the block-importance estimate open; this call
+ * implements mean pooling of Q and K over each block, the pooled product and
+ * a row softmax:
+ *   Qbar[b,h,i,:] = mean_{t in block i} Q[b,t,h,:],  Kbar likewise per KV head,
+ *   scores[b,h,i,j] = softmax_j(scale * Qbar[b,h,i,:] . Kbar[b,h/g,j,:]).
+ * scores: fp32 [B, H, nb, nb] row-major.  scale <= 0 means 1/sqrt(d).
+ * workspace: at least sdl_scores_workspace_bytes(shape) bytes (pooled Q, K). */
+sdl_status sdl_block_scores(const void* q, const void* k, const sdl_shape* shape, float scale,
+                            float* scores, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Mask selection (anchor steps): the head-adaptive global budget of the
+ * Step-dLLM abstract.  Per batch element, every diagonal block (i, i) of every
+ * head is kept, and the rest of the budget goes to the largest off-diagonal
+ * scores of ALL heads together (ties: lower flat index (h*nb + i)*nb + j
+ * first), so heads whose mass is concentrated in few blocks keep few blocks.
+ * Output is CSR over query-block rows r = (b*H + h)*nb + i:
+ *   row_ptr: int32 [B*H*nb + 1], col_idx: int32 [budget], ascending j per row.
+ * col_capacity must be >= sdl_mask_budget() (else SDL_ERR_CAPACITY).
+ * mask_u8 (nullable): uint8 [B, H, nb, nb], 1 = kept.
+ * workspace: at least sdl_select_workspace_bytes(shape) bytes; its contents
+ * on entry do not matter.  Only shape->B, H, L, block are read. */
+sdl_status sdl_select_mask(const float* scores, const sdl_shape* shape, double sparsity,
+                           int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                           uint8_t* mask_u8, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* Block-sparse attention (every step), the fused kernel of the Step-dLLM
+ * abstract: for token t of query block i of head h,
+ *   O[b,t,h,:] = sum_u softmax_u(scale * q_t . k_u) v_u
+ * over the tokens u of the blocks col_idx[row_ptr[r] .. row_ptr[r+1]) of row
+ * r = (b*H + h)*nb + i, non-causal, K and V read from KV head h / (H/H_kv).
+ * Lists must be ascending with entries in [0, nb); a bad entry is skipped and
+ * reported as SDL_ERR_BAD_MASK by sdl_last_device_status().
+ * lse (nullable): fp32 [B, H, L], natural-log sum of exp of the logits.
+ * scale <= 0 means 1/sqrt(d).  bf16 runs on tcgen05 tensor cores (fp32
+ * accumulation, output rounded to nearest even); fp32 runs on CUDA cores. */
+sdl_status sdl_sparse_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,
+                           const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
+                           float* lse, void* stream);
+
+/* Dense bidirectional attention, the baseline of the same abstract: the
+ * sparse call with every block of every row kept. */
+sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,
+                          float scale, void* o, float* lse, void* stream);
+
+/* Synchronizes `stream`, then reports and clears the device status word set by
+ * kernels: SDL_ERR_TIMEOUT if a bounded wait ran out, SDL_ERR_BAD_MASK if a
+ * list entry was rejected, SDL_OK otherwise. */
+sdl_status sdl_last_device_status(void* stream);
+
+/* cudaError_t of the last failed CUDA call in this thread (0 if none). */
+int sdl_last_cuda_error(void);
+
+/* Static description of a status code. */
+const char* sdl_status_string(sdl_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDL_H */

@@ -1,0 +1,98 @@
+"""The C-ABI library: loads without a GPU, exports every declared symbol, and
+validates arguments on the host (no call here reaches the GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sdl.h")
+
+sdl = pytest.importorskip("block_sparse_attention_sdl_b200")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(sdl_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 10
+    lib = sdl.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(sdl.EXPORTS)
+
+
+def _shape(B=1, H=32, Hkv=32, L=8192, d=128, block=64, dtype=0):
+    s = sdl.Shape()
+    s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, Hkv, L, d, block, dtype
+    for arr in (s.q_strides, s.k_strides, s.v_strides, s.o_strides):
+        arr[:] = (L * H * d, H * d, d)
+    return s
+
+
+@pytest.mark.parametrize("H,L,block,s", [(2, 512, 64, 0.5), (32, 2048, 64, 0.8),
+                                         (32, 8192, 64, 0.9), (28, 16384, 64, 0.9),
+                                         (32, 65536, 128, 0.95), (4, 1024, 128, 0.3)])
+def test_budget_matches_oracle(H, L, block, s):
+    shp = _shape(H=H, Hkv=H if H != 28 else 4, L=L, block=block)
+    nb = L // block
+    assert sdl.mask_budget(shp, s) == oracle.budget(H, nb, s)
+    shp.B = 3
+    assert sdl.mask_budget(shp, s) == 3 * oracle.budget(H, nb, s)
+
+
+def test_budget_rejects_bad_sparsity():
+    shp = _shape(H=2, Hkv=2, L=512)
+    for s in (1.0, -0.01, float("nan"), 0.9):  # 0.9 keeps 13 < 16 diagonal blocks
+        assert sdl.mask_budget(shp, s) == -1
+
+
+def test_shape_validation():
+    lib = sdl.lib()
+    assert sdl.scores_workspace_bytes(_shape()) > 0
+    assert sdl.select_workspace_bytes(_shape()) > 0
+    for bad in (_shape(block=96), _shape(d=96), _shape(L=8192 + 32), _shape(L=8192 + 64, block=128), _shape(Hkv=5),
+                _shape(B=0), _shape(dtype=7), _shape(L=131072)):
+        assert sdl.select_workspace_bytes(bad) == 0
+        assert sdl.mask_budget(bad, 0.5) == -1
+    P = ctypes.c_void_p
+    # null pointers and bad shapes are refused before any CUDA call
+    rc = lib.sdl_dense_attn(None, None, None, ctypes.byref(_shape()), 0.0, None, None, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+    rc = lib.sdl_dense_attn(P(16), P(16), P(16), ctypes.byref(_shape(block=96)), 0.0, P(16),
+                            None, None)
+    assert rc == sdl.SDL_ERR_UNSUPPORTED
+    rc = lib.sdl_dense_attn(P(8), P(16), P(16), ctypes.byref(_shape()), 0.0, P(16), None, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG  # misaligned q
+    bad_stride = _shape()
+    bad_stride.k_strides[1] = 4100
+    rc = lib.sdl_dense_attn(P(16), P(16), P(16), ctypes.byref(bad_stride), 0.0, P(16), None, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+    rc = lib.sdl_sparse_attn(P(16), P(16), P(16), ctypes.byref(_shape()), None, None, 0.0,
+                             P(16), None, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+    rc = lib.sdl_block_scores(P(16), P(16), ctypes.byref(_shape()), 0.0, P(16), None, 0, None)
+    assert rc == sdl.SDL_ERR_WORKSPACE
+    shp = _shape(H=2, Hkv=2, L=512)
+    rc = lib.sdl_select_mask(P(16), ctypes.byref(shp), 0.5, P(16), P(16), 10, None, P(16),
+                             1 << 20, None)
+    assert rc == sdl.SDL_ERR_CAPACITY
+    rc = lib.sdl_select_mask(P(16), ctypes.byref(shp), 0.5, P(16), P(16), 64, None, P(16), 16,
+                             None)
+    assert rc == sdl.SDL_ERR_WORKSPACE
+    rc = lib.sdl_select_mask(P(16), ctypes.byref(shp), 1.5, P(16), P(16), 64, None, P(16),
+                             1 << 20, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    lib = sdl.lib()
+    for code in range(8):
+        assert lib.sdl_status_string(code)
+    assert lib.sdl_last_cuda_error() == 0

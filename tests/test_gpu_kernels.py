@@ -1,0 +1,238 @@
+"""GPU parity of each library call against the fp64 oracle on small shapes.
+
+Shapes span several 128-row tiles and a ragged tail (odd block counts), both
+block sizes, both head dims, GQA groups 1/2/7, bf16 and fp32, and strided
+(fused-QKV) layouts.  Attention is checked with the GPU's own mask, so mask
+parity and attention parity are independent.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.parity_util import (TOL, bf16_to_f64, check_close, check_csr, compare_masks,
+                               csr_to_mask)
+
+pytestmark = pytest.mark.gpu
+
+sdl = pytest.importorskip("block_sparse_attention_sdl_b200")
+
+
+def _inputs(w, step=0):
+    host = synth.host_inputs(w, step)
+    dev = synth.device_inputs(w, step)
+    return host, dev
+
+
+def _mask_to_csr(mask):
+    B, H, nb, _ = mask.shape
+    flat = mask.reshape(-1, nb)
+    row_ptr = np.zeros(flat.shape[0] + 1, dtype=np.int32)
+    row_ptr[1:] = np.cumsum(flat.sum(1))
+    col_idx = np.concatenate([np.nonzero(r)[0] for r in flat]).astype(np.int32)
+    return torch.from_numpy(row_ptr).cuda(), torch.from_numpy(col_idx).cuda()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("L,H,Hkv,d", [(256, 2, 2, 64), (1024, 4, 2, 128), (640, 7, 1, 128)])
+def test_generator_twins_bit_identical(dtype, L, H, Hkv, d):
+    w = synth.small_workload(dtype=dtype, L=L, H=H, H_kv=Hkv, d=d, planted=2)
+    for step in (0, 3):
+        for x in ("q", "k", "v"):
+            host = synth.host_tensor(w, x, step)
+            dev = synth.device_tensor(w, x, step).cpu()
+            if dtype == "bf16":
+                dev = dev.view(torch.int16).numpy().view(np.uint16)
+            else:
+                dev = dev.numpy()
+            assert np.array_equal(host, dev), (x, step)
+
+
+SCORE_CASES = [
+    ("bf16", 512, 2, 2, 64, 64),
+    ("bf16", 2048, 4, 4, 128, 64),
+    ("bf16", 1024, 7, 1, 128, 64),
+    ("bf16", 2048, 2, 1, 128, 128),
+    ("fp32", 512, 2, 2, 64, 64),
+    ("fp32", 1024, 4, 2, 128, 128),
+]
+
+
+@pytest.mark.parametrize("dtype,L,H,Hkv,d,bs", SCORE_CASES)
+def test_block_scores(dtype, L, H, Hkv, d, bs):
+    w = synth.small_workload(dtype=dtype, L=L, H=H, H_kv=Hkv, d=d, bs=bs, planted=2)
+    host, dev = _inputs(w)
+    P = sdl.block_scores(dev["q"], dev["k"], bs)
+    torch.cuda.synchronize()
+    want = oracle.block_scores(host["q"], host["k"], bs)
+    got = P.cpu().numpy().astype(np.float64)
+    rel = np.abs(got - want) / want
+    assert rel.max() < 2e-5, rel.max()
+    assert np.allclose(got.sum(-1), 1.0, atol=1e-5)
+
+
+@pytest.mark.parametrize("B,H,nb,s", [(1, 2, 8, 0.5), (1, 4, 32, 0.8), (2, 3, 16, 0.7),
+                                      (1, 32, 128, 0.9), (1, 2, 5, 0.3)])
+def test_select_matches_oracle(B, H, nb, s):
+    rng = np.random.default_rng(nb * 7 + H)
+    logits = rng.standard_normal((B, H, nb, nb)) * rng.uniform(0.2, 3.0, (1, H, 1, 1))
+    P = np.exp(logits) / np.exp(logits).sum(-1, keepdims=True)
+    P32 = P.astype(np.float32)
+    # the oracle sees the same fp32 values the kernel sees
+    want, tau, kept = oracle.select(P32.astype(np.float64), s)
+    row_ptr, col_idx, mask = sdl.select_mask(torch.from_numpy(P32).cuda(), s, 64, nb * 64,
+                                             want_mask=True)
+    torch.cuda.synchronize()
+    rp, ci = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
+    check_csr(rp, ci, B, H, nb, kept)
+    got = csr_to_mask(rp, ci, B, H, nb)
+    assert np.array_equal(got, mask.cpu().numpy())
+    assert np.array_equal(got, want)  # identical fp32 inputs: no excuse needed
+
+
+def test_select_exact_ties_follow_flat_index():
+    B, H, nb = 1, 3, 16
+    P = np.full((B, H, nb, nb), 1.0 / nb, dtype=np.float32)
+    P[0, 1, :, 5] = 0.5  # some strictly larger entries
+    for s in (0.6, 0.75, 0.9):
+        want, _, kept = oracle.select(P.astype(np.float64), s)
+        rp, ci, _ = sdl.select_mask(torch.from_numpy(P).cuda(), s, 64, nb * 64)
+        got = csr_to_mask(rp.cpu().numpy(), ci.cpu().numpy(), B, H, nb)
+        assert np.array_equal(got, want), s
+
+
+def test_select_extremes():
+    P = torch.rand(1, 2, 8, 8).cuda()
+    rp, ci, _ = sdl.select_mask(P, 0.0, 64, 512)
+    assert ci.numel() == 128 and torch.equal(rp[-1].cpu(), torch.tensor(128, dtype=torch.int32))
+    s_diag = 1.0 - 16 / 128
+    rp, ci, _ = sdl.select_mask(P, s_diag, 64, 512)
+    assert torch.equal(ci.cpu(), torch.arange(8, dtype=torch.int32).repeat(2))
+
+
+def test_select_reuses_workspace_across_calls():
+    """Workspace contents on entry do not matter: a dirty workspace gives the same mask."""
+    P = torch.rand(1, 4, 32, 32, device="cuda")
+    P = P / P.sum(-1, keepdim=True)
+    ws = torch.full((1 << 20,), 0xAB, dtype=torch.uint8, device="cuda")
+    a = sdl.select_mask(P, 0.8, 64, 2048, workspace=ws)
+    b = sdl.select_mask(P, 0.8, 64, 2048, workspace=ws)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+ATTN_CASES = [
+    # dtype, B, L, H, Hkv, d, bs, density
+    ("bf16", 1, 256, 2, 2, 128, 64, 0.5),
+    ("bf16", 1, 320, 2, 1, 128, 64, 0.5),  # odd block count: ragged last tile
+    ("bf16", 2, 1024, 4, 2, 128, 64, 0.3),
+    ("bf16", 1, 1024, 7, 1, 128, 64, 0.25),
+    ("bf16", 1, 1024, 2, 2, 128, 128, 0.4),
+    ("bf16", 1, 512, 2, 2, 64, 64, 0.5),
+    ("bf16", 1, 768, 4, 4, 64, 128, 0.5),
+    ("fp32", 1, 512, 2, 2, 64, 64, 0.5),
+    ("fp32", 1, 512, 2, 1, 128, 128, 0.5),
+]
+
+
+def _random_mask(B, H, nb, density, rng):
+    m = (rng.random((B, H, nb, nb)) < density).astype(np.uint8)
+    for i in range(nb):
+        m[:, :, i, i] = 1
+    return m
+
+
+@pytest.mark.parametrize("dtype,B,L,H,Hkv,d,bs,density", ATTN_CASES)
+def test_sparse_attention(dtype, B, L, H, Hkv, d, bs, density):
+    w = synth.Workload("t", dtype, B, H, Hkv, L, d, bs, 0.5, 1, 1, 0.02, ("uniform", 0.3, 4.0), 1)
+    host, dev = _inputs(w)
+    nb = L // bs
+    rng = np.random.default_rng(L + H)
+    mask = _random_mask(B, H, nb, density, rng)
+    rp, ci = _mask_to_csr(mask)
+    O, lse = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, bs, want_lse=True)
+    assert sdl.last_device_status() == sdl.SDL_OK
+    Ow, lw = oracle.attention(host["q"], host["k"], host["v"], bs, mask=mask)
+    got = bf16_to_f64(O).transpose(0, 2, 1, 3)
+    check_close(got, Ow, dtype)
+    assert np.abs(lse.cpu().numpy() - lw).max() <= TOL[dtype]["lse"]
+
+
+@pytest.mark.parametrize("kind", ["diag", "ones", "single_far"])
+@pytest.mark.parametrize("bs", [64, 128])
+def test_sparse_attention_edge_masks(kind, bs):
+    w = synth.small_workload(L=1024, H=2, H_kv=2, d=128, bs=bs)
+    host, dev = _inputs(w)
+    nb = 1024 // bs
+    if kind == "diag":
+        mask = np.broadcast_to(np.eye(nb, dtype=np.uint8), (1, 2, nb, nb)).copy()
+    elif kind == "ones":
+        mask = np.ones((1, 2, nb, nb), np.uint8)
+    else:  # diagonal plus the farthest block only
+        mask = np.broadcast_to(np.eye(nb, dtype=np.uint8), (1, 2, nb, nb)).copy()
+        for i in range(nb):
+            mask[0, :, i, nb - 1 - i] = 1
+    rp, ci = _mask_to_csr(mask)
+    O = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, bs)
+    Ow, _ = oracle.attention(host["q"], host["k"], host["v"], bs, mask=mask)
+    check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, "bf16")
+
+
+@pytest.mark.parametrize("dtype,L,H,Hkv,d", [("bf16", 1024, 4, 2, 128), ("bf16", 640, 2, 2, 64),
+                                             ("fp32", 512, 2, 2, 64)])
+def test_dense_attention(dtype, L, H, Hkv, d):
+    w = synth.small_workload(dtype=dtype, L=L, H=H, H_kv=Hkv, d=d)
+    host, dev = _inputs(w)
+    O, lse = sdl.dense_attn(dev["q"], dev["k"], dev["v"], want_lse=True)
+    Ow, lw = oracle.attention(host["q"], host["k"], host["v"], 64)
+    check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, dtype)
+    assert np.abs(lse.cpu().numpy() - lw).max() <= TOL[dtype]["lse"]
+
+
+def test_strided_fused_qkv_layout():
+    """Q, K, V as views into one [B, L, H + 2*H_kv, d] buffer (fused projection)."""
+    w = synth.small_workload(L=512, H=4, H_kv=2, d=128)
+    host, dev = _inputs(w)
+    fused = torch.empty((1, 512, 8, 128), dtype=torch.bfloat16, device="cuda")
+    fused[:, :, 0:4] = dev["q"]
+    fused[:, :, 4:6] = dev["k"]
+    fused[:, :, 6:8] = dev["v"]
+    q, k, v = fused[:, :, 0:4], fused[:, :, 4:6], fused[:, :, 6:8]
+    o_big = torch.zeros((1, 512, 4, 256), dtype=torch.bfloat16, device="cuda")
+    o = o_big[..., 64:192]  # strided output
+    mask = _random_mask(1, 4, 8, 0.5, np.random.default_rng(1))
+    rp, ci = _mask_to_csr(mask)
+    sdl.sparse_attn(q, k, v, rp, ci, 64, out=o)
+    Ow, _ = oracle.attention(host["q"], host["k"], host["v"], 64, mask=mask)
+    check_close(bf16_to_f64(o).transpose(0, 2, 1, 3), Ow, "bf16")
+    assert torch.count_nonzero(o_big[..., :64]) == 0 and torch.count_nonzero(o_big[..., 192:]) == 0
+    P = sdl.block_scores(q, k, 64)
+    want = oracle.block_scores(host["q"], host["k"], 64)
+    assert np.abs(P.cpu().numpy() - want).max() / want.min() < 1e-4
+
+
+def test_bad_list_entry_is_reported_and_skipped():
+    w = synth.small_workload(L=256, H=1, H_kv=1, d=128)
+    _, dev = _inputs(w)
+    rp = torch.tensor([0, 2, 3, 4, 6], dtype=torch.int32, device="cuda")
+    ci = torch.tensor([0, 99, 1, 2, 3, 3], dtype=torch.int32, device="cuda")  # 99 out of range
+    sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64)
+    assert sdl.last_device_status() == sdl.SDL_ERR_BAD_MASK
+    assert sdl.last_device_status() == sdl.SDL_OK  # reading clears it
+
+
+def test_argument_errors_do_not_launch():
+    q = torch.zeros((1, 256, 2, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sdl.SdlError) as e:
+        sdl.dense_attn(q, q[:, :, :1], q[:, :, :1], block=96)
+    assert e.value.status == sdl.SDL_ERR_UNSUPPORTED
+    k3 = torch.zeros((1, 256, 3, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sdl.SdlError) as e:
+        sdl.dense_attn(q, k3, k3)  # 2 query heads over 3 KV heads
+    assert e.value.status == sdl.SDL_ERR_INVALID_ARG
+    P = torch.rand(1, 2, 4, 4, device="cuda")
+    with pytest.raises(sdl.SdlError) as e:
+        sdl.select_mask(P, 0.5, 64, 256, col_idx=torch.empty(3, dtype=torch.int32, device="cuda"))
+    assert e.value.status == sdl.SDL_ERR_CAPACITY

@@ -1,0 +1,104 @@
+"""GPU parity on the five workloads, through the anchor-step schedule.
+
+fp32-L512 and bf16-L2048: every checked step compared in full (scores, mask,
+all output rows).  The full-size bf16 workloads (8K, 16K GQA, 64K with
+128-token blocks): scores and mask in full at anchor steps, attention on
+sampled rows that always include the first and last query block and the
+longest kept list of every head, in the same launch configuration the
+benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.parity_util import (TOL, bf16_to_f64, check_close, check_csr, compare_masks,
+                               csr_to_mask, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+sdl = pytest.importorskip("block_sparse_attention_sdl_b200")
+from block_sparse_attention_sdl_b200.runtime import StepSparseAttention, anchor_of  # noqa: E402
+
+DT = {"bf16": torch.bfloat16, "fp32": torch.float32}
+
+
+def _layer(w):
+    return StepSparseAttention(w.B, w.H, w.H_kv, w.L, w.d, w.bs, w.sparsity, w.anchor_every,
+                               dtype=DT[w.dtype])
+
+
+def _check_anchor(att, w, host):
+    P_or = oracle.block_scores(host["q"], host["k"], w.bs)
+    P_gpu = att.scores.cpu().numpy().astype(np.float64)
+    assert (np.abs(P_gpu - P_or) / P_or).max() < 2e-5
+    want, tau, kept = oracle.select(P_or, w.sparsity)
+    rp, ci = att.row_ptr.cpu().numpy(), att.col_idx.cpu().numpy()
+    check_csr(rp, ci, w.B, w.H, w.nb, kept)
+    got = csr_to_mask(rp, ci, w.B, w.H, w.nb)
+    excused = compare_masks(got, want, P_or, tau)
+    return got, excused
+
+
+@pytest.mark.parametrize("name,steps", [("fp32-L512-H2-s50", [0, 1, 2, 3]),
+                                        ("bf16-L2048-H32-s80", [0, 1, 4, 6])])
+def test_schedule_full_parity(name, steps):
+    w = synth.WORKLOADS[name]
+    att = _layer(w)
+    csr_at_anchor = None
+    for step in range(max(steps) + 1):
+        dev = synth.device_inputs(w, step)
+        out = att(dev["q"], dev["k"], dev["v"], step)
+        assert att.mask_step == anchor_of(step, w.anchor_every)
+        if w.is_anchor(step):
+            csr_at_anchor = (att.row_ptr.clone(), att.col_idx.clone())
+        else:  # the mask is reused unchanged between anchors
+            assert torch.equal(att.row_ptr, csr_at_anchor[0])
+            assert torch.equal(att.col_idx, csr_at_anchor[1])
+        if step not in steps:
+            continue
+        host = synth.host_inputs(w, step)
+        if w.is_anchor(step):
+            mask, _ = _check_anchor(att, w, host)
+        else:
+            mask = csr_to_mask(att.row_ptr.cpu().numpy(), att.col_idx.cpu().numpy(), w.B, w.H,
+                               w.nb)
+        Ow, _ = oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=mask)
+        check_close(bf16_to_f64(out).transpose(0, 2, 1, 3), Ow, w.dtype)
+    assert sdl.last_device_status() == sdl.SDL_OK
+
+
+@pytest.mark.parametrize("name,step", [("bf16-L8192-H32-s90", 0), ("bf16-L8192-H32-s90", 64),
+                                       ("bf16-L16384-H28kv4-s90", 16),
+                                       ("bf16-L65536-H32-bs128-s95", 0)])
+def test_full_size_anchor_and_sampled_rows(name, step):
+    w = synth.WORKLOADS[name]
+    att = _layer(w)
+    dev = synth.device_inputs(w, step)
+    out, lse = att(dev["q"], dev["k"], dev["v"], step,
+                   lse=torch.empty((w.B, w.H, w.L), dtype=torch.float32, device="cuda"))
+    torch.cuda.synchronize()
+    host = synth.host_inputs(w, step)
+    mask, excused = _check_anchor(att, w, host)
+    print(f"{name} step {step}: {excused} near-threshold mask differences excused")
+    rows = sample_rows(w.B, w.H, w.L, w.bs, mask.sum(-1), n_blocks=4, rows_per_block=8)
+    Ow, lw = oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=mask, rows=rows)
+    got = bf16_to_f64(out)[rows[:, 0], rows[:, 2], rows[:, 1]]
+    check_close(got, Ow, "bf16")
+    lse_got = lse.cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    assert np.abs(lse_got - lw).max() <= TOL["bf16"]["lse"]
+    assert sdl.last_device_status() == sdl.SDL_OK
+
+
+def test_dense_full_size_sampled_rows():
+    w = synth.WORKLOADS["bf16-L8192-H32-s90"]
+    dev = synth.device_inputs(w, 5)
+    out = sdl.dense_attn(dev["q"], dev["k"], dev["v"])
+    torch.cuda.synchronize()
+    host = synth.host_inputs(w, 5)
+    rows = sample_rows(w.B, w.H, w.L, w.bs, np.ones((w.B, w.H, w.nb)), n_blocks=2,
+                       rows_per_block=4)
+    Ow, _ = oracle.attention(host["q"], host["k"], host["v"], w.bs, rows=rows)
+    got = bf16_to_f64(out)[rows[:, 0], rows[:, 2], rows[:, 1]]
+    check_close(got, Ow, "bf16")
