@@ -26,7 +26,8 @@ SDL_ERR_WORKSPACE, SDL_ERR_CUDA, SDL_ERR_TIMEOUT, SDL_ERR_BAD_MASK = 4, 5, 6, 7
 SDL_BF16, SDL_FP32 = 0, 1
 
 EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspace_bytes",
-           "sdl_block_scores", "sdl_select_mask", "sdl_sparse_attn", "sdl_dense_attn",
+           "sdl_block_scores", "sdl_select_mask", "sdl_select_mask_noalloc", "sdl_sparse_attn",
+           "sdl_dense_attn",
            "sdl_last_device_status", "sdl_last_cuda_error", "sdl_status_string")
 
 

@@ -103,6 +103,22 @@ sdl_status sdl_select_mask(const float* scores, const sdl_shape* shape, double s
                            uint8_t* mask_u8, void* workspace, size_t workspace_bytes,
                            void* stream);
 
+/* Allocation-free variant of sdl_select_mask (no counterpart in the paper; it
+ * exists for callers that cannot allocate device memory, such as code running
+ * inside a device-memory pool's own callbacks or a serving process that reserves
+ * all of its memory at start-up and forbids cudaMalloc afterwards).
+ * Same arguments and results as sdl_select_mask minus the workspace: the
+ * scratch is a fixed 2 MiB array inside libsdl (held by every GPU that loads the
+ * library until exit).  Problems needing more scratch than that
+ * (sdl_select_workspace_bytes > 2 MiB) return SDL_ERR_WORKSPACE without launching.
+ * The first call on each device looks up the array's device address; make it
+ * before any stream capture.  Nothing is allocated by any call.  All calls share
+ * the array: calls that may overlap on the GPU (other streams, other threads)
+ * race and must be serialized by the caller. */
+sdl_status sdl_select_mask_noalloc(const float* scores, const sdl_shape* shape, double sparsity,
+                                   int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                   uint8_t* mask_u8, void* stream);
+
 /* Block-sparse attention (every step), the fused kernel of the Step-dLLM
  * abstract: for token t of query block i of head h,
  *   O[b,t,h,:] = sum_u softmax_u(scale * q_t . k_u) v_u
