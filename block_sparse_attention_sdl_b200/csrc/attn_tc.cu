@@ -11,11 +11,12 @@
 //                             M=128, N=128, fp32 accumulator in TMEM;
 //                 O += P V    A = P (bf16) from TMEM, B = V from shared memory
 //                             (N-major), M=128, N=d.
-//   warps 2-5   softmax: one thread per query row (its TMEM lane), online
-//               softmax in the log2 domain with the running max raised only
-//               when it grows by more than 8 (a factor 256), O rescaled in
-//               TMEM only then; P written back as bf16 over its S columns and
-//               the row sum taken over those rounded weights.
+//   warps 2-9   softmax in two warpgroups: each thread one query row (its
+//               TMEM lane) and one 64-column half of the step; online softmax
+//               in the log2 domain with the running max raised only when it
+//               grows by more than 8 (a factor 256), O rescaled in TMEM only
+//               then; P written back as bf16 over its S columns and the row
+//               sum taken over those rounded weights.
 //               Epilogue: O / l rounded to bf16, LSE.
 //
 // With 64-token blocks a 128-row tile covers two query blocks; the kernel
@@ -40,10 +41,12 @@ constexpr int kBM = 128;        // query rows per CTA
 constexpr int kBN = 128;        // key rows per step
 constexpr int kStages = 2;      // K/V ring depth
 constexpr int kMaxSub = 1024;   // 64-token sub-blocks per sequence (L <= 65536)
-constexpr int kThreads = 192;   // 6 warps
+constexpr int kThreads = 352;   // 11 warps
+constexpr int kVWarp = 10;      // V producer
 constexpr int kBox = 64 * 128;  // bytes of one 64-row x 64-column bf16 box
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr int kPolyPer8 = 0;  // of every 8 weights, how many take exp2_poly (FMA pipe)
 
 template <int D>
 struct Layout {
@@ -63,11 +66,13 @@ struct Bars {
   uint64_t q;
   uint64_t kfull[kStages];
   uint64_t vfull[kStages];
-  uint64_t kvempty[kStages];
+  uint64_t kempty[kStages];  // K slot free: its S product completed
+  uint64_t vempty[kStages];  // V slot free: its PV product completed
   uint64_t s[2];
   uint64_t p[2];
   uint64_t o;
   uint64_t done;
+  uint64_t soft;  // barrier of the 256 softmax threads
 };
 
 __device__ __forceinline__ void raise_timeout(volatile int* abort_flag, int* status) {
@@ -75,7 +80,7 @@ __device__ __forceinline__ void raise_timeout(volatile int* abort_flag, int* sta
   atomicOr(status, kDevTimeout);
 }
 
-template <int D>
+template <int D, bool kLse>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                    const __grid_constant__ CUtensorMap tmv, AttnArgs a) {
@@ -89,6 +94,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t ent[kMaxSub];  // sub-block | keep bits << 16
   __shared__ uint32_t bmask[2][kMaxSub / 32];
   __shared__ int n_ent_sh;
+  __shared__ float sh_max[2][2][kBM];  // [step parity][group][row] tile maxima
+  __shared__ float sh_sum[2][2][kBM];  // [rounded, unrounded][group][row] row sums
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -154,14 +161,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < kStages; ++s) {
         mbar_init(&bars.kfull[s], 1);
         mbar_init(&bars.vfull[s], 1);
-        mbar_init(&bars.kvempty[s], 1);
+        mbar_init(&bars.kempty[s], 1);
+        mbar_init(&bars.vempty[s], 1);
       }
       for (int s = 0; s < 2; ++s) {
         mbar_init(&bars.s[s], 1);
-        mbar_init(&bars.p[s], 128);
+        mbar_init(&bars.p[s], 256);
       }
       mbar_init(&bars.o, 1);
       mbar_init(&bars.done, 1);
+      mbar_init(&bars.soft, 256);
       abort_sh = 0;
       fence_barrier_init();
     }
@@ -176,53 +185,54 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_ent = n_ent_sh;
   const int n_steps = (n_ent + 1) / 2;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------- producer
+  if (warp == 0 || warp == kVWarp) {
+    // --------------------------------------------------------- producers
+    // Warp 0 loads Q once and then the K sub-blocks of every step, warp
+    // kVWarp the V sub-blocks: two issuing threads, two independent rings
+    // (one thread's tensor-copy issue rate alone falls short of a step).
+    const bool isk = warp == 0;
+    uint64_t* full = isk ? bars.kfull : bars.vfull;
+    uint64_t* empty = isk ? bars.kempty : bars.vempty;
+    const CUtensorMap* tm = isk ? &tmk : &tmv;
+    uint8_t* ring = dsm + (isk ? Lay::kOffK : Lay::kOffV);
     if (lane == 0 && n_steps > 0) {
-      prefetch_tensormap(&tmq);
-      prefetch_tensormap(&tmk);
-      prefetch_tensormap(&tmv);
-      uint8_t* sq = dsm + Lay::kOffQ;
-      mbar_arrive_expect_tx(&bars.q, Lay::kQBytes);
-      for (int c = 0; c < Lay::kChunks; ++c)
-        for (int s = 0; s < 2; ++s)
-          tma_load_4d(sq + c * Lay::kChunkRowsQ + s * kBox, &tmq, &bars.q, c * 64, t0 + 64 * s, h,
-                      b);
-      int issued[kStages] = {0};
+      prefetch_tensormap(tm);
+      if (isk) {
+        prefetch_tensormap(&tmq);
+        uint8_t* sq = dsm + Lay::kOffQ;
+        mbar_arrive_expect_tx(&bars.q, Lay::kQBytes);
+        for (int c = 0; c < Lay::kChunks; ++c)
+          for (int s = 0; s < 2; ++s)
+            tma_load_4d(sq + c * Lay::kChunkRowsQ + s * kBox, &tmq, &bars.q, c * 64, t0 + 64 * s,
+                        h, b);
+      }
+      int done_steps = 0;
       for (int st = 0; st < n_steps; ++st) {
         const int stage = st % kStages;
-        if (st >= kStages) {
-          if (!mbar_wait(&bars.kvempty[stage], ((st / kStages) - 1) & 1, &abort_sh, a.status, kWaitLimitNs)) {
-            raise_timeout(&abort_sh, a.status);
-            break;
-          }
+        if (st >= kStages &&
+            !mbar_wait(&empty[stage], ((st / kStages) - 1) & 1, &abort_sh, a.status,
+                       kWaitLimitNs)) {
+          raise_timeout(&abort_sh, a.status);
+          break;
         }
         const uint32_t e0 = ent[2 * st];
         const uint32_t e1 = (2 * st + 1 < n_ent) ? ent[2 * st + 1] : e0;
-        const int sub[2] = {(int)(e0 & 0xFFFFu), (int)(e1 & 0xFFFFu)};
-        uint8_t* sk = dsm + Lay::kOffK + stage * Lay::kKVBytes;
-        uint8_t* sv = dsm + Lay::kOffV + stage * Lay::kKVBytes;
-        mbar_arrive_expect_tx(&bars.kfull[stage], Lay::kKVBytes);
+        const int sub0 = (int)(e0 & 0xFFFFu), sub1 = (int)(e1 & 0xFFFFu);
+        uint8_t* dst = ring + stage * Lay::kKVBytes;
+        mbar_arrive_expect_tx(&full[stage], Lay::kKVBytes);
         for (int c = 0; c < Lay::kChunks; ++c)
           for (int s = 0; s < 2; ++s)
-            tma_load_4d(sk + c * Lay::kChunkRowsKV + s * kBox, &tmk, &bars.kfull[stage], c * 64,
-                        sub[s] * kSubBlock, kh, b);
-        mbar_arrive_expect_tx(&bars.vfull[stage], Lay::kKVBytes);
-        for (int c = 0; c < Lay::kChunks; ++c)
-          for (int s = 0; s < 2; ++s)
-            tma_load_4d(sv + c * Lay::kChunkRowsKV + s * kBox, &tmv, &bars.vfull[stage], c * 64,
-                        sub[s] * kSubBlock, kh, b);
-        ++issued[stage];
+            tma_load_4d(dst + c * Lay::kChunkRowsKV + s * kBox, tm, &full[stage], c * 64,
+                        (s ? sub1 : sub0) * kSubBlock, kh, b);
+        done_steps = st + 1;
       }
       // Drain: every copy this thread issued has landed before the CTA exits.
       volatile int no_abort = 0;
-      if (!mbar_wait(&bars.q, 0, &no_abort, nullptr, kWaitLimitNs)) atomicOr(a.status, kDevTimeout);
-      for (int s = 0; s < kStages; ++s) {
-        if (issued[s] == 0) continue;
-        const uint32_t par = (issued[s] - 1) & 1;
-        if (!mbar_wait(&bars.kfull[s], par, &no_abort, nullptr, kWaitLimitNs)) atomicOr(a.status, kDevTimeout);
-        if (!mbar_wait(&bars.vfull[s], par, &no_abort, nullptr, kWaitLimitNs)) atomicOr(a.status, kDevTimeout);
-      }
+      if (isk && !mbar_wait(&bars.q, 0, &no_abort, nullptr, kWaitLimitNs))
+        atomicOr(a.status, kDevTimeout);
+      for (int st = (done_steps > kStages ? done_steps - kStages : 0); st < done_steps; ++st)
+        if (!mbar_wait(&full[st % kStages], (st / kStages) & 1, &no_abort, nullptr, kWaitLimitNs))
+          atomicOr(a.status, kDevTimeout);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA
@@ -247,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = smem_desc_sw128(kb + (kk / 4) * Lay::kChunkRowsKV + off, 16, 1024);
           mma_bf16_ss(dcol, ad, bd, idS, kk > 0 ? 1u : 0u);
         }
+        tc_commit(&bars.kempty[stage]);
         tc_commit(&bars.s[st & 1]);
         return true;
       };
@@ -266,9 +277,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, Lay::kChunkRowsKV, 1024);
-          mma_bf16_ts(tmem + kColO, pcol + kk * 8, bd, idPV, (st > 0 || kk > 0) ? 1u : 0u);
+          // P elements [16 kk, 16 kk + 16): columns 64 (kk / 4) + 8 (kk % 4)
+          mma_bf16_ts(tmem + kColO, pcol + 64 * (kk / 4) + 8 * (kk % 4), bd, idPV,
+                      (st > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&bars.kvempty[stage]);
+        tc_commit(&bars.vempty[stage]);
         tc_commit(&bars.o);
       }
       if (!ok) raise_timeout(&abort_sh, a.status);
@@ -279,14 +292,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // --------------------------------------------------------- softmax
+    // Two warpgroups: group g owns key columns [64 g, 64 g + 64) of each S
+    // row (key sub-block g of the step) and columns [64 g, 64 g + 64) of O.
+    // The two threads of a row swap their tile maxima through shared memory
+    // once per step.  Each group writes its half of P (bf16 pairs) over the
+    // first 32 of its own 64 S columns, so neither group overwrites S the
+    // other may still read.
+    const int grp = (warp - 2) / 4;
     const int quad = warp & 3;  // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;
     const int half = row >> 6;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
     const float sl2 = a.scale_log2;
     float m = -INFINITY;  // running max (log2 units) used as the exponent reference
-    float l = 0.f;        // sum of the bf16-rounded weights (normalises O)
-    float lx = 0.f;       // sum of the unrounded weights (for the LSE)
+    float l = 0.f;        // this half-row's sum of the bf16-rounded weights
+    float lx = 0.f;       // this half-row's sum of the unrounded weights (LSE only)
+    uint32_t soft_uses = 0;
     bool ok = true;
     for (int st = 0; st < n_steps; ++st) {
       const int buf = st & 1;
@@ -298,102 +319,113 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t e0 = ent[2 * st];
       const uint32_t e1 = (2 * st + 1 < n_ent) ? ent[2 * st + 1] : (e0 & 0xFFFFu);
-      const bool v0 = (e0 >> (16 + half)) & 1u;
-      const bool v1 = (e1 >> (16 + half)) & 1u;
+      const bool keep = ((grp ? e1 : e0) >> (16 + half)) & 1u;
       const uint32_t scol = trow + (buf ? kColS1 : kColS0);
-      uint32_t sr[4][32];
-      tmem_ld32(scol + 0, sr[0]);
-      tmem_ld32(scol + 32, sr[1]);
-      tmem_ld32(scol + 64, sr[2]);
-      tmem_ld32(scol + 96, sr[3]);
-      tmem_wait_ld();
+      float sv[64];
+      {
+        uint32_t r[64];
+        tmem_ld32(scol + 64 * grp, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(scol + 64 * grp + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 64; ++x) sv[x] = keep ? __uint_as_float(r[x]) * sl2 : -INFINITY;
+      }
       float mt = -INFINITY;
-      if (v0) {
 #pragma unroll
-        for (int x = 0; x < 32; ++x) mt = fmaxf(mt, fmaxf(__uint_as_float(sr[0][x]), __uint_as_float(sr[1][x])));
-      }
-      if (v1) {
-#pragma unroll
-        for (int x = 0; x < 32; ++x) mt = fmaxf(mt, fmaxf(__uint_as_float(sr[2][x]), __uint_as_float(sr[3][x])));
-      }
-      mt *= sl2;
+      for (int x = 0; x < 64; x += 2) mt = fmaxf(mt, fmaxf(sv[x], sv[x + 1]));
+      sh_max[st & 1][grp][row] = mt;
+      if (!(ok = group_sync(&bars.soft, soft_uses, &abort_sh, a.status, kWaitLimitNs))) break;
+      mt = fmaxf(mt, sh_max[st & 1][grp ^ 1][row]);
       const bool raise = mt > m + 8.0f;
-      if (st > 0) {
-        ok = mbar_wait(&bars.o, (st - 1) & 1, &abort_sh, a.status, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // tcgen05.ld/st are warp-collective: the warp rescales together, alpha = 1
-        // on rows whose reference max stays.
-        if (__any_sync(0xffffffffu, raise)) {
+      if (__any_sync(0xffffffffu, raise)) {
+        if (st > 0) {
+          // O must hold every product issued so far before it is rescaled;
+          // PV(st-2) is complete (S(st) was committed after it), PV(st-1) may
+          // not be, so this wait is unambiguous.
+          ok = mbar_wait(&bars.o, (st - 1) & 1, &abort_sh, a.status, kWaitLimitNs);
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           const float alpha = raise ? ex2_approx(m - mt) : 1.0f;
           l *= alpha;
           lx *= alpha;
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
             uint32_t ov[32];
-            tmem_ld32(trow + kColO + c * 32, ov);
+            const uint32_t oc = trow + kColO + (D / 2) * grp + c * 32;
+            tmem_ld32(oc, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
-            tmem_st32(trow + kColO + c * 32, ov);
+            tmem_st32(oc, ov);
           }
+          tmem_wait_st();
         }
+        if (raise) m = mt;
       }
-      if (raise) m = mt;
-      // P = exp2(S * scale * log2e - m) on kept quadrants, 0 elsewhere; bf16 pairs.
+      // P = exp2(S * scale * log2e - m) on a kept half, 0 otherwise (a kept
+      // half always has a finite reference here: its own maximum raised it)
+      if (keep) {
+#pragma unroll
+        for (int x = 0; x < 64; ++x)
+          sv[x] = (x & 7) < 8 - kPolyPer8 ? ex2_approx(sv[x] - m) : exp2_poly(sv[x] - m);
+      } else {
+#pragma unroll
+        for (int x = 0; x < 64; ++x) sv[x] = 0.f;
+      }
+      // bf16 pairs of P over the S columns; l sums the rounded weights
       float rs = 0.f, rx = 0.f;
-      uint32_t pw[2][32];
+      uint32_t pw[32];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const bool keep = g < 2 ? v0 : v1;
-#pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float p0 = 0.f, p1 = 0.f;
-          if (keep) {
-            p0 = ex2_approx(fmaf(__uint_as_float(sr[g][x]), sl2, -m));
-            p1 = ex2_approx(fmaf(__uint_as_float(sr[g][x + 1]), sl2, -m));
-          }
-          // l sums the bf16-rounded weights that the PV product uses, so the
-          // normalisation matches the numerator exactly
-          __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
-          const float2 pr = __bfloat1622float2(pk);
-          rs += pr.x + pr.y;
-          rx += p0 + p1;
-          pw[g >> 1][(g & 1) * 16 + x / 2] = *reinterpret_cast<uint32_t*>(&pk);
-        }
+      for (int x = 0; x < 64; x += 2) {
+        __nv_bfloat162 pk = __floats2bfloat162_rn(sv[x], sv[x + 1]);
+        const uint32_t u = *reinterpret_cast<uint32_t*>(&pk);
+        rs += __uint_as_float(u << 16) + __uint_as_float(u & 0xFFFF0000u);
+        if constexpr (kLse) rx += sv[x] + sv[x + 1];
+        pw[x / 2] = u;
       }
       l += rs;
       lx += rx;
-      tmem_st32(scol + 0, pw[0]);
-      tmem_st32(scol + 32, pw[1]);
+      // P of this half goes over this half's own S columns [64 grp, 64 grp + 32)
+      // (never over columns the other group may still read)
+      tmem_st32(scol + 64 * grp, pw);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars.p[buf]);
     }
     // ------------------------------------------------------- epilogue
     const int t = t0 + row;
+    if (ok && n_steps > 0) {
+      // full-row sums from the two halves
+      sh_sum[0][grp][row] = l;
+      sh_sum[1][grp][row] = lx;
+      ok = group_sync(&bars.soft, soft_uses, &abort_sh, a.status, kWaitLimitNs);
+      l += sh_sum[0][grp ^ 1][row];
+      lx += sh_sum[1][grp ^ 1][row];
+    }
     if (!ok) {
       raise_timeout(&abort_sh, a.status);
     } else if (n_steps == 0) {
       if (t < a.L) {
         __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(a.o) + b * a.os[0] +
-                            (int64_t)t * a.os[1] + h * a.os[2];
-        for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(op + c) = make_uint4(0, 0, 0, 0);
-        if (a.lse) a.lse[((int64_t)b * a.H + h) * a.L + t] = -INFINITY;
+                            (int64_t)t * a.os[1] + h * a.os[2] + (D / 2) * grp;
+        for (int c = 0; c < D / 2; c += 8) *reinterpret_cast<uint4*>(op + c) = make_uint4(0, 0, 0, 0);
+        if (a.lse && grp == 0) a.lse[((int64_t)b * a.H + h) * a.L + t] = -INFINITY;
       }
     } else if (__all_sync(0xffffffffu,
-                          mbar_wait(&bars.o, (n_steps - 1) & 1, &abort_sh, a.status, kWaitLimitNs))) {
+                          mbar_wait(&bars.done, 0, &abort_sh, a.status, kWaitLimitNs))) {
+      // (bars.done completes once, after every MMA of the tile: with the lazy
+      //  waits above, the last two products may still be running here)
       tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
       __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(a.o) + b * a.os[0] +
-                          (int64_t)t * a.os[1] + h * a.os[2];
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+                          (int64_t)t * a.os[1] + h * a.os[2] + (D / 2) * grp;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t ov[32];
-        tmem_ld32(trow + kColO + c * 32, ov);
+        tmem_ld32(trow + kColO + (D / 2) * grp + c * 32, ov);
         tmem_wait_ld();
         if (t < a.L) {
           uint32_t pk[16];
@@ -409,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
         }
       }
-      if (a.lse && t < a.L)
+      if (a.lse && grp == 0 && t < a.L)
         a.lse[((int64_t)b * a.H + h) * a.L + t] =
             lx > 0.f ? (m + log2f(lx)) * 0.69314718055994531f : -INFINITY;
     } else {
@@ -428,23 +460,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+template <int D, bool kLse>
+static cudaError_t launch_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
+                             const CUtensorMap* tv, cudaStream_t st) {
+  using Lay = Layout<D>;
+  dim3 grid((a.L + kBM - 1) / kBM, a.H, a.B);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, kLse>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmem);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<D, kLse><<<grid, kThreads, Lay::kSmem, st>>>(*tq, *tk, *tv, a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, cudaStream_t st) {
-  dim3 grid((a.L + kBM - 1) / kBM, a.H, a.B);
-  if (a.d == 128) {
-    using Lay = Layout<128>;
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<128>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmem);
-    if (e != cudaSuccess) return e;
-    attn_tc_kernel<128><<<grid, kThreads, Lay::kSmem, st>>>(*tq, *tk, *tv, a);
-  } else {
-    using Lay = Layout<64>;
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<64>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmem);
-    if (e != cudaSuccess) return e;
-    attn_tc_kernel<64><<<grid, kThreads, Lay::kSmem, st>>>(*tq, *tk, *tv, a);
-  }
-  return cudaGetLastError();
+  if (a.d == 128)
+    return a.lse ? launch_tc<128, true>(a, tq, tk, tv, st) : launch_tc<128, false>(a, tq, tk, tv, st);
+  return a.lse ? launch_tc<64, true>(a, tq, tk, tv, st) : launch_tc<64, false>(a, tq, tk, tv, st);
 }
 
 }  // namespace sdl

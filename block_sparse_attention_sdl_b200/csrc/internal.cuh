@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/sdl.h"
+#include "sdl.h"
 
 namespace sdl {
 
@@ -45,6 +45,8 @@ cudaError_t launch_select(const float* scores, int B, int H, int nb, int64_t kb,
                           int32_t* col_idx, uint8_t* mask, void* ws, cudaStream_t st);
 size_t select_workspace_bytes(int B, int H, int nb);
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
+                           const CUtensorMap* tv, cudaStream_t st);
+cudaError_t launch_attn_km(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t st);
 

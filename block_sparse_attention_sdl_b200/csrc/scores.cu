@@ -97,9 +97,9 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolTensor tq, PoolT
   }
 }
 
-constexpr int kTI = 32;  // query blocks per CTA
+constexpr int kTI = 16;  // query blocks per CTA (4 per warp)
 constexpr int kTJ = 64;  // key blocks per shared-memory tile
-constexpr int kScoreThreads = 256;
+constexpr int kScoreThreads = 128;
 
 // grid: (ceil(nb / kTI), H, B).  Dynamic shared memory:
 //   qs [kTI][d+4], ks [kTJ][d+4], z [kTI][nb] floats.

@@ -23,6 +23,17 @@ __constant__ int kShift[kPasses] = {21, 10, 0};
 __constant__ int kWidth[kPasses] = {11, 11, 10};
 constexpr int kThreads = 256;
 
+// Shared-memory histogram increment aggregated over the lanes of a warp that
+// hit the same bin (block scores of one workload often share their top bits,
+// which would otherwise serialise the atomics on one address).
+__device__ __forceinline__ void hist_add(int* sh, int bin, bool active) {
+  const unsigned act = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const unsigned peers = __match_any_sync(act, bin);
+  const int leader = __ffs(peers) - 1;
+  if ((int)(threadIdx.x % 32) == leader) atomicAdd(&sh[bin], __popc(peers));
+}
+
 struct SelWs {
   int* hist;      // [kPasses][B][kBins]
   int* gt;        // [R] off-diagonal scores above the threshold, per row
@@ -127,29 +138,43 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(const float* __restrict_
   const float* base = scores + (int64_t)b * per_b;
   // 16-byte loads only when every batch element's slice starts 16-byte aligned
   const int64_t n4 = (per_b % 4 == 0) ? per_b / 4 : 0;
-  for (int64_t x = (int64_t)blockIdx.x * kThreads + threadIdx.x; x < n4;
+  // whole warps iterate together so the lane-aggregated increments stay convergent
+  const int64_t n4_round = (n4 + kThreads - 1) / kThreads * kThreads;
+  for (int64_t x = (int64_t)blockIdx.x * kThreads + threadIdx.x; x < n4_round;
        x += (int64_t)gridDim.x * kThreads) {
-    float4 v = __ldg(reinterpret_cast<const float4*>(base) + x);
-    float vals[4] = {v.x, v.y, v.z, v.w};
+    float vals[4] = {0.f, 0.f, 0.f, 0.f};
+    const bool in = x < n4;
+    if (in) {
+      float4 v = __ldg(reinterpret_cast<const float4*>(base) + x);
+      vals[0] = v.x;
+      vals[1] = v.y;
+      vals[2] = v.z;
+      vals[3] = v.w;
+    }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      int64_t e = 4 * x + u;
-      int j = (int)(e % nb);
-      int i = (int)((e / nb) % nb);
-      if (i == j) continue;
-      uint32_t key = __float_as_uint(vals[u]);
-      if (hs < 32 && (key >> hs) != want) continue;
-      atomicAdd(&sh[(key >> shift) & dmask], 1);
+      const int64_t e = 4 * x + u;
+      const int j = (int)(e % nb);
+      const int i = (int)((e / nb) % nb);
+      const uint32_t key = __float_as_uint(vals[u]);
+      const bool take = in && i != j && (hs >= 32 || (key >> hs) == want);
+      hist_add(sh, (int)((key >> shift) & dmask), take);
     }
   }
-  for (int64_t e = n4 * 4 + (int64_t)blockIdx.x * kThreads + threadIdx.x; e < per_b;
+  const int64_t tail0 = n4 * 4;
+  const int64_t tail_round = tail0 + (per_b - tail0 + kThreads - 1) / kThreads * kThreads;
+  for (int64_t e = tail0 + (int64_t)blockIdx.x * kThreads + threadIdx.x; e < tail_round;
        e += (int64_t)gridDim.x * kThreads) {
-    int j = (int)(e % nb);
-    int i = (int)((e / nb) % nb);
-    if (i == j) continue;
-    uint32_t key = __float_as_uint(base[e]);
-    if (hs < 32 && (key >> hs) != want) continue;
-    atomicAdd(&sh[(key >> shift) & dmask], 1);
+    const bool in = e < per_b;
+    uint32_t key = 0;
+    int i = 0, j = 0;
+    if (in) {
+      j = (int)(e % nb);
+      i = (int)((e / nb) % nb);
+      key = __float_as_uint(base[e]);
+    }
+    const bool take = in && i != j && (hs >= 32 || (key >> hs) == want);
+    hist_add(sh, (int)((key >> shift) & dmask), take);
   }
   __syncthreads();
   int* gh = ws.hist + ((size_t)pass * B + b) * kBins;
@@ -339,9 +364,9 @@ cudaError_t launch_select(const float* scores, int B, int H, int nb, int64_t kb,
   const size_t nh = (size_t)kPasses * B * kBins;
   zero_kernel<<<(unsigned)((nh + 255) / 256), 256, 0, st>>>(ws.hist, nh);
   const int64_t per_b = (int64_t)H * nb * nb;
-  int chunks = (int)((per_b / 4 + kThreads * 8 - 1) / (kThreads * 8));
+  int chunks = (int)((per_b / 4 + kThreads - 1) / kThreads);
   if (chunks < 1) chunks = 1;
-  if (chunks > 148 * 8) chunks = 148 * 8;
+  if (chunks > 148 * 4) chunks = 148 * 4;
   for (int p = 0; p < kPasses; ++p)
     hist_kernel<<<dim3(chunks, B), kThreads, 0, st>>>(scores, B, H, nb, kfree, p, ws);
   int rchunks = (H * nb + (kThreads / 32) - 1) / (kThreads / 32);
