@@ -46,7 +46,7 @@ constexpr int kVWarp = 10;      // V producer
 constexpr int kBox = 64 * 128;  // bytes of one 64-row x 64-column bf16 box
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
-constexpr int kPolyPer8 = 0;  // of every 8 weights, how many take exp2_poly (FMA pipe)
+constexpr int kPolyPer8 = 2;  // of every 8 weights, how many take exp2_poly (FMA pipe)
 
 template <int D>
 struct Layout {
@@ -166,11 +166,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int s = 0; s < 2; ++s) {
         mbar_init(&bars.s[s], 1);
-        mbar_init(&bars.p[s], 256);
+        mbar_init(&bars.p[s], 8);  // one elected arrival per softmax warp
       }
       mbar_init(&bars.o, 1);
       mbar_init(&bars.done, 1);
-      mbar_init(&bars.soft, 256);
+      mbar_init(&bars.soft, 8);  // the 8 softmax warps
       abort_sh = 0;
       fence_barrier_init();
     }
@@ -369,8 +369,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // half always has a finite reference here: its own maximum raised it)
       if (keep) {
 #pragma unroll
-        for (int x = 0; x < 64; ++x)
-          sv[x] = (x & 7) < 8 - kPolyPer8 ? ex2_approx(sv[x] - m) : exp2_poly(sv[x] - m);
+        for (int x = 0; x < 64; x += 2) {
+          if ((x & 7) < 8 - kPolyPer8) {
+            sv[x] = ex2_approx(sv[x] - m);
+            sv[x + 1] = ex2_approx(sv[x + 1] - m);
+          } else {
+            const float2 e = exp2_poly2(sv[x] - m, sv[x + 1] - m);
+            sv[x] = e.x;
+            sv[x + 1] = e.y;
+          }
+        }
       } else {
 #pragma unroll
         for (int x = 0; x < 64; ++x) sv[x] = 0.f;
@@ -393,7 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st32(scol + 64 * grp, pw);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars.p[buf]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.p[buf]);
     }
     // ------------------------------------------------------- epilogue
     const int t = t0 + row;

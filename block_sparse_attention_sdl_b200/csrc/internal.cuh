@@ -46,8 +46,6 @@ cudaError_t launch_select(const float* scores, int B, int H, int nb, int64_t kb,
 size_t select_workspace_bytes(int B, int H, int nb);
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, cudaStream_t st);
-cudaError_t launch_attn_km(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
-                           const CUtensorMap* tv, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t st);
 
 }  // namespace sdl

@@ -272,18 +272,62 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 
 
-// Barrier among the threads of a group, built on an mbarrier initialised with
-// the group size: every thread arrives once per use and waits (bounded) for
-// the phase of that use.  `uses` counts the group's uses (identical in every
-// member).  tcgen05 fences order TMEM accesses across the barrier.
+// Barrier among the warps of a group, built on an mbarrier initialised with
+// the number of warps: every warp arrives once per use (one elected lane,
+// after the warp converges) and all threads wait (bounded) for the phase of
+// that use.  `uses` counts the group's uses (identical in every member).
+// tcgen05 fences order TMEM accesses across the barrier.
 __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& uses, volatile int* abort_flag,
                                            const volatile int* gstatus, uint64_t limit_ns) {
   tc_fence_before();
-  mbar_arrive(bar);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
   const bool ok = mbar_wait(bar, uses & 1u, abort_flag, gstatus, limit_ns);
   ++uses;
   tc_fence_after();
   return ok;
+}
+
+// Packed pairs of fp32 (Blackwell f32x2 arithmetic: one instruction per pair).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack2(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// exp2_poly on a pair, with the pair arithmetic packed (see exp2_poly).
+__device__ __forceinline__ float2 exp2_poly2(float x0, float x1) {
+  const uint64_t x = pack2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t C = pack2(12582912.0f, 12582912.0f);
+  const uint64_t t = add2(x, C);
+  const uint64_t f = sub2(x, sub2(t, C));
+  uint64_t p = fma2(f, pack2(0x1.c34958p-5f, 0x1.c34958p-5f), pack2(0x1.f0da64p-3f, 0x1.f0da64p-3f));
+  p = fma2(p, f, pack2(0x1.62f51ap-1f, 0x1.62f51ap-1f));
+  p = fma2(p, f, pack2(0x1.fff6b0p-1f, 0x1.fff6b0p-1f));
+  const float2 tp = unpack2(t), pp = unpack2(p);
+  const int j0 = __float_as_int(tp.x) - 0x4B400000, j1 = __float_as_int(tp.y) - 0x4B400000;
+  return make_float2(__int_as_float(__float_as_int(pp.x) + (j0 << 23)),
+                     __int_as_float(__float_as_int(pp.y) + (j1 << 23)));
 }
 
 }  // namespace sdl
