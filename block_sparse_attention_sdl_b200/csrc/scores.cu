@@ -4,9 +4,10 @@
 //
 // Two kernels:
 //   pool_kernel   reads Q and K once (16-byte vector loads, coalesced along the
-//                 contiguous (h, d) plane of each token) and writes fp32 block
-//                 means Qbar [B,H,nb,d] and Kbar [B,H_kv,nb,d].  HBM-bound.
-//   score_kernel  per (b, h, 32 query blocks): fp32 FFMA products against all
+//                 contiguous (h, d) plane of each token, one warp per block and
+//                 256-element chunk) and writes fp32 block means Qbar
+//                 [B,H,nb,d] and Kbar [B,H_kv,nb,d].  HBM-bound.
+//   score_kernel  per (b, h, 16 query blocks): fp32 FFMA products against all
 //                 Kbar rows of the KV head, then the row softmax in shared memory.
 #include <cuda_bf16.h>
 #include <math.h>
@@ -17,8 +18,7 @@ namespace sdl {
 namespace {
 
 constexpr int kPoolThreads = 256;
-constexpr int kPoolCols = 64;                          // threads along the (h, d) plane
-constexpr int kPoolGroups = kPoolThreads / kPoolCols;  // token groups
+constexpr int kLaneElems = 16;  // bytes per lane per token (one 16-byte load)
 
 template <typename T>
 struct Vec;
@@ -50,50 +50,49 @@ struct PoolTensor {
   const void* x;
   float* out;
   int Hx;
+  int chunks;  // 32-lane chunks of the (h, d) plane
   int64_t s0, s1, s2;
 };
 
+// One warp per work item (tensor, b, block i, chunk of 32 lanes x 16 bytes of
+// the contiguous (h, d) plane): each lane sums its elements over the block's
+// tokens with independent 16-byte loads, then writes the means.  Items of Q
+// come first, then those of K.
 template <typename T>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolTensor tq, PoolTensor tk, int L,
-                                                            int d, int bs) {
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolTensor tq, PoolTensor tk, int B,
+                                                            int L, int d, int bs) {
   constexpr int V = Vec<T>::N;
-  const PoolTensor& tx = (blockIdx.z & 1) ? tk : tq;
-  const int b = blockIdx.z >> 1;
-  const int i = blockIdx.y;
   const int nb = L / bs;
-  const int col = threadIdx.x % kPoolCols;
-  const int grp = threadIdx.x / kPoolCols;
-  const int e = (blockIdx.x * kPoolCols + col) * V;  // element of the (h, d) plane
-  const bool active = e < tx.Hx * d;
-  float acc[V];
-#pragma unroll
-  for (int v = 0; v < V; ++v) acc[v] = 0.f;
-  if (active) {
+  const int64_t items_q = (int64_t)B * nb * tq.chunks;
+  const int64_t items = items_q + (int64_t)B * nb * tk.chunks;
+  const int lane = threadIdx.x % 32;
+  for (int64_t it = ((int64_t)blockIdx.x * kPoolThreads + threadIdx.x) / 32; it < items;
+       it += (int64_t)gridDim.x * (kPoolThreads / 32)) {
+    const bool isq = it < items_q;
+    const PoolTensor& tx = isq ? tq : tk;
+    const int64_t r = isq ? it : it - items_q;
+    const int chunk = (int)(r % tx.chunks);
+    const int i = (int)((r / tx.chunks) % nb);
+    const int b = (int)(r / ((int64_t)tx.chunks * nb));
+    const int e = (chunk * 32 + lane) * V;  // element of the (h, d) plane
+    if (e >= tx.Hx * d) continue;
     const int h = e / d, c = e % d;
-    const T* base = reinterpret_cast<const T*>(tx.x) + b * tx.s0 + h * tx.s2 + c;
-    const int per = bs / kPoolGroups;
-    const int t0 = i * bs + grp * per;
-#pragma unroll 8
-    for (int t = 0; t < per; ++t) {
-      uint4 u = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)(t0 + t) * tx.s1));
+    const T* base = reinterpret_cast<const T*>(tx.x) + b * tx.s0 + h * tx.s2 + c +
+                    (int64_t)i * bs * tx.s1;
+    float acc[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) acc[v] = 0.f;
+#pragma unroll 16
+    for (int t = 0; t < bs; ++t) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)t * tx.s1));
       Vec<T>::add(acc, u);
     }
-  }
-  __shared__ float red[kPoolGroups][kPoolCols][V + 1];
-#pragma unroll
-  for (int v = 0; v < V; ++v) red[grp][col][v] = acc[v];
-  __syncthreads();
-  if (grp == 0 && active) {
-    const int h = e / d, c = e % d;
     const float inv = 1.0f / (float)bs;
     float* dst = tx.out + (((int64_t)b * tx.Hx + h) * nb + i) * d + c;
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-      float s = 0.f;
-#pragma unroll
-      for (int g = 0; g < kPoolGroups; ++g) s += red[g][col][v];
-      dst[v] = s * inv;
-    }
+    for (int v = 0; v < V; v += 4)
+      *reinterpret_cast<float4*>(dst + v) =
+          make_float4(acc[v] * inv, acc[v + 1] * inv, acc[v + 2] * inv, acc[v + 3] * inv);
   }
 }
 
@@ -186,16 +185,21 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const float* __res
 cudaError_t launch_pool(const void* q, const void* k, const sdl_shape& s, float* qbar,
                         float* kbar, cudaStream_t st) {
   const int nb = s.L / s.block;
-  PoolTensor tq{q, qbar, s.H, s.q_strides[0], s.q_strides[1], s.q_strides[2]};
-  PoolTensor tk{k, kbar, s.H_kv, s.k_strides[0], s.k_strides[1], s.k_strides[2]};
   const int V = s.dtype == SDL_BF16 ? 8 : 4;
-  const int chunk = kPoolCols * V;
-  const int chunks = (s.H * s.d + chunk - 1) / chunk;  // H >= H_kv
-  dim3 grid(chunks, nb, s.B * 2);
+  const int per_warp = 32 * V;  // elements of the (h, d) plane per work item
+  PoolTensor tq{q, qbar, s.H, (s.H * s.d + per_warp - 1) / per_warp, s.q_strides[0],
+                s.q_strides[1], s.q_strides[2]};
+  PoolTensor tk{k, kbar, s.H_kv, (s.H_kv * s.d + per_warp - 1) / per_warp, s.k_strides[0],
+                s.k_strides[1], s.k_strides[2]};
+  const int64_t items = (int64_t)s.B * nb * (tq.chunks + tk.chunks);
+  const int64_t warps_per_cta = kPoolThreads / 32;
+  int64_t grid = (items + warps_per_cta - 1) / warps_per_cta;
+  if (grid > 148 * 16) grid = 148 * 16;  // beyond that, warps loop over items
   if (s.dtype == SDL_BF16)
-    pool_kernel<__nv_bfloat16><<<grid, kPoolThreads, 0, st>>>(tq, tk, s.L, s.d, s.block);
+    pool_kernel<__nv_bfloat16><<<(unsigned)grid, kPoolThreads, 0, st>>>(tq, tk, s.B, s.L, s.d,
+                                                                        s.block);
   else
-    pool_kernel<float><<<grid, kPoolThreads, 0, st>>>(tq, tk, s.L, s.d, s.block);
+    pool_kernel<float><<<(unsigned)grid, kPoolThreads, 0, st>>>(tq, tk, s.B, s.L, s.d, s.block);
   return cudaGetLastError();
 }
 
