@@ -14,7 +14,7 @@ import torch
 import oracle
 import synth
 from tests.parity_util import (TOL, bf16_to_f64, check_close, check_csr, compare_masks,
-                               csr_to_mask)
+                               csr_to_mask, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -178,6 +178,79 @@ def test_sparse_attention_edge_masks(kind, bs):
     O = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, bs)
     Ow, _ = oracle.attention(host["q"], host["k"], host["v"], bs, mask=mask)
     check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, "bf16")
+
+
+@pytest.mark.parametrize("bs", [64, 128])
+def test_sparse_attention_empty_rows(bs):
+    """A caller's mask may leave rows empty: those rows are zero with LSE -inf.
+
+    Covers a 128-row tile with both query blocks empty, one with only one,
+    and empty tiles between non-empty ones in a CTA's schedule.
+    """
+    w = synth.small_workload(L=1024, H=4, H_kv=2, d=128, bs=bs)
+    host, dev = _inputs(w)
+    nb = 1024 // bs
+    rng = np.random.default_rng(7 + bs)
+    mask = (rng.random((1, 4, nb, nb)) < 0.3).astype(np.uint8)
+    mask[0, 0, :, :] = 0  # a whole head empty
+    mask[0, 1, 0:2, :] = 0  # the first tile of head 1 (both 64-token halves at bs 64)
+    mask[0, 2, 3, :] = 0  # one row only
+    mask[0, 3, nb - 1, :] = 0  # the last row
+    rp, ci = _mask_to_csr(mask)
+    O, lse = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, bs, want_lse=True)
+    assert sdl.last_device_status() == sdl.SDL_OK
+    Ow, lw = oracle.attention(host["q"], host["k"], host["v"], bs, mask=mask)
+    check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, "bf16")
+    lg = lse.cpu().numpy()
+    assert np.array_equal(np.isinf(lg), np.isinf(lw))
+    fin = np.isfinite(lw)
+    assert np.abs(lg[fin] - lw[fin]).max() <= TOL["bf16"]["lse"]
+
+
+@pytest.mark.parametrize("bs,density", [(64, 0.15), (128, 0.3)])
+def test_sparse_attention_many_tiles_per_cta(bs, density):
+    """More 128-row tiles than SMs: each persistent CTA walks several tiles,
+    reusing both list / Q / O slots; checked on sampled rows of every head."""
+    w = synth.Workload("t", "bf16", 2, 12, 4, 4096, 128, bs, 0.5, 1, 1, 0.02,
+                       ("uniform", 0.3, 4.0), 1)
+    host, dev = _inputs(w)
+    nb = 4096 // bs
+    rng = np.random.default_rng(11)
+    mask = _random_mask(2, 12, nb, density, rng)
+    rp, ci = _mask_to_csr(mask)
+    O, lse = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, bs, want_lse=True)
+    assert sdl.last_device_status() == sdl.SDL_OK
+    rows = sample_rows(2, 12, 4096, bs, mask.sum(-1), n_blocks=6, rows_per_block=6)
+    Ow, lw = oracle.attention(host["q"], host["k"], host["v"], bs, mask=mask, rows=rows)
+    got = bf16_to_f64(O)[rows[:, 0], rows[:, 2], rows[:, 1]]
+    check_close(got, Ow, "bf16")
+    lg = lse.cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    assert np.abs(lg - lw).max() <= TOL["bf16"]["lse"]
+
+
+def test_repeated_launches_on_two_streams_are_identical():
+    """The attention kernel's CTAs take tiles from a per-launch counter that the
+    last CTA resets; 150 launches, alternating over two streams, must all give
+    the result of the first, bit for bit."""
+    w = synth.small_workload(L=2048, H=8, H_kv=2, d=128, bs=64)
+    _, dev = _inputs(w)
+    mask = _random_mask(1, 8, 32, 0.3, np.random.default_rng(3))
+    rp, ci = _mask_to_csr(mask)
+    ref = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64)
+    ref_dense = sdl.dense_attn(dev["q"], dev["k"], dev["v"])
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [torch.empty_like(ref) for _ in range(4)]
+    torch.cuda.synchronize()
+    for n in range(150):
+        with torch.cuda.stream(streams[n % 2]):
+            if n % 3 == 2:
+                sdl.dense_attn(dev["q"], dev["k"], dev["v"], out=outs[2 + n % 2])
+            else:
+                sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, out=outs[n % 2])
+    torch.cuda.synchronize()
+    assert sdl.last_device_status() == sdl.SDL_OK
+    assert torch.equal(outs[0], ref) and torch.equal(outs[1], ref)
+    assert torch.equal(outs[2], ref_dense) and torch.equal(outs[3], ref_dense)
 
 
 @pytest.mark.parametrize("dtype,L,H,Hkv,d", [("bf16", 1024, 4, 2, 128), ("bf16", 640, 2, 2, 64),
