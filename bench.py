@@ -55,6 +55,9 @@ def parse():
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--profile", choices=["sparse", "dense"], default=None,
+                   help="launch only this attention kernel (warmup + steps times, one input) "
+                        "and print its event-timed average; for profiler captures")
     return p.parse_args()
 
 
@@ -317,6 +320,35 @@ def run_reference(args):
     print(json.dumps(line))
 
 
+def profile_kernel(runner, args):
+    """Only the chosen attention kernel, back to back on one input (mask from one
+    anchor refresh): the launch list is warmup + steps launches of that kernel."""
+    w, sdl = runner.w, runner.sdl
+    x = runner.make_inputs([0])[0]
+    runner.att.refresh(x["q"], x["k"], 0)
+    torch.cuda.synchronize()
+    if args.profile == "sparse":
+        fn = lambda: sdl.sparse_attn(x["q"], x["k"], x["v"], runner.att.row_ptr,
+                                     runner.att.col_idx, w.bs, out=runner.out)
+        flop = 4.0 * w.bs * w.bs * w.d * runner.att.budget
+    else:
+        fn = lambda: sdl.dense_attn(x["q"], x["k"], x["v"], out=runner.out)
+        flop = 4.0 * w.B * w.H * w.L * w.L * w.d
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / max(args.steps, 1)
+    print(json.dumps({"profile": args.profile, "workload": args.workload, "ms": ms,
+                      "tflops": flop / (ms * 1e-3) / 1e12,
+                      "status": sdl.last_device_status()}))
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -336,6 +368,9 @@ def main():
     w = synth.WORKLOADS[args.workload]
     seed = args.seed + rank  # each rank: its own independent sequence
     runner = Runner(w, seed, device)
+    if args.profile:
+        profile_kernel(runner, args)
+        return
     steps = list(range(args.steps))
     inputs = runner.make_inputs(steps)
     warm = [inputs[i % len(inputs)] for i in range(args.warmup)]

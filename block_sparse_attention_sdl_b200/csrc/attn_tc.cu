@@ -3,45 +3,54 @@
 // The fused IO-aware block-sparse kernel of the Step-dLLM abstract,
 // re-designed for Blackwell.  A work item is a 128-row query tile of one
 // head; it walks the kept key blocks of its rows, two 64-token sub-blocks
-// (128 keys) per step.  CTAs are persistent (one per SM) and take items from
-// a global counter, first come first served (tiles differ in cost by the
-// length of their kept lists).  The next item's kept list and Q tile are staged while the
-// current one computes, the MMA issuer looks one step ahead across items, and
-// two O accumulators let one item's epilogue overlap the next item's products.
+// (128 keys) per step.  CTAs are persistent (one per SM).  Each runs two
+// independent item streams: the MMA issuer alternates between them, so one
+// stream's softmax overlaps the other stream's products.  Items come from a
+// global counter, first come first served (tiles differ in cost by the length
+// of their kept lists).
 //
-//   warp 0        K producer: K sub-blocks of every step by TMA
-//                 (128-byte-swizzled 64x64 boxes) into a 2-deep ring.
-//   warp 10       V producer: the V sub-blocks into their own 2-deep ring (one
-//                 issuing thread alone cannot copy a step's K and V in time).
-//   warp 11       item producer: the union list of the next item's rows into
-//                 one of two shared-memory slots, then its Q tile by TMA into
-//                 the matching Q slot.  Items whose lists are empty (only a
-//                 caller's mask can have empty rows) are written here as zero
-//                 rows and never reach the other warps.
+//   warp 0        K producer: the K sub-blocks of every step by TMA
+//                 (128-byte-swizzled 64x64 boxes) into a 2-deep ring, in the
+//                 merged step order of the two streams (below); the Q tile of
+//                 a stream's next item once that stream's last S product of
+//                 the previous item has completed.
+//   warp 2        V producer: the V sub-blocks, same order, own 2-deep ring.
+//   warp 3        item producer: takes items, builds the union list of an
+//                 item's two query blocks into a free list slot of whichever
+//                 stream has one (two per stream) and prefetches its Q tile
+//                 into L2.  Items whose lists are empty (only a caller's mask
+//                 can have empty rows) are written here as zero rows.
 //   warp 1        TMEM allocator and MMA issuer (one thread):
-//                   S = Q K^T   tcgen05.mma kind::f16, A and B from shared
-//                               memory, M=128, N=128, fp32 into one of two
-//                               TMEM S buffers (by step parity);
-//                   O += P V    A = P (bf16) from TMEM, B = V from shared
-//                               memory (N-major), M=128, N=d, into the
-//                               item's TMEM O buffer (by slot).
-//   warps 2-9     softmax in two warpgroups: each thread one query row (its
-//                 TMEM lane) and one 64-column half of the step; online
-//                 softmax in the log2 domain with the running max raised
-//                 only when it grows by more than 8 (a factor 256) and O
-//                 rescaled in TMEM only then; P written back as bf16 over the
-//                 thread's own S columns, the row sum taken over those
-//                 rounded weights; 2 of every 8 exponentials on the FMA pipe.
-//                 Epilogue per item: O / l rounded to bf16, LSE.
+//                   S_t = Q_t K^T  tcgen05.mma kind::f16, A and B from shared
+//                                  memory, M=128, N=128, fp32 in TMEM;
+//                   O_t += P_t V   A = P_t (bf16, over S_t's first 64 TMEM
+//                                  columns), B = V from shared memory
+//                                  (N-major), M=128, N=d.
+//                 A stream's next S is issued after its PV product (the two
+//                 share S_t's columns), which also leaves O_t quiescent for
+//                 that stream's softmax once the S product has completed.
+//   warps 4-7     softmax of stream 0, warps 8-11 of stream 1: one thread per
+//                 query row (its TMEM lane), all 128 columns of the step.
+//                 Online softmax in the log2 domain; the running max is raised
+//                 only when it grows by more than 8 (a factor 256), and O_t is
+//                 rescaled in TMEM only then; P written back as bf16, the row
+//                 sum taken over those rounded weights; 2 of every 8
+//                 exponentials on the FMA pipe.  Epilogue per item: O / l
+//                 rounded to bf16, LSE.
+//
+// Merged step order: the producers and the MMA issuer take the steps of the
+// two streams alternately (0, 1, 0, 1, ...); once a stream has no more items
+// the other continues alone.  Each derives this order from the published
+// lists, so the K and V rings are filled and drained in one order.
 //
 // With 64-token blocks a 128-row tile covers two query blocks; the item walks
 // the union of their kept lists and masks, per 64x64 quadrant, the key
 // sub-blocks a query block did not keep.  With 128-token blocks both halves
 // share one list.  Dense attention is the same walk over every sub-block.
 //
-// TMEM (512 columns): S buffers at columns 0 and 128, O buffers at 256, 384.
-// Every mbarrier wait is bounded; on timeout the CTA raises the device
-// status word, drains its own copies and MMAs, frees TMEM and exits.
+// TMEM (512 columns): S_0 at column 0, S_1 at 128, O_0 at 256, O_1 at 384.
+// Every mbarrier wait is bounded; on timeout the CTA raises the device status
+// word, drains its own copies and MMAs, frees TMEM and exits.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -56,17 +65,17 @@ namespace {
 constexpr int kBM = 128;         // query rows per item
 constexpr int kBN = 128;         // key rows per step
 constexpr int kStages = 2;       // K and V ring depth
-constexpr int kSlots = 2;        // item slots: list, Q tile, O accumulator
+constexpr int kStreams = 2;
+constexpr int kSlots = 2;        // list slots per stream
 constexpr int kMaxSub = 1024;    // 64-token sub-blocks per sequence (L <= 65536)
 constexpr int kThreads = 384;    // 12 warps
-constexpr int kVWarp = 10;       // V producer
-constexpr int kItemWarp = 11;    // item producer
-constexpr int kSoftWarps = 8;
+constexpr int kKWarp = 0, kMmaWarp = 1, kVWarp = 2, kItemWarp = 3, kSoftWarp0 = 4;
 constexpr int kBox = 64 * 128;   // bytes of one 64-row x 64-column bf16 box
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;    // S buffer u at kColS + 128 u
-constexpr uint32_t kColO = 256;  // O buffer of slot s at kColO + 128 s
 constexpr int kPolyPer8 = 2;     // of every 8 weights, how many take exp2_poly (FMA pipe)
+
+__host__ __device__ constexpr uint32_t col_s(int t) { return 128u * (uint32_t)t; }
+__host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * (uint32_t)t; }
 
 template <int D>
 struct Layout {
@@ -75,35 +84,33 @@ struct Layout {
   static constexpr int kKVBytes = kBN * D * 2;     // one stage of K (or V)
   static constexpr int kChunkRowsQ = kBM * 128;    // bytes per Q column chunk
   static constexpr int kChunkRowsKV = kBN * 128;   // bytes per K/V column chunk
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kSlots * kQBytes;
+  static constexpr int kOffQ = 0;                  // one Q tile per stream
+  static constexpr int kOffK = kStreams * kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKVBytes;
   static constexpr int kBytes = kOffV + kStages * kKVBytes;
   static constexpr int kSmem = kBytes + 1024;      // + alignment slack
 };
 
+// Consumers of a list slot: K producer, V producer, MMA, the stream's 4 softmax warps.
+constexpr int kListConsumers = 3 + 4;
+
 struct Bars {
-  uint64_t list_full[kSlots];   // slot published by the item producer
-  uint64_t list_empty[kSlots];  // slot released by every consumer
-  uint64_t q_full[kSlots];
-  uint64_t q_empty[kSlots];     // every S product reading the Q slot completed
-  uint64_t kfull[kStages], kempty[kStages];  // K slot free once its S product completed
-  uint64_t vfull[kStages], vempty[kStages];  // V slot free once its PV product completed
-  uint64_t s[2];                // S buffer filled
-  uint64_t p[2];                // P written over that S buffer
-  uint64_t o;                   // one completion per PV product
-  uint64_t o_full[kSlots];      // every product of the slot's item completed
-  uint64_t o_empty[kSlots];     // the slot's O read by the epilogue
-  uint64_t soft;                // barrier of the softmax warps
+  uint64_t list_full[kStreams][kSlots];   // slot published by the item producer
+  uint64_t list_empty[kStreams][kSlots];  // slot released by every consumer
+  uint64_t q_full[kStreams];
+  uint64_t q_empty[kStreams];  // the S products of the stream's item completed
+  uint64_t s_full[kStreams];   // S_t written
+  uint64_t p_full[kStreams];   // P_t written (one arrival per softmax warp)
+  uint64_t o_full[kStreams];   // every product of the stream's item completed
+  uint64_t kfull[kStages], kempty[kStages];
+  uint64_t vfull[kStages], vempty[kStages];
   uint64_t done;
 };
-
-constexpr int kListConsumers = 3 + kSoftWarps;  // MMA, K and V producers, softmax warps
 
 // One published item: its kept list, sub-block index | keep bits << 16
 // (bit 0: query rows 0..63 keep it, bit 1: rows 64..127).
 struct Slot {
-  int item;  // -1: end of this CTA's schedule
+  int item;  // -1: end of the stream
   int n_ent;
   int b, h, t0;
   uint32_t ent[kMaxSub];
@@ -119,6 +126,46 @@ struct Sched {
 };
 __device__ Sched g_sched[kSchedRing];
 
+// A single-thread consumer's position in the merged step order.
+struct Cursor {
+  int k0, k1;  // ordinal of each stream's current item (-1: none yet)
+  int j0, j1;  // next step of that item
+  int n0, n1;  // steps of that item
+  bool live0, live1;
+  int turn;
+  __device__ void init() {
+    k0 = k1 = -1;
+    j0 = j1 = n0 = n1 = 0;
+    live0 = live1 = true;
+    turn = 0;
+  }
+  __device__ int k(int t) const { return t ? k1 : k0; }
+  __device__ bool live(int t) const { return t ? live1 : live0; }
+  __device__ bool at_end(int t) const { return t ? j1 == n1 : j0 == n0; }
+  __device__ void open(int t, int k_, int n_) {
+    if (t) {
+      k1 = k_;
+      j1 = 0;
+      n1 = n_;
+    } else {
+      k0 = k_;
+      j0 = 0;
+      n0 = n_;
+    }
+  }
+  __device__ void kill(int t) {
+    if (t)
+      live1 = false;
+    else
+      live0 = false;
+  }
+  // consumes stream t's next step: returns its index within the item
+  __device__ int take(int t) {
+    turn = t ^ 1;
+    return t ? j1++ : j0++;
+  }
+};
+
 __device__ __forceinline__ void raise_timeout(volatile int* abort_flag, int* status) {
   *abort_flag = 1;
   atomicOr(status, kDevTimeout);
@@ -126,7 +173,8 @@ __device__ __forceinline__ void raise_timeout(volatile int* abort_flag, int* sta
 
 // Zero output rows (and -inf LSE) of a 128-row tile whose kept list is empty.
 template <int D>
-__device__ __forceinline__ void write_empty_tile(const AttnArgs& a, int b, int h, int t0, int lane) {
+__device__ __forceinline__ void write_empty_tile(const AttnArgs& a, int b, int h, int t0,
+                                                 int lane) {
   for (int r = lane; r < kBM; r += 32) {
     const int t = t0 + r;
     if (t >= a.L) break;
@@ -147,26 +195,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
                                             ~(uintptr_t)1023);
   __shared__ Bars bars;
-  __shared__ Slot slots[kSlots];
+  __shared__ Slot slots[kStreams][kSlots];
   __shared__ uint32_t bmask[2][kMaxSub / 32];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
-  __shared__ float sh_max[2][2][kBM];  // [step parity][group][row] tile maxima
-  __shared__ float sh_sum[2][2][kBM];  // [rounded, unrounded][group][row] row sums
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = (a.L + kBM - 1) / kBM;
   const int n_items = a.B * a.H * n_qt;
 
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     if (lane == 0) {
-      for (int s = 0; s < kSlots; ++s) {
-        mbar_init(&bars.list_full[s], 1);
-        mbar_init(&bars.list_empty[s], kListConsumers);
-        mbar_init(&bars.q_full[s], 1);
-        mbar_init(&bars.q_empty[s], 1);
-        mbar_init(&bars.o_full[s], 1);
-        mbar_init(&bars.o_empty[s], kSoftWarps);
+      for (int t = 0; t < kStreams; ++t) {
+        for (int s = 0; s < kSlots; ++s) {
+          mbar_init(&bars.list_full[t][s], 1);
+          mbar_init(&bars.list_empty[t][s], kListConsumers);
+        }
+        mbar_init(&bars.q_full[t], 1);
+        mbar_init(&bars.q_empty[t], 1);
+        mbar_init(&bars.s_full[t], 1);
+        mbar_init(&bars.p_full[t], 4);
+        mbar_init(&bars.o_full[t], 1);
       }
       for (int s = 0; s < kStages; ++s) {
         mbar_init(&bars.kfull[s], 1);
@@ -174,12 +223,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars.vfull[s], 1);
         mbar_init(&bars.vempty[s], 1);
       }
-      for (int s = 0; s < 2; ++s) {
-        mbar_init(&bars.s[s], 1);
-        mbar_init(&bars.p[s], kSoftWarps);  // one elected arrival per softmax warp
-      }
-      mbar_init(&bars.o, 1);
-      mbar_init(&bars.soft, kSoftWarps);
       mbar_init(&bars.done, 1);
       abort_sh = 0;
       fence_barrier_init();
@@ -193,441 +236,523 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
+  // (The producer and MMA roles run warp-converged; one elected lane issues
+  // their copies, MMAs and arrivals, and every wait is made warp-uniform.)
+  // Stream of the next step in the merged order, opening that stream's next
+  // item when its current one is used up (on_open(t) runs then); -1 once both
+  // streams have ended, -2 on timeout.  If blocked(t), the caller cannot take
+  // a step of stream t yet: t is returned and nothing is opened.
+  auto peek = [&](Cursor& C, auto&& blocked, auto&& on_open) -> int {
+    for (int attempt = 0; attempt < 2; ++attempt) {
+      const int t = C.turn ^ attempt;
+      if (!C.live(t)) continue;
+      if (blocked(t)) return t;
+      if (C.at_end(t)) {
+        const int kn = C.k(t) + 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.list_full[t][kn % kSlots], (kn / kSlots) & 1,
+                                                &abort_sh, a.status, kWaitLimitNs)))
+          return -2;
+        const Slot& S = slots[t][kn % kSlots];
+        if (S.item < 0) {
+          C.kill(t);
+          continue;
+        }
+        C.open(t, kn, (S.n_ent + 1) / 2);
+        if (!on_open(t)) return -2;
+      }
+      return t;
+    }
+    return -1;
+  };
+
   if (warp == kItemWarp) {
     // ====================================================== item producer
-    // Takes items from the launch's counter and publishes the non-empty ones,
-    // in order, into slots k % kSlots (k = publication ordinal), then the
-    // end marker.
     const int nsub = a.L / kSubBlock;
-    int qiss0 = 0, qiss1 = 0;  // Q loads issued per slot
+    int pub0 = 0, pub1 = 0;  // slots published per stream (end marker included)
+    bool ended0 = false, ended1 = false;
+    bool exhausted = false;  // the launch's counter ran out
     bool ok = true;
-    int k = 0;
-    bool slot_free = true;  // slot k % kSlots may be written without a wait
-    for (;;) {
-      unsigned taken = 0;
-      if (lane == 0) taken = atomicAdd(&g_sched[sched_slot].next, 1u);
-      taken = __shfl_sync(0xffffffffu, taken, 0);
-      const bool have = taken < (unsigned)n_items;
-      const int item = (int)taken;
-      const int slot = k % kSlots;
-      if (!slot_free) {
-        if (lane == 0)
-          ok = mbar_wait(&bars.list_empty[slot], ((k / kSlots) - 1) & 1, &abort_sh, a.status,
-                         kWaitLimitNs);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) break;
-        slot_free = true;
-      }
-      Slot& S = slots[slot];
-      if (!have) {
-        if (lane == 0) {
-          S.item = -1;
-          S.n_ent = 0;
-          mbar_arrive(&bars.list_full[slot]);
+    uint64_t t_idle = 0;
+    while (ok && !(ended0 && ended1)) {
+      bool progressed = false;
+#pragma unroll 1
+      for (int t = 0; t < kStreams; ++t) {
+        if (t ? ended1 : ended0) continue;
+        const int pub = t ? pub1 : pub0;
+        const int slot = pub % kSlots;
+        bool free_slot = pub < kSlots;
+        if (!free_slot) {
+          if (lane == 0)
+            free_slot = mbar_test_wait(&bars.list_empty[t][slot], ((pub / kSlots) - 1) & 1);
+          free_slot = __shfl_sync(0xffffffffu, free_slot ? 1 : 0, 0) != 0;
         }
-        break;
-      }
-      const int b = item / (a.H * n_qt);
-      const int h = (item / n_qt) % a.H;
-      const int t0 = (item % n_qt) * kBM;
-      // kept 64-token key sub-blocks of the two query halves, as bitmaps
-      for (int w = lane; w < kMaxSub / 32; w += 32) bmask[0][w] = bmask[1][w] = 0;
-      __syncwarp();
-      if (a.row_ptr == nullptr) {
-        for (int s = lane; s < nsub; s += 32) {
-          atomicOr(&bmask[0][s / 32], 1u << (s % 32));
-          if (t0 + 64 < a.L) atomicOr(&bmask[1][s / 32], 1u << (s % 32));
-        }
-      } else {
-        const int per = a.block / kSubBlock;  // sub-blocks per block: 1 or 2
-        const int rows_in_tile = a.block == 64 ? 2 : 1;
-        for (int rr = 0; rr < rows_in_tile; ++rr) {
-          const int i = t0 / a.block + rr;
-          if (i >= a.nb) break;
-          const int64_t r = ((int64_t)b * a.H + h) * a.nb + i;
-          const int beg = a.row_ptr[r], end = a.row_ptr[r + 1];
-          for (int x = beg + lane; x < end; x += 32) {
-            const int j = a.col_idx[x];
-            const bool bad_range = j < 0 || j >= a.nb;
-            if (bad_range || (x > beg && a.col_idx[x - 1] >= j)) atomicOr(a.status, kDevBadMask);
-            if (bad_range) continue;
-            for (int u = 0; u < per; ++u) {
-              const int s = j * per + u;
-              if (a.block == 64) {
-                atomicOr(&bmask[rr][s / 32], 1u << (s % 32));
-              } else {
-                atomicOr(&bmask[0][s / 32], 1u << (s % 32));
-                atomicOr(&bmask[1][s / 32], 1u << (s % 32));
+        if (!free_slot) continue;
+        progressed = true;
+        Slot& S = slots[t][slot];
+        // take items until a non-empty one (or none is left)
+        int item = -1, n_ent = 0, b = 0, h = 0, t0 = 0;
+        while (!exhausted) {
+          unsigned taken = 0;
+          if (lane == 0) taken = atomicAdd(&g_sched[sched_slot].next, 1u);
+          taken = __shfl_sync(0xffffffffu, taken, 0);
+          if (taken >= (unsigned)n_items) {
+            exhausted = true;
+            break;
+          }
+          item = (int)taken;
+          b = item / (a.H * n_qt);
+          h = (item / n_qt) % a.H;
+          t0 = (item % n_qt) * kBM;
+          // kept 64-token key sub-blocks of the two query halves, as bitmaps
+          for (int w = lane; w < kMaxSub / 32; w += 32) bmask[0][w] = bmask[1][w] = 0;
+          __syncwarp();
+          if (a.row_ptr == nullptr) {
+            for (int s = lane; s < nsub; s += 32) {
+              atomicOr(&bmask[0][s / 32], 1u << (s % 32));
+              if (t0 + 64 < a.L) atomicOr(&bmask[1][s / 32], 1u << (s % 32));
+            }
+          } else {
+            const int per = a.block / kSubBlock;  // sub-blocks per block: 1 or 2
+            const int rows_in_tile = a.block == 64 ? 2 : 1;
+            for (int rr = 0; rr < rows_in_tile; ++rr) {
+              const int i = t0 / a.block + rr;
+              if (i >= a.nb) break;
+              const int64_t r = ((int64_t)b * a.H + h) * a.nb + i;
+              const int beg = a.row_ptr[r], end = a.row_ptr[r + 1];
+              for (int x = beg + lane; x < end; x += 32) {
+                const int jb = a.col_idx[x];
+                const bool bad_range = jb < 0 || jb >= a.nb;
+                if (bad_range || (x > beg && a.col_idx[x - 1] >= jb))
+                  atomicOr(a.status, kDevBadMask);
+                if (bad_range) continue;
+                for (int u = 0; u < per; ++u) {
+                  const int s = jb * per + u;
+                  if (a.block == 64) {
+                    atomicOr(&bmask[rr][s / 32], 1u << (s % 32));
+                  } else {
+                    atomicOr(&bmask[0][s / 32], 1u << (s % 32));
+                    atomicOr(&bmask[1][s / 32], 1u << (s % 32));
+                  }
+                }
               }
             }
           }
+          __syncwarp();
+          // ascending union with per-half keep bits: lane w handles bitmap word w
+          const uint32_t w0 = bmask[0][lane], w1 = bmask[1][lane];
+          const uint32_t wu = w0 | w1;
+          const int c = __popc(wu);
+          int incl = c;
+          for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+          }
+          n_ent = __shfl_sync(0xffffffffu, incl, 31);
+          __syncwarp();
+          if (n_ent == 0) {
+            write_empty_tile<D>(a, b, h, t0, lane);
+            __syncwarp();
+            continue;
+          }
+          int pos = incl - c;
+          for (uint32_t mb = wu; mb; mb &= mb - 1) {
+            const int bit = __ffs(mb) - 1;
+            const uint32_t keep = ((w0 >> bit) & 1u) | (((w1 >> bit) & 1u) << 1);
+            S.ent[pos++] = (uint32_t)(lane * 32 + bit) | (keep << 16);
+          }
+          break;
         }
-      }
-      __syncwarp();
-      // ascending union with per-half keep bits: lane w handles bitmap word w
-      const uint32_t w0 = bmask[0][lane], w1 = bmask[1][lane];
-      const uint32_t wu = w0 | w1;
-      const int c = __popc(wu);
-      int incl = c;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const int n_ent = __shfl_sync(0xffffffffu, incl, 31);
-      if (n_ent == 0) {
-        write_empty_tile<D>(a, b, h, t0, lane);
+        const bool end_marker = n_ent == 0;  // (only when the counter ran out)
+        if (lane == 0) {
+          if (end_marker) {
+            S.item = -1;
+            S.n_ent = 0;
+          } else {
+            S.item = item;
+            S.n_ent = n_ent;
+            S.b = b;
+            S.h = h;
+            S.t0 = t0;
+            // its Q tile is loaded when this stream's previous item is done; warm L2 now
+            for (int cc = 0; cc < Lay::kChunks; ++cc)
+              for (int s = 0; s < 2; ++s) tma_prefetch_l2_4d(&tmq, cc * 64, t0 + 64 * s, h, b);
+          }
+        }
         __syncwarp();
-        continue;  // the slot stays free for the next item
-      }
-      int pos = incl - c;
-      for (uint32_t mb = wu; mb; mb &= mb - 1) {
-        const int bit = __ffs(mb) - 1;
-        const uint32_t keep = ((w0 >> bit) & 1u) | (((w1 >> bit) & 1u) << 1);
-        S.ent[pos++] = (uint32_t)(lane * 32 + bit) | (keep << 16);
-      }
-      if (lane == 0) {
-        S.item = item;
-        S.n_ent = n_ent;
-        S.b = b;
-        S.h = h;
-        S.t0 = t0;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bars.list_full[slot]);
-        // Q tile of the item; the slot's previous Q is free once the S
-        // products that read it completed
-        const int qiss = slot ? qiss1 : qiss0;
-        if (qiss > 0)
-          ok = mbar_wait(&bars.q_empty[slot], (qiss - 1) & 1, &abort_sh, a.status, kWaitLimitNs);
-        if (ok) {
-          uint8_t* sq = dsm + Lay::kOffQ + slot * Lay::kQBytes;
-          mbar_arrive_expect_tx(&bars.q_full[slot], Lay::kQBytes);
-          for (int cc = 0; cc < Lay::kChunks; ++cc)
-            for (int s = 0; s < 2; ++s)
-              tma_load_4d(sq + cc * Lay::kChunkRowsQ + s * kBox, &tmq, &bars.q_full[slot],
-                          cc * 64, t0 + 64 * s, h, b);
-          if (slot) ++qiss1; else ++qiss0;
+        if (lane == 0) mbar_arrive(&bars.list_full[t][slot]);
+        if (t) {
+          ++pub1;
+          ended1 = end_marker;
+        } else {
+          ++pub0;
+          ended0 = end_marker;
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      ++k;
-      slot_free = k < kSlots;
-    }
-    if (lane == 0) {
-      if (!ok) raise_timeout(&abort_sh, a.status);
-      // Drain: the Q copies issued above land before the CTA exits.
-      volatile int no_abort = 0;
-      for (int s = 0; s < kSlots; ++s) {
-        const int qiss = s ? qiss1 : qiss0;
-        if (qiss > 0 &&
-            !mbar_wait(&bars.q_full[s], (qiss - 1) & 1, &no_abort, nullptr, kWaitLimitNs))
-          atomicOr(a.status, kDevTimeout);
+      if (progressed) {
+        t_idle = 0;
+      } else {
+        // every slot of both streams is busy: back off, bounded by the wait limit
+        if (t_idle == 0) t_idle = globaltimer_ns();
+        __nanosleep(500);
+        if (abort_sh || globaltimer_ns() - t_idle > kWaitLimitNs) ok = false;
       }
     }
-  } else if (warp == 0 || warp == kVWarp) {
+    if (lane == 0 && !ok) raise_timeout(&abort_sh, a.status);
+  } else if (warp == kKWarp || warp == kVWarp) {
     // ================================================= K and V producers
-    const bool isk = warp == 0;
+    const bool isk = warp == kKWarp;
     uint64_t* full = isk ? bars.kfull : bars.vfull;
     uint64_t* empty = isk ? bars.kempty : bars.vempty;
     const CUtensorMap* tm = isk ? &tmk : &tmv;
     uint8_t* ring = dsm + (isk ? Lay::kOffK : Lay::kOffV);
     const int group = a.H / a.Hkv;
-    if (lane == 0) {
-      prefetch_tensormap(tm);
-      if (isk) prefetch_tensormap(&tmq);
-      int g = 0;  // global step: ring stage g % kStages
+    {
+      const bool leader = elect_one_sync();
+      if (leader) {
+        prefetch_tensormap(tm);
+        if (isk) prefetch_tensormap(&tmq);
+      }
+      Cursor C;
+      C.init();
+      int qiss0 = 0, qiss1 = 0;  // Q tiles loaded per stream
       bool ok = true;
-      for (int k = 0; ok; ++k) {
-        const int slot = k % kSlots;
-        if (!(ok = mbar_wait(&bars.list_full[slot], (k / kSlots) & 1, &abort_sh, a.status,
-                             kWaitLimitNs)))
+      int g = 0;  // position in the merged order: ring stage g % kStages
+      auto never = [](int) { return false; };
+      auto on_open = [&](int t) -> bool {
+        if (!isk) return true;
+        // Q of the stream's new item, once its previous item's S products completed
+        const int n = t ? qiss1 : qiss0;
+        if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars.q_empty[t], (n - 1) & 1, &abort_sh,
+                                                        a.status, kWaitLimitNs)))
+          return false;
+        const Slot& S = slots[t][C.k(t) % kSlots];
+        uint8_t* sq = dsm + Lay::kOffQ + t * Lay::kQBytes;
+        if (leader) {
+          mbar_arrive_expect_tx(&bars.q_full[t], Lay::kQBytes);
+          for (int cc = 0; cc < Lay::kChunks; ++cc)
+            for (int s = 0; s < 2; ++s)
+              tma_load_4d(sq + cc * Lay::kChunkRowsQ + s * kBox, &tmq, &bars.q_full[t], cc * 64,
+                          S.t0 + 64 * s, S.h, S.b);
+        }
+        if (t)
+          ++qiss1;
+        else
+          ++qiss0;
+        return true;
+      };
+      for (;;) {
+        const int t = peek(C, never, on_open);
+        if (t == -2) ok = false;
+        if (t < 0) break;
+        const int jj = C.take(t);
+        const int slot = C.k(t) % kSlots;
+        const Slot& S = slots[t][slot];
+        const int n_ent = S.n_ent;
+        const uint32_t e0 = S.ent[2 * jj];
+        const uint32_t e1 = (2 * jj + 1 < n_ent) ? S.ent[2 * jj + 1] : e0;
+        const int sub0 = (int)(e0 & 0xFFFFu), sub1 = (int)(e1 & 0xFFFFu);
+        const int kh = S.h / group, b = S.b;
+        const int st = g % kStages;
+        if (g >= kStages &&
+            !(ok = __all_sync(0xffffffffu, mbar_wait(&empty[st], ((g / kStages) - 1) & 1,
+                                                     &abort_sh, a.status, kWaitLimitNs))))
           break;
-        const Slot& S = slots[slot];
-        if (S.item < 0) break;
-        const int n_ent = S.n_ent, b = S.b, kh = S.h / group;
-        const int steps = (n_ent + 1) / 2;
-        for (int j = 0; j < steps; ++j, ++g) {
-          const uint32_t e0 = S.ent[2 * j];
-          const uint32_t e1 = (2 * j + 1 < n_ent) ? S.ent[2 * j + 1] : e0;
-          const int sub0 = (int)(e0 & 0xFFFFu), sub1 = (int)(e1 & 0xFFFFu);
-          const int st = g % kStages;
-          if (g >= kStages &&
-              !(ok = mbar_wait(&empty[st], ((g / kStages) - 1) & 1, &abort_sh, a.status,
-                               kWaitLimitNs)))
-            break;
-          uint8_t* dst = ring + st * Lay::kKVBytes;
+        uint8_t* dst = ring + st * Lay::kKVBytes;
+        if (leader) {
           mbar_arrive_expect_tx(&full[st], Lay::kKVBytes);
           for (int c = 0; c < Lay::kChunks; ++c)
             for (int s = 0; s < 2; ++s)
               tma_load_4d(dst + c * Lay::kChunkRowsKV + s * kBox, tm, &full[st], c * 64,
                           (s ? sub1 : sub0) * kSubBlock, kh, b);
+          if (C.at_end(t)) mbar_arrive(&bars.list_empty[t][slot]);
         }
-        if (ok) mbar_arrive(&bars.list_empty[slot]);
-      }
-      if (!ok) raise_timeout(&abort_sh, a.status);
-      // Drain: every copy issued above lands before the CTA exits.
-      volatile int no_abort = 0;
-      for (int st = (g > kStages ? g - kStages : 0); st < g; ++st)
-        if (!mbar_wait(&full[st % kStages], (st / kStages) & 1, &no_abort, nullptr, kWaitLimitNs))
-          atomicOr(a.status, kDevTimeout);
-    }
-  } else if (warp == 1) {
-    // ================================================================ MMA
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, false);
-      constexpr uint32_t idPV = idesc_bf16_f32(kBM, D, true);
-      const uint32_t q_base = smem_u32(dsm + Lay::kOffQ);
-      const uint32_t k_base = smem_u32(dsm + Lay::kOffK);
-      const uint32_t v_base = smem_u32(dsm + Lay::kOffV);
-      int quse0 = 0, quse1 = 0;  // Q tiles consumed per slot
-      int ouse0 = 0, ouse1 = 0;  // items accumulated per O slot
-      bool ok = true;
-
-      // Opens publication ordinal k: its step count, or -1 at the end.
-      auto open_item = [&](int k) -> int {
-        const int slot = k % kSlots;
-        if (!mbar_wait(&bars.list_full[slot], (k / kSlots) & 1, &abort_sh, a.status,
-                       kWaitLimitNs)) {
-          ok = false;
-          return -1;
-        }
-        const Slot& S = slots[slot];
-        if (S.item < 0) return -1;
-        if (!mbar_wait(&bars.q_full[slot], (slot ? quse1 : quse0) & 1, &abort_sh, a.status,
-                       kWaitLimitNs)) {
-          ok = false;
-          return -1;
-        }
-        if (slot) ++quse1; else ++quse0;
-        tc_fence_after();
-        return (S.n_ent + 1) / 2;
-      };
-      auto issue_s = [&](int g, int qslot) -> bool {
-        const int st = g % kStages;
-        if (!mbar_wait(&bars.kfull[st], (g / kStages) & 1, &abort_sh, a.status, kWaitLimitNs))
-          return false;
-        tc_fence_after();
-        const uint32_t kb = k_base + st * Lay::kKVBytes;
-        const uint32_t qb = q_base + qslot * Lay::kQBytes;
-        const uint32_t dcol = tmem + kColS + 128u * (uint32_t)(g & 1);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)(kk % 4) * 32;  // 16 bf16 of K inside the swizzle atom
-          const uint64_t ad = smem_desc_sw128(qb + (kk / 4) * Lay::kChunkRowsQ + off, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(kb + (kk / 4) * Lay::kChunkRowsKV + off, 16, 1024);
-          mma_bf16_ss(dcol, ad, bd, idS, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bars.kempty[st]);
-        tc_commit(&bars.s[g & 1]);
-        return true;
-      };
-
-      int k = 0, j = 0, g = 0;
-      int steps = open_item(0);
-      if (steps > 0) {
-        ok = issue_s(0, 0);
-        if (ok && steps == 1) tc_commit(&bars.q_empty[0]);
-      }
-      while (ok && steps > 0) {
-        // S of the next step, into the next item when this one ends here
-        int k2 = k, j2 = j + 1, steps2 = steps;
-        if (j2 == steps) {
-          k2 = k + 1;
-          j2 = 0;
-          steps2 = open_item(k2);
-          if (!ok) break;
-        }
-        if (steps2 > 0) {
-          if (!(ok = issue_s(g + 1, k2 % kSlots))) break;
-          if (j2 == steps2 - 1) tc_commit(&bars.q_empty[k2 % kSlots]);
-        }
-        // O += P V for the current step
-        const int slot = k % kSlots;
-        if (!(ok = mbar_wait(&bars.p[g & 1], (g >> 1) & 1, &abort_sh, a.status, kWaitLimitNs)))
-          break;
-        const int st = g % kStages;
-        if (!(ok = mbar_wait(&bars.vfull[st], (g / kStages) & 1, &abort_sh, a.status,
-                             kWaitLimitNs)))
-          break;
-        const int ouse = slot ? ouse1 : ouse0;
-        if (j == 0 && ouse > 0 &&
-            !(ok = mbar_wait(&bars.o_empty[slot], (ouse - 1) & 1, &abort_sh, a.status,
-                             kWaitLimitNs)))
-          break;
-        tc_fence_after();
-        const uint32_t vb = v_base + st * Lay::kKVBytes;
-        const uint32_t pcol = tmem + kColS + 128u * (uint32_t)(g & 1);
-        const uint32_t ocol = tmem + kColO + 128u * (uint32_t)slot;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, Lay::kChunkRowsKV, 1024);
-          // P elements [16 kk, 16 kk + 16): columns 64 (kk / 4) + 8 (kk % 4)
-          mma_bf16_ts(ocol, pcol + 64 * (kk / 4) + 8 * (kk % 4), bd, idPV,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&bars.vempty[st]);
-        tc_commit(&bars.o);
-        if (j == steps - 1) {
-          tc_commit(&bars.o_full[slot]);
-          if (slot) ++ouse1; else ++ouse0;
-          mbar_arrive(&bars.list_empty[slot]);
-        }
-        k = k2;
-        j = j2;
-        steps = steps2;
         ++g;
       }
-      if (!ok) raise_timeout(&abort_sh, a.status);
-      // Every MMA issued above completes before TMEM is released.
-      tc_commit(&bars.done);
-      volatile int no_abort = 0;
-      if (!mbar_wait(&bars.done, 0, &no_abort, nullptr, kWaitLimitNs))
-        atomicOr(a.status, kDevTimeout);
+      if (leader) {
+        if (!ok) raise_timeout(&abort_sh, a.status);
+        // Drain: every copy issued above lands before the CTA exits.
+        volatile int no_abort = 0;
+        for (int st = (g > kStages ? g - kStages : 0); st < g; ++st)
+          if (!mbar_wait(&full[st % kStages], (st / kStages) & 1, &no_abort, nullptr,
+                         kWaitLimitNs))
+            atomicOr(a.status, kDevTimeout);
+        if (qiss0 > 0 &&
+            !mbar_wait(&bars.q_full[0], (qiss0 - 1) & 1, &no_abort, nullptr, kWaitLimitNs))
+          atomicOr(a.status, kDevTimeout);
+        if (qiss1 > 0 &&
+            !mbar_wait(&bars.q_full[1], (qiss1 - 1) & 1, &no_abort, nullptr, kWaitLimitNs))
+          atomicOr(a.status, kDevTimeout);
+      }
+      __syncwarp();
+    }
+  } else if (warp == kMmaWarp) {
+    // ================================================================ MMA
+    {
+      const bool leader = elect_one_sync();
+      constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(kBM, D, true);
+      // Descriptors are built once: the start-address field (bits 0..13,
+      // address >> 4) of the descriptor for address x + off is the base
+      // descriptor's plus off >> 4, without carry (shared addresses < 2^18).
+      const uint64_t dq = smem_desc_sw128(smem_u32(dsm + Lay::kOffQ), 16, 1024);
+      const uint64_t dk = smem_desc_sw128(smem_u32(dsm + Lay::kOffK), 16, 1024);
+      const uint64_t dv = smem_desc_sw128(smem_u32(dsm + Lay::kOffV), Lay::kChunkRowsKV, 1024);
+      Cursor C;
+      C.init();
+      int qw0 = 0, qw1 = 0;  // Q tiles consumed per stream
+      int gs = 0;            // S products issued: K ring position
+      int gv = 0;            // PV products issued: V ring position
+      int np0 = 0, np1 = 0;  // PV products issued per stream
+      // a stream's pending step: its S issued, its PV not yet (at most one each)
+      bool pend0 = false, pend1 = false;
+      bool first0 = false, first1 = false, last0 = false, last1 = false;
+      int slot0 = 0, slot1 = 0;
+      int oldest = -1;  // stream of the older pending step
+      bool ok = true;
+      auto pending = [&](int t) { return t ? pend1 : pend0; };
+      auto on_open = [&](int t) -> bool {
+        const int n = t ? qw1 : qw0;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&bars.q_full[t], n & 1, &abort_sh, a.status, kWaitLimitNs)))
+          return false;
+        if (t)
+          ++qw1;
+        else
+          ++qw0;
+        return true;
+      };
+      // S for the next step of the merged order if its stream has no pending
+      // step: 1 issued, 0 not now (or nothing left), -2 timeout.
+      auto try_issue_s = [&]() -> int {
+        const int t = peek(C, pending, on_open);
+        if (t == -2) return -2;
+        if (t < 0 || pending(t)) return 0;
+        const int jj = C.take(t);
+        const int st = gs % kStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.kfull[st], (gs / kStages) & 1, &abort_sh,
+                                                a.status, kWaitLimitNs)))
+          return -2;
+        tc_fence_after();
+        const uint64_t ad0 = dq + (uint64_t)((t * Lay::kQBytes) >> 4);
+        const uint64_t bd0 = dk + (uint64_t)((st * Lay::kKVBytes) >> 4);
+        const uint32_t dcol = tmem + col_s(t);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // 16 d-columns: chunk kk / 4, 32 bytes (kk % 4) inside the swizzle atom
+          const uint64_t offq = (uint64_t)(((kk / 4) * Lay::kChunkRowsQ + (kk % 4) * 32) >> 4);
+          const uint64_t offk = (uint64_t)(((kk / 4) * Lay::kChunkRowsKV + (kk % 4) * 32) >> 4);
+          if (leader) mma_bf16_ss(dcol, ad0 + offq, bd0 + offk, idS, kk > 0 ? 1u : 0u);
+        }
+        const bool last = C.at_end(t);
+        if (leader) {
+          tc_commit(&bars.kempty[st]);
+          tc_commit(&bars.s_full[t]);
+          if (last) tc_commit(&bars.q_empty[t]);
+        }
+        ++gs;
+        const int slot = C.k(t) % kSlots;
+        if (t) {
+          pend1 = true;
+          first1 = jj == 0;
+          last1 = last;
+          slot1 = slot;
+        } else {
+          pend0 = true;
+          first0 = jj == 0;
+          last0 = last;
+          slot0 = slot;
+        }
+        if (oldest < 0) oldest = t;
+        return 1;
+      };
+      int r;
+      while ((r = try_issue_s()) == 1) {
+      }
+      if (r == -2) ok = false;
+      while (ok && oldest >= 0) {
+        // O_t += P_t V for the older pending step
+        const int t = oldest;
+        const int np = t ? np1 : np0;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.p_full[t], np & 1, &abort_sh,
+                                                     a.status, kWaitLimitNs))))
+          break;
+        const int st = gv % kStages;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.vfull[st], (gv / kStages) & 1,
+                                                     &abort_sh, a.status, kWaitLimitNs))))
+          break;
+        tc_fence_after();
+        const uint64_t bd0 = dv + (uint64_t)((st * Lay::kKVBytes) >> 4);
+        const uint32_t pcol = tmem + col_s(t);
+        const uint32_t ocol = tmem + col_o(t);
+        const bool first = t ? first1 : first0;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // keys [16 kk, 16 kk + 16): V rows 16 kk.. (128 bytes each); P elements
+          // packed in columns [8 kk, 8 kk + 8)
+          if (leader)
+            mma_bf16_ts(ocol, pcol + 8 * kk, bd0 + (uint64_t)((kk * 16 * 128) >> 4), idPV,
+                        (!first || kk > 0) ? 1u : 0u);
+        }
+        if (leader) tc_commit(&bars.vempty[st]);
+        ++gv;
+        if (t) {
+          ++np1;
+          pend1 = false;
+        } else {
+          ++np0;
+          pend0 = false;
+        }
+        oldest = pending(t ^ 1) ? (t ^ 1) : -1;
+        if ((t ? last1 : last0) && leader) {
+          tc_commit(&bars.o_full[t]);
+          mbar_arrive(&bars.list_empty[t][t ? slot1 : slot0]);
+        }
+        while ((r = try_issue_s()) == 1) {
+        }
+        if (r == -2) ok = false;
+      }
+      if (leader) {
+        if (!ok) raise_timeout(&abort_sh, a.status);
+        // Every MMA issued above completes before TMEM is released.
+        tc_commit(&bars.done);
+        volatile int no_abort = 0;
+        if (!mbar_wait(&bars.done, 0, &no_abort, nullptr, kWaitLimitNs))
+          atomicOr(a.status, kDevTimeout);
+      }
+      __syncwarp();
     }
   } else {
     // ============================================================ softmax
-    // Two warpgroups: group g owns key columns [64 g, 64 g + 64) of each S
-    // row (key sub-block g of the step) and columns [d/2 g, d/2 g + d/2) of
-    // O.  The two threads of a row swap their tile maxima through shared
-    // memory once per step.  Each group writes its half of P (bf16 pairs)
-    // over the first 32 of its own 64 S columns, so neither group overwrites
-    // S the other may still read.
-    const int grp = (warp - 2) / 4;
-    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int t = (warp - kSoftWarp0) / 4;  // stream
+    const int quad = warp & 3;              // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;
     const int half = row >> 6;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t scol = trow + col_s(t);
+    const uint32_t ocol = trow + col_o(t);
     const float sl2 = a.scale_log2;
-    uint32_t soft_uses = 0;
-    int ouse0 = 0, ouse1 = 0;  // items finished per O slot
-    int g = 0;  // global step
+    int n = 0;  // steps of this stream so far
     bool ok = true;
     for (int k = 0;; ++k) {
       const int slot = k % kSlots;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars.list_full[slot], (k / kSlots) & 1, &abort_sh,
-                                             a.status, kWaitLimitNs));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars.list_full[t][slot], (k / kSlots) & 1,
+                                             &abort_sh, a.status, kWaitLimitNs));
       if (!ok) break;
-      const Slot& S = slots[slot];
+      const Slot& S = slots[t][slot];
       if (S.item < 0) break;
-      const int n_ent = S.n_ent, b = S.b, h = S.h, t = S.t0 + row;
+      const int n_ent = S.n_ent, b = S.b, h = S.h, tok = S.t0 + row;
       const int n_steps = (n_ent + 1) / 2;
       float m = -INFINITY;  // running max (log2 units) used as the exponent reference
-      float l = 0.f;        // this half-row's sum of the bf16-rounded weights
-      float lx = 0.f;       // this half-row's sum of the unrounded weights (LSE only)
-      const uint32_t ocol = trow + kColO + 128u * (uint32_t)slot + (D / 2) * grp;
-      for (int j = 0; j < n_steps; ++j, ++g) {
-        const int buf = g & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars.s[buf], (g >> 1) & 1, &abort_sh, a.status,
+      float l = 0.f;        // row sum of the bf16-rounded weights
+      float lx = 0.f;       // row sum of the unrounded weights (LSE only)
+      for (int j = 0; j < n_steps; ++j, ++n) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full[t], n & 1, &abort_sh, a.status,
                                                kWaitLimitNs));
         if (!ok) break;
         tc_fence_after();
         const uint32_t e0 = S.ent[2 * j];
         const uint32_t e1 = (2 * j + 1 < n_ent) ? S.ent[2 * j + 1] : (e0 & 0xFFFFu);
         // (keep is uniform over a warp: its 32 rows lie in one query block)
-        const bool keep = ((grp ? e1 : e0) >> (16 + half)) & 1u;
-        const uint32_t scol = trow + kColS + 128u * (uint32_t)buf + 64 * grp;
-        float sv[64];
-        {
-          uint32_t r[64];
-          tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-          tmem_wait_ld();
+        const bool keep0 = (e0 >> (16 + half)) & 1u;
+        const bool keep1 = (e1 >> (16 + half)) & 1u;
+        uint32_t r[128];
+        tmem_ld32(scol + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld32(scol + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+        tmem_ld32(scol + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+        tmem_wait_ld();
+        float mh[2];
 #pragma unroll
-          for (int x = 0; x < 64; ++x) sv[x] = keep ? __uint_as_float(r[x]) * sl2 : -INFINITY;
+        for (int hf = 0; hf < 2; ++hf) {
+          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+          for (int x = 64 * hf; x < 64 * hf + 64; x += 4) {
+            m0 = fmaxf(m0, __uint_as_float(r[x]));
+            m1 = fmaxf(m1, __uint_as_float(r[x + 1]));
+            m2 = fmaxf(m2, __uint_as_float(r[x + 2]));
+            m3 = fmaxf(m3, __uint_as_float(r[x + 3]));
+          }
+          mh[hf] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
         }
-        float mt = -INFINITY;
-#pragma unroll
-        for (int x = 0; x < 64; x += 2) mt = fmaxf(mt, fmaxf(sv[x], sv[x + 1]));
-        sh_max[buf][grp][row] = mt;
-        if (!(ok = group_sync(&bars.soft, soft_uses, &abort_sh, a.status, kWaitLimitNs))) break;
-        mt = fmaxf(mt, sh_max[buf][grp ^ 1][row]);
+        const float mt = fmaxf(keep0 ? mh[0] : -INFINITY, keep1 ? mh[1] : -INFINITY) * sl2;
         const bool raise = mt > m + 8.0f;
         if (__any_sync(0xffffffffu, raise)) {
           if (j > 0) {
-            // O must hold every product of this item issued so far before it
-            // is rescaled.  PV(g-2) is complete (S(g) was committed after it)
-            // and PV(g) cannot start before this step's P, so the parity of
-            // PV(g-1) names one completion.
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars.o, (g - 1) & 1, &abort_sh, a.status,
-                                                   kWaitLimitNs));
-            if (!ok) break;
-            tc_fence_after();
+            // O_t is quiescent: this step's S product was issued after the
+            // stream's previous PV product and has completed.
             const float alpha = raise ? ex2_approx(m - mt) : 1.0f;
             l *= alpha;
             lx *= alpha;
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-              uint32_t ov[32];
-              tmem_ld32(ocol + c * 32, ov);
+#pragma unroll 1
+            for (int c = 0; c < D / 16; ++c) {
+              uint32_t ov[16];
+              tmem_ld16(ocol + c * 16, ov);
               tmem_wait_ld();
 #pragma unroll
-              for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
-              tmem_st32(ocol + c * 32, ov);
+              for (int x = 0; x < 16; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
+              tmem_st16(ocol + c * 16, ov);
             }
             tmem_wait_st();
           }
           if (raise) m = mt;
         }
         // P = exp2(S * scale * log2e - m) on a kept half, 0 otherwise (a kept
-        // half always has a finite reference here: its own maximum raised it)
-        if (keep) {
-#pragma unroll
-          for (int x = 0; x < 64; x += 2) {
-            if ((x & 7) < 8 - kPolyPer8) {
-              sv[x] = ex2_approx(sv[x] - m);
-              sv[x + 1] = ex2_approx(sv[x + 1] - m);
-            } else {
-              const float2 e = exp2_poly2(sv[x] - m, sv[x + 1] - m);
-              sv[x] = e.x;
-              sv[x + 1] = e.y;
-            }
-          }
-        } else {
-#pragma unroll
-          for (int x = 0; x < 64; ++x) sv[x] = 0.f;
-        }
-        // bf16 pairs of P over this half's own S columns; l sums the rounded weights
+        // half always has a finite reference here: its own maximum raised it);
+        // bf16 pairs over S_t's first 64 columns; l sums the rounded weights
+        const float nm = -m;
         float rs = 0.f, rx = 0.f;
-        uint32_t pw[32];
 #pragma unroll
-        for (int x = 0; x < 64; x += 2) {
-          __nv_bfloat162 pk = __floats2bfloat162_rn(sv[x], sv[x + 1]);
-          const uint32_t u = *reinterpret_cast<uint32_t*>(&pk);
-          rs += __uint_as_float(u << 16) + __uint_as_float(u & 0xFFFF0000u);
-          if constexpr (kLse) rx += sv[x] + sv[x + 1];
-          pw[x / 2] = u;
+        for (int c = 0; c < 4; ++c) {  // 32 weights -> 16 packed columns at a time
+          const bool kp = c < 2 ? keep0 : keep1;
+          uint32_t pw[16];
+          if (kp) {
+#pragma unroll
+            for (int x = 0; x < 32; x += 2) {
+              const float x0 = fmaf(__uint_as_float(r[32 * c + x]), sl2, nm);
+              const float x1 = fmaf(__uint_as_float(r[32 * c + x + 1]), sl2, nm);
+              float p0, p1;
+              if ((x & 7) < 8 - kPolyPer8) {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              } else {
+                const float2 e = exp2_poly2(x0, x1);
+                p0 = e.x;
+                p1 = e.y;
+              }
+              __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+              const uint32_t u = *reinterpret_cast<uint32_t*>(&pk);
+              rs += __uint_as_float(u << 16) + __uint_as_float(u & 0xFFFF0000u);
+              if constexpr (kLse) rx += p0 + p1;
+              pw[x / 2] = u;
+            }
+          } else {
+#pragma unroll
+            for (int x = 0; x < 16; ++x) pw[x] = 0u;
+          }
+          tmem_st16(scol + 16 * c, pw);
         }
         l += rs;
         lx += rx;
-        tmem_st32(scol, pw);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p[buf]);
+        if (lane == 0) mbar_arrive(&bars.p_full[t]);
       }
       if (!ok) break;
       // --------------------------------------------------------- epilogue
-      sh_sum[0][grp][row] = l;
-      sh_sum[1][grp][row] = lx;
-      if (!(ok = group_sync(&bars.soft, soft_uses, &abort_sh, a.status, kWaitLimitNs))) break;
-      l += sh_sum[0][grp ^ 1][row];
-      lx += sh_sum[1][grp ^ 1][row];
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars.o_full[slot], (slot ? ouse1 : ouse0) & 1,
-                                             &abort_sh, a.status, kWaitLimitNs));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars.o_full[t], k & 1, &abort_sh, a.status,
+                                             kWaitLimitNs));
       if (!ok) break;
-      if (slot) ++ouse1; else ++ouse0;
       tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
       __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(a.o) + b * a.os[0] +
-                          (int64_t)t * a.os[1] + h * a.os[2] + (D / 2) * grp;
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+                          (int64_t)tok * a.os[1] + h * a.os[2];
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
         tmem_ld32(ocol + c * 32, ov);
         tmem_wait_ld();
-        if (t < a.L) {
+        if (tok < a.L) {
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
@@ -643,12 +768,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bars.o_empty[slot]);
-        mbar_arrive(&bars.list_empty[slot]);
-      }
-      if (a.lse && grp == 0 && t < a.L)
-        a.lse[((int64_t)b * a.H + h) * a.L + t] =
+      if (lane == 0) mbar_arrive(&bars.list_empty[t][slot]);
+      if (a.lse && tok < a.L)
+        a.lse[((int64_t)b * a.H + h) * a.L + tok] =
             lx > 0.f ? (m + log2f(lx)) * 0.69314718055994531f : -INFINITY;
     }
     if (!ok) raise_timeout(&abort_sh, a.status);
@@ -657,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -698,9 +820,11 @@ cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUten
     e = cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
   }
-  // one persistent CTA per SM (the shared-memory footprint admits one)
+  // one persistent CTA per SM (the shared-memory footprint admits one), each
+  // running two tiles at a time
   const int64_t n_items = (int64_t)a.B * a.H * ((a.L + kBM - 1) / kBM);
-  const int grid = (int)(n_items < g_num_sms[dev] ? n_items : g_num_sms[dev]);
+  const int64_t want = (n_items + kStreams - 1) / kStreams;
+  const int grid = (int)(want < g_num_sms[dev] ? want : g_num_sms[dev]);
   if (a.d == 128)
     return a.lse ? launch_tc<128, true>(a, tq, tk, tv, st, grid)
                  : launch_tc<128, false>(a, tq, tk, tv, st, grid);

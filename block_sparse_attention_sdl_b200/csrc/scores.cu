@@ -18,7 +18,6 @@ namespace sdl {
 namespace {
 
 constexpr int kPoolThreads = 256;
-constexpr int kLaneElems = 16;  // bytes per lane per token (one 16-byte load)
 
 template <typename T>
 struct Vec;
