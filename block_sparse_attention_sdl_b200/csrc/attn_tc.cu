@@ -116,6 +116,14 @@ struct Slot {
   uint32_t ent[kMaxSub];
 };
 
+// Step records, written by the K producer for the MMA issuer, one per step
+// of the merged order (ring position g % kCmdRing):
+//   bit 0 stream, bit 1 first step of its item, bit 2 last step of its item,
+//   bit 3 the item's list slot, bits 4-5 distance back to the stream's
+//   previous step in the merged order (0: none), bit 7 end of the order.
+constexpr int kCmdRing = 8;
+constexpr uint32_t kCmdEnd = 0x80u;
+
 // Item counters of in-flight launches.  Launch n uses entry n % kSchedRing;
 // its CTAs take items with atomicAdd on `next`, and the last CTA to finish
 // puts the entry back to zero for a later launch.
@@ -199,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t bmask[2][kMaxSub / 32];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
+  __shared__ uint32_t cmd[kCmdRing];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = (a.L + kBM - 1) / kBM;
@@ -415,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Cursor C;
       C.init();
       int qiss0 = 0, qiss1 = 0;  // Q tiles loaded per stream
+      int last_g0 = -1, last_g1 = -1;  // merged position of each stream's previous step
       bool ok = true;
       int g = 0;  // position in the merged order: ring stage g % kStages
       auto never = [](int) { return false; };
@@ -458,6 +468,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                      &abort_sh, a.status, kWaitLimitNs))))
           break;
         uint8_t* dst = ring + st * Lay::kKVBytes;
+        if (isk) {
+          const int prev = t ? last_g1 : last_g0;
+          const uint32_t rec = (uint32_t)t | (jj == 0 ? 2u : 0u) | (C.at_end(t) ? 4u : 0u) |
+                               ((uint32_t)slot << 3) | ((uint32_t)(prev < 0 ? 0 : g - prev) << 4);
+          if (t)
+            last_g1 = g;
+          else
+            last_g0 = g;
+          if (leader) cmd[g % kCmdRing] = rec;  // published by the arrive below
+        }
         if (leader) {
           mbar_arrive_expect_tx(&full[st], Lay::kKVBytes);
           for (int c = 0; c < Lay::kChunks; ++c)
@@ -484,9 +504,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           atomicOr(a.status, kDevTimeout);
       }
       __syncwarp();
+      if (isk && ok) {
+        // End of the merged order: an end record, published through the next
+        // stage's full barrier once that stage is free (a plain arrival, no
+        // bytes).  It comes after the drain above, whose waits name the
+        // phases of the last copies.
+        const int st = g % kStages;
+        if (g >= kStages)
+          ok = __all_sync(0xffffffffu, mbar_wait(&empty[st], ((g / kStages) - 1) & 1, &abort_sh,
+                                                 a.status, kWaitLimitNs));
+        if (ok && leader) {
+          cmd[g % kCmdRing] = kCmdEnd;
+          mbar_arrive(&full[st]);
+        }
+        if (!ok && leader) raise_timeout(&abort_sh, a.status);
+      }
     }
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA
+    // Steps come as records in the merged order.  S of step s may be issued
+    // once the PV product of its stream's previous step has been (the two
+    // share S_t's columns); at most two S products run ahead of the PVs.
     {
       const bool leader = elect_one_sync();
       constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, false);
@@ -497,41 +535,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dq = smem_desc_sw128(smem_u32(dsm + Lay::kOffQ), 16, 1024);
       const uint64_t dk = smem_desc_sw128(smem_u32(dsm + Lay::kOffK), 16, 1024);
       const uint64_t dv = smem_desc_sw128(smem_u32(dsm + Lay::kOffV), Lay::kChunkRowsKV, 1024);
-      Cursor C;
-      C.init();
-      int qw0 = 0, qw1 = 0;  // Q tiles consumed per stream
-      int gs = 0;            // S products issued: K ring position
-      int gv = 0;            // PV products issued: V ring position
+      int nq0 = 0, nq1 = 0;  // Q tiles consumed per stream
       int np0 = 0, np1 = 0;  // PV products issued per stream
-      // a stream's pending step: its S issued, its PV not yet (at most one each)
-      bool pend0 = false, pend1 = false;
-      bool first0 = false, first1 = false, last0 = false, last1 = false;
-      int slot0 = 0, slot1 = 0;
-      int oldest = -1;  // stream of the older pending step
+      int p = 0;             // next PV (merged position)
+      int s = 0;             // next S (merged position)
+      bool s_end = false;    // the end record has been read
+      uint32_t s_rec = 0;    // record of step s, once read
+      bool s_read = false;
       bool ok = true;
-      auto pending = [&](int t) { return t ? pend1 : pend0; };
-      auto on_open = [&](int t) -> bool {
-        const int n = t ? qw1 : qw0;
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(&bars.q_full[t], n & 1, &abort_sh, a.status, kWaitLimitNs)))
-          return false;
-        if (t)
-          ++qw1;
-        else
-          ++qw0;
-        return true;
-      };
-      // S for the next step of the merged order if its stream has no pending
-      // step: 1 issued, 0 not now (or nothing left), -2 timeout.
-      auto try_issue_s = [&]() -> int {
-        const int t = peek(C, pending, on_open);
-        if (t == -2) return -2;
-        if (t < 0 || pending(t)) return 0;
-        const int jj = C.take(t);
-        const int st = gs % kStages;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.kfull[st], (gs / kStages) & 1, &abort_sh,
-                                                a.status, kWaitLimitNs)))
-          return -2;
+      // Issues S of step s if its record allows it now: 1 issued, 0 not now.
+      auto try_s = [&]() -> int {
+        if (s_end || s >= p + 2) return 0;
+        const int st = s % kStages;
+        if (!s_read) {
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.kfull[st], (s / kStages) & 1,
+                                                       &abort_sh, a.status, kWaitLimitNs))))
+            return 0;
+          s_rec = cmd[s % kCmdRing];
+          s_read = true;
+          if (s_rec & kCmdEnd) {
+            s_end = true;
+            return 0;
+          }
+        }
+        const int gap = (int)((s_rec >> 4) & 3u);
+        if (gap > 0 && s - gap >= p) return 0;  // that stream's PV is not issued yet
+        const int t = (int)(s_rec & 1u);
+        if (s_rec & 2u) {  // first step of an item: its Q tile
+          const int n = t ? nq1 : nq0;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.q_full[t], n & 1, &abort_sh,
+                                                       a.status, kWaitLimitNs))))
+            return 0;
+          if (t)
+            ++nq1;
+          else
+            ++nq0;
+        }
         tc_fence_after();
         const uint64_t ad0 = dq + (uint64_t)((t * Lay::kQBytes) >> 4);
         const uint64_t bd0 = dk + (uint64_t)((st * Lay::kKVBytes) >> 4);
@@ -543,48 +582,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t offk = (uint64_t)(((kk / 4) * Lay::kChunkRowsKV + (kk % 4) * 32) >> 4);
           if (leader) mma_bf16_ss(dcol, ad0 + offq, bd0 + offk, idS, kk > 0 ? 1u : 0u);
         }
-        const bool last = C.at_end(t);
         if (leader) {
           tc_commit(&bars.kempty[st]);
           tc_commit(&bars.s_full[t]);
-          if (last) tc_commit(&bars.q_empty[t]);
+          if (s_rec & 4u) tc_commit(&bars.q_empty[t]);
         }
-        ++gs;
-        const int slot = C.k(t) % kSlots;
-        if (t) {
-          pend1 = true;
-          first1 = jj == 0;
-          last1 = last;
-          slot1 = slot;
-        } else {
-          pend0 = true;
-          first0 = jj == 0;
-          last0 = last;
-          slot0 = slot;
-        }
-        if (oldest < 0) oldest = t;
+        ++s;
+        s_read = false;
         return 1;
       };
-      int r;
-      while ((r = try_issue_s()) == 1) {
+      while (ok && try_s() == 1) {
       }
-      if (r == -2) ok = false;
-      while (ok && oldest >= 0) {
-        // O_t += P_t V for the older pending step
-        const int t = oldest;
+      while (ok && p < s) {
+        // O_t += P_t V for step p
+        const uint32_t rec = cmd[p % kCmdRing];
+        const int t = (int)(rec & 1u);
         const int np = t ? np1 : np0;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.p_full[t], np & 1, &abort_sh,
                                                      a.status, kWaitLimitNs))))
           break;
-        const int st = gv % kStages;
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.vfull[st], (gv / kStages) & 1,
+        const int st = p % kStages;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.vfull[st], (p / kStages) & 1,
                                                      &abort_sh, a.status, kWaitLimitNs))))
           break;
         tc_fence_after();
         const uint64_t bd0 = dv + (uint64_t)((st * Lay::kKVBytes) >> 4);
         const uint32_t pcol = tmem + col_s(t);
         const uint32_t ocol = tmem + col_o(t);
-        const bool first = t ? first1 : first0;
+        const bool first = (rec & 2u) != 0;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           // keys [16 kk, 16 kk + 16): V rows 16 kk.. (128 bytes each); P elements
@@ -593,23 +618,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16_ts(ocol, pcol + 8 * kk, bd0 + (uint64_t)((kk * 16 * 128) >> 4), idPV,
                         (!first || kk > 0) ? 1u : 0u);
         }
-        if (leader) tc_commit(&bars.vempty[st]);
-        ++gv;
-        if (t) {
+        if (leader) {
+          tc_commit(&bars.vempty[st]);
+          if (rec & 4u) {
+            tc_commit(&bars.o_full[t]);
+            mbar_arrive(&bars.list_empty[t][(rec >> 3) & 1u]);
+          }
+        }
+        ++p;
+        if (t)
           ++np1;
-          pend1 = false;
-        } else {
+        else
           ++np0;
-          pend0 = false;
+        while (ok && try_s() == 1) {
         }
-        oldest = pending(t ^ 1) ? (t ^ 1) : -1;
-        if ((t ? last1 : last0) && leader) {
-          tc_commit(&bars.o_full[t]);
-          mbar_arrive(&bars.list_empty[t][t ? slot1 : slot0]);
-        }
-        while ((r = try_issue_s()) == 1) {
-        }
-        if (r == -2) ok = false;
       }
       if (leader) {
         if (!ok) raise_timeout(&abort_sh, a.status);
@@ -661,18 +683,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(scol + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
         tmem_ld32(scol + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
         tmem_wait_ld();
+        // tile maxima of the two 64-column halves (three-input max)
         float mh[2];
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+          const int x0 = 64 * hf;
+          float m0 = __uint_as_float(r[x0]), m1 = __uint_as_float(r[x0 + 1]);
 #pragma unroll
-          for (int x = 64 * hf; x < 64 * hf + 64; x += 4) {
-            m0 = fmaxf(m0, __uint_as_float(r[x]));
-            m1 = fmaxf(m1, __uint_as_float(r[x + 1]));
-            m2 = fmaxf(m2, __uint_as_float(r[x + 2]));
-            m3 = fmaxf(m3, __uint_as_float(r[x + 3]));
+          for (int x = x0 + 2; x < x0 + 62; x += 4) {
+            m0 = max3f(m0, __uint_as_float(r[x]), __uint_as_float(r[x + 1]));
+            m1 = max3f(m1, __uint_as_float(r[x + 2]), __uint_as_float(r[x + 3]));
           }
-          mh[hf] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+          mh[hf] = max3f(m0, m1, fmaxf(__uint_as_float(r[x0 + 62]), __uint_as_float(r[x0 + 63])));
         }
         const float mt = fmaxf(keep0 ? mh[0] : -INFINITY, keep1 ? mh[1] : -INFINITY) * sl2;
         const bool raise = mt > m + 8.0f;
@@ -699,8 +721,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P = exp2(S * scale * log2e - m) on a kept half, 0 otherwise (a kept
         // half always has a finite reference here: its own maximum raised it);
         // bf16 pairs over S_t's first 64 columns; l sums the rounded weights
-        const float nm = -m;
-        float rs = 0.f, rx = 0.f;
+        // (pair arithmetic packed: x = s * scale_log2 - m, row sums)
+        const uint64_t sl2x2 = pack2(sl2, sl2), nmx2 = pack2(-m, -m);
+        uint64_t rs2 = pack2(0.f, 0.f), rx2 = pack2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {  // 32 weights -> 16 packed columns at a time
           const bool kp = c < 2 ? keep0 : keep1;
@@ -708,21 +731,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kp) {
 #pragma unroll
             for (int x = 0; x < 32; x += 2) {
-              const float x0 = fmaf(__uint_as_float(r[32 * c + x]), sl2, nm);
-              const float x1 = fmaf(__uint_as_float(r[32 * c + x + 1]), sl2, nm);
+              const float2 xv = unpack2(fma2(
+                  pack2(__uint_as_float(r[32 * c + x]), __uint_as_float(r[32 * c + x + 1])), sl2x2,
+                  nmx2));
               float p0, p1;
               if ((x & 7) < 8 - kPolyPer8) {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
+                p0 = ex2_approx(xv.x);
+                p1 = ex2_approx(xv.y);
               } else {
-                const float2 e = exp2_poly2(x0, x1);
+                const float2 e = exp2_poly2(xv.x, xv.y);
                 p0 = e.x;
                 p1 = e.y;
               }
               __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
               const uint32_t u = *reinterpret_cast<uint32_t*>(&pk);
-              rs += __uint_as_float(u << 16) + __uint_as_float(u & 0xFFFF0000u);
-              if constexpr (kLse) rx += p0 + p1;
+              rs2 = add2(rs2, pack2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
+              if constexpr (kLse) rx2 = add2(rx2, pack2(p0, p1));
               pw[x / 2] = u;
             }
           } else {
@@ -731,8 +755,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st16(scol + 16 * c, pw);
         }
-        l += rs;
-        lx += rx;
+        {
+          const float2 a2 = unpack2(rs2), b2 = unpack2(rx2);
+          l += a2.x + a2.y;
+          lx += b2.x + b2.y;
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

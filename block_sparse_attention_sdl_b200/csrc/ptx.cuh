@@ -347,6 +347,13 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
   return d;
 }
 
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // exp2_poly on a pair, with the pair arithmetic packed (see exp2_poly).
 __device__ __forceinline__ float2 exp2_poly2(float x0, float x1) {
   const uint64_t x = pack2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
