@@ -174,6 +174,16 @@ def barrier(dist_on):
         dist.barrier()
 
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Seed of the independent sequence a rank runs (weak scaling over sequences)."""
+    return seed + rank
+
+
+def job_rate(flop_per_step: float, n_steps: int, world: int, ms_max: float) -> float:
+    """Whole-job TFLOP/s: every rank's steps over the slowest rank's device time."""
+    return flop_per_step * n_steps * world / (ms_max * 1e-3) / 1e12
+
+
 def max_over_ranks(x, dist_on, device):
     if not dist_on:
         return x
@@ -366,7 +376,7 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     w = synth.WORKLOADS[args.workload]
-    seed = args.seed + rank  # each rank: its own independent sequence
+    seed = rank_seed(args.seed, rank)  # each rank: its own independent sequence
     runner = Runner(w, seed, device)
     if args.profile:
         profile_kernel(runner, args)
@@ -390,7 +400,7 @@ def main():
     pk, pk_kind = peaks()
     budget = runner.att.budget
     flop_step = 4.0 * w.bs * w.bs * w.d * budget
-    value = flop_step * len(steps) * world / (ms_max * 1e-3) / 1e12
+    value = job_rate(flop_step, len(steps), world, ms_max)
     sparse_ms = [a.elapsed_time(b) for a, b in zip(ev["s0"], ev["s1"])]
     anchor_ms = [a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])]
     sp_avg = statistics.mean(sparse_ms)
@@ -437,7 +447,7 @@ def main():
     if not args.no_e2e:
         e_ms, bi, bo = e2e_measure(runner, inputs, steps, device)
         e_ms = max_over_ranks(e_ms, dist_on, device)
-        e2e = {"value": flop_step * len(steps) * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_rate(flop_step, len(steps), world, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e_ms / len(steps)}
 
     cpu = None

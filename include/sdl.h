@@ -14,8 +14,11 @@
  * Conventions for every call:
  *   - All pointers named q, k, v, o, lse, scores, row_ptr, col_idx, mask_u8
  *     and workspace are DEVICE pointers owned by the caller.  The library
- *     allocates no device memory per call.  It keeps one device status word
- *     and, per device, a small cache of TMA descriptors.
+ *     allocates no device memory per call.  Its own device state is static:
+ *     one status word, the fixed scratch array of sdl_select_mask_noalloc,
+ *     and a ring of 64 tile counters for the attention kernels (each launch
+ *     takes the next one and its last CTA resets it, so at most 64 attention
+ *     launches may be in flight on one device at a time).
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL is the legacy default stream).  Argument errors are returned
  *     before anything is launched; a launch failure returns SDL_ERR_CUDA and
