@@ -162,7 +162,8 @@ class Runner:
         if ev is not None:
             ev["s0"].append(torch.cuda.Event(enable_timing=True))
             ev["s0"][-1].record()
-        self.sdl.sparse_attn(x["q"], x["k"], x["v"], att.row_ptr, att.col_idx, w.bs, out=self.out)
+        self.sdl.sparse_attn(x["q"], x["k"], x["v"], att.row_ptr, att.col_idx, w.bs, out=self.out,
+                             plan=att.plan)
         if ev is not None:
             ev["s1"].append(torch.cuda.Event(enable_timing=True))
             ev["s1"][-1].record()
@@ -209,9 +210,9 @@ def time_steps(runner, inputs, steps, dist_on, device, with_events=True):
     return ms, ev
 
 
-def launches_per_anchor():
-    # pool, score; select: zero, 3 histogram passes, count, scan, write
-    return 2 + 7
+def launches_per_anchor(block: int):
+    # pool, score; select: zero, 3 histogram passes, count, scan, write; tile plan (64-token blocks)
+    return 2 + 7 + (1 if block == 64 else 0)
 
 
 def e2e_measure(runner, inputs, steps, device):
@@ -339,7 +340,8 @@ def profile_kernel(runner, args):
     torch.cuda.synchronize()
     if args.profile == "sparse":
         fn = lambda: sdl.sparse_attn(x["q"], x["k"], x["v"], runner.att.row_ptr,
-                                     runner.att.col_idx, w.bs, out=runner.out)
+                                     runner.att.col_idx, w.bs, out=runner.out,
+                                     plan=runner.att.plan)
         flop = 4.0 * w.bs * w.bs * w.d * runner.att.budget
     else:
         fn = lambda: sdl.dense_attn(x["q"], x["k"], x["v"], out=runner.out)
@@ -483,7 +485,7 @@ def main():
                      "traffic": traffic},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": len(steps) + n_anchor * launches_per_anchor(),
+        "gpu_launches": len(steps) + n_anchor * launches_per_anchor(w.bs),
         "clocks": sampler.summary(),
     }
     if rank == 0:

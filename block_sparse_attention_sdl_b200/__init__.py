@@ -27,7 +27,7 @@ SDL_BF16, SDL_FP32 = 0, 1
 
 EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspace_bytes",
            "sdl_block_scores", "sdl_select_mask", "sdl_select_mask_noalloc", "sdl_sparse_attn",
-           "sdl_dense_attn",
+           "sdl_tile_plan", "sdl_sparse_attn_planned", "sdl_dense_attn",
            "sdl_last_device_status", "sdl_last_cuda_error", "sdl_status_string")
 
 
@@ -70,12 +70,15 @@ def _lib():
         L.sdl_block_scores.argtypes = [P, P, SP, F, P, P, SZ, P]
         L.sdl_select_mask.argtypes = [P, SP, D, P, P, I64, P, P, SZ, P]
         L.sdl_sparse_attn.argtypes = [P, P, P, SP, P, P, F, P, P, P]
+        L.sdl_tile_plan.argtypes = [P, P, SP, P, P]
+        L.sdl_sparse_attn_planned.argtypes = [P, P, P, SP, P, P, P, F, P, P, P]
         L.sdl_dense_attn.argtypes = [P, P, P, SP, F, P, P, P]
         L.sdl_last_device_status.argtypes = [P]
         L.sdl_last_cuda_error.argtypes = []
         L.sdl_status_string.argtypes = [ctypes.c_int]
         L.sdl_status_string.restype = ctypes.c_char_p
-        for f in ("sdl_block_scores", "sdl_select_mask", "sdl_sparse_attn", "sdl_dense_attn",
+        for f in ("sdl_block_scores", "sdl_select_mask", "sdl_sparse_attn", "sdl_tile_plan",
+                  "sdl_sparse_attn_planned", "sdl_dense_attn",
                   "sdl_last_device_status", "sdl_last_cuda_error"):
             getattr(L, f).restype = ctypes.c_int
         _L = L
@@ -191,19 +194,42 @@ def select_mask(scores, sparsity: float, block: int, L: int, row_ptr=None, col_i
     return row_ptr, col_idx, mask
 
 
+def tile_plan(row_ptr, col_idx, B: int, H: int, L: int, block: int = 64, plan=None,
+              stream=None):
+    """int32 [B, H, ceil(nb/2), 2] tile plan for 64-token blocks (see ``sdl_tile_plan``)."""
+    import torch
+    nb = L // block
+    s = Shape()
+    s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, H, L, 64, block, SDL_BF16
+    if plan is None:
+        plan = torch.empty((B, H, (nb + 1) // 2, 2), dtype=torch.int32, device=row_ptr.device)
+    _check(_lib().sdl_tile_plan(row_ptr.data_ptr(), col_idx.data_ptr(), ctypes.byref(s),
+                                plan.data_ptr(), _stream(stream)), "sdl_tile_plan")
+    return plan
+
+
 def sparse_attn(q, k, v, row_ptr, col_idx, block: int, scale: float = 0.0, out=None, lse=None,
-                want_lse: bool = False, stream=None):
-    """O like q (and LSE fp32 [B,H,L] when asked) over the kept blocks."""
+                want_lse: bool = False, plan=None, stream=None):
+    """O like q (and LSE fp32 [B,H,L] when asked) over the kept blocks; ``plan`` is an
+    optional tile plan from :func:`tile_plan` (results equal up to fp32 summation order)."""
     import torch
     if out is None:
         out = torch.empty_like(q)
     s = make_shape(q, k, block, v, out)
     if lse is None and want_lse:
         lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
-    _check(_lib().sdl_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(s),
-                                  row_ptr.data_ptr(), col_idx.data_ptr(), float(scale),
-                                  out.data_ptr(), None if lse is None else lse.data_ptr(),
-                                  _stream(stream)), "sdl_sparse_attn")
+    if plan is None:
+        _check(_lib().sdl_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(s),
+                                      row_ptr.data_ptr(), col_idx.data_ptr(), float(scale),
+                                      out.data_ptr(), None if lse is None else lse.data_ptr(),
+                                      _stream(stream)), "sdl_sparse_attn")
+    else:
+        _check(_lib().sdl_sparse_attn_planned(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                              ctypes.byref(s), row_ptr.data_ptr(),
+                                              col_idx.data_ptr(), plan.data_ptr(), float(scale),
+                                              out.data_ptr(),
+                                              None if lse is None else lse.data_ptr(),
+                                              _stream(stream)), "sdl_sparse_attn_planned")
     return (out, lse) if want_lse or lse is not None else out
 
 

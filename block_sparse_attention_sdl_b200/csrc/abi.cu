@@ -94,8 +94,8 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, const sdl_shape& s, int
 }
 
 sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_shape* shape,
-                       const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
-                       float* lse, void* stream) {
+                       const int32_t* row_ptr, const int32_t* col_idx, const int32_t* plan,
+                       float scale, void* o, float* lse, void* stream) {
   sdl_status e = check_shape(shape);
   if (e) return e;
   const sdl_shape& s = *shape;
@@ -115,6 +115,7 @@ sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_sh
   a.lse = lse;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
+  a.plan = (row_ptr && s.block == 64) ? plan : nullptr;
   a.B = s.B;
   a.H = s.H;
   a.Hkv = s.H_kv;
@@ -237,12 +238,33 @@ sdl_status sdl_sparse_attn(const void* q, const void* k, const void* v, const sd
                            const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
                            float* lse, void* stream) {
   if (!row_ptr || !col_idx) return SDL_ERR_INVALID_ARG;
-  return attn_common(q, k, v, shape, row_ptr, col_idx, scale, o, lse, stream);
+  return attn_common(q, k, v, shape, row_ptr, col_idx, nullptr, scale, o, lse, stream);
+}
+
+sdl_status sdl_sparse_attn_planned(const void* q, const void* k, const void* v,
+                                   const sdl_shape* shape, const int32_t* row_ptr,
+                                   const int32_t* col_idx, const int32_t* plan, float scale,
+                                   void* o, float* lse, void* stream) {
+  if (!row_ptr || !col_idx) return SDL_ERR_INVALID_ARG;
+  return attn_common(q, k, v, shape, row_ptr, col_idx, plan, scale, o, lse, stream);
+}
+
+sdl_status sdl_tile_plan(const int32_t* row_ptr, const int32_t* col_idx, const sdl_shape* shape,
+                         int32_t* plan, void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  if (!row_ptr || !col_idx || !plan) return SDL_ERR_INVALID_ARG;
+  if (shape->block != 64) return SDL_ERR_UNSUPPORTED;
+  const cudaError_t ce = launch_plan(row_ptr, col_idx, shape->B, shape->H,
+                                     shape->L / shape->block, plan,
+                                     static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
 }
 
 sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,
                           float scale, void* o, float* lse, void* stream) {
-  return attn_common(q, k, v, shape, nullptr, nullptr, scale, o, lse, stream);
+  return attn_common(q, k, v, shape, nullptr, nullptr, nullptr, scale, o, lse, stream);
 }
 
 sdl_status sdl_last_device_status(void* stream) {

@@ -112,7 +112,8 @@ struct Bars {
 struct Slot {
   int item;  // -1: end of the stream
   int n_ent;
-  int b, h, t0;
+  int b, h;
+  int t0, t1;  // first tokens of the tile's two 64-row halves (L: half unused)
   uint32_t ent[kMaxSub];
 };
 
@@ -181,11 +182,11 @@ __device__ __forceinline__ void raise_timeout(volatile int* abort_flag, int* sta
 
 // Zero output rows (and -inf LSE) of a 128-row tile whose kept list is empty.
 template <int D>
-__device__ __forceinline__ void write_empty_tile(const AttnArgs& a, int b, int h, int t0,
+__device__ __forceinline__ void write_empty_tile(const AttnArgs& a, int b, int h, int t0, int t1,
                                                  int lane) {
   for (int r = lane; r < kBM; r += 32) {
-    const int t = t0 + r;
-    if (t >= a.L) break;
+    const int t = (r < 64 ? t0 : t1) + (r & 63);
+    if (t >= a.L) continue;
     uint4* op = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + b * a.os[0] +
                                          (int64_t)t * a.os[1] + h * a.os[2]);
 #pragma unroll
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         progressed = true;
         Slot& S = slots[t][slot];
         // take items until a non-empty one (or none is left)
-        int item = -1, n_ent = 0, b = 0, h = 0, t0 = 0;
+        int item = -1, n_ent = 0, b = 0, h = 0, t0 = 0, t1 = 0;
         while (!exhausted) {
           unsigned taken = 0;
           if (lane == 0) taken = atomicAdd(&g_sched[sched_slot].next, 1u);
@@ -311,21 +312,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           item = (int)taken;
           b = item / (a.H * n_qt);
           h = (item / n_qt) % a.H;
-          t0 = (item % n_qt) * kBM;
+          if (a.plan != nullptr) {
+            // the tile's two query blocks from the plan (64-token blocks)
+            const int qb0 = a.plan[2 * (int64_t)item], qb1 = a.plan[2 * (int64_t)item + 1];
+            if (qb0 >= a.nb || qb0 < -1 || qb1 >= a.nb || qb1 < -1)
+              atomicOr(a.status, kDevBadMask);
+            t0 = (qb0 >= 0 && qb0 < a.nb) ? qb0 * 64 : a.L;
+            t1 = (qb1 >= 0 && qb1 < a.nb) ? qb1 * 64 : a.L;
+          } else {
+            t0 = (item % n_qt) * kBM;
+            t1 = t0 + 64 < a.L ? t0 + 64 : a.L;
+          }
           // kept 64-token key sub-blocks of the two query halves, as bitmaps
           for (int w = lane; w < kMaxSub / 32; w += 32) bmask[0][w] = bmask[1][w] = 0;
           __syncwarp();
           if (a.row_ptr == nullptr) {
             for (int s = lane; s < nsub; s += 32) {
-              atomicOr(&bmask[0][s / 32], 1u << (s % 32));
-              if (t0 + 64 < a.L) atomicOr(&bmask[1][s / 32], 1u << (s % 32));
+              if (t0 < a.L) atomicOr(&bmask[0][s / 32], 1u << (s % 32));
+              if (t1 < a.L) atomicOr(&bmask[1][s / 32], 1u << (s % 32));
             }
           } else {
             const int per = a.block / kSubBlock;  // sub-blocks per block: 1 or 2
             const int rows_in_tile = a.block == 64 ? 2 : 1;
             for (int rr = 0; rr < rows_in_tile; ++rr) {
-              const int i = t0 / a.block + rr;
-              if (i >= a.nb) break;
+              const int tr = rr ? t1 : t0;
+              if (tr >= a.L) continue;
+              const int i = tr / a.block;
               const int64_t r = ((int64_t)b * a.H + h) * a.nb + i;
               const int beg = a.row_ptr[r], end = a.row_ptr[r + 1];
               for (int x = beg + lane; x < end; x += 32) {
@@ -359,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           n_ent = __shfl_sync(0xffffffffu, incl, 31);
           __syncwarp();
           if (n_ent == 0) {
-            write_empty_tile<D>(a, b, h, t0, lane);
+            write_empty_tile<D>(a, b, h, t0, t1, lane);
             __syncwarp();
             continue;
           }
@@ -382,9 +394,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             S.b = b;
             S.h = h;
             S.t0 = t0;
+            S.t1 = t1;
             // its Q tile is loaded when this stream's previous item is done; warm L2 now
             for (int cc = 0; cc < Lay::kChunks; ++cc)
-              for (int s = 0; s < 2; ++s) tma_prefetch_l2_4d(&tmq, cc * 64, t0 + 64 * s, h, b);
+              for (int s = 0; s < 2; ++s)
+                if ((s ? t1 : t0) < a.L) tma_prefetch_l2_4d(&tmq, cc * 64, s ? t1 : t0, h, b);
           }
         }
         __syncwarp();
@@ -442,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cc = 0; cc < Lay::kChunks; ++cc)
             for (int s = 0; s < 2; ++s)
               tma_load_4d(sq + cc * Lay::kChunkRowsQ + s * kBox, &tmq, &bars.q_full[t], cc * 64,
-                          S.t0 + 64 * s, S.h, S.b);
+                          s ? S.t1 : S.t0, S.h, S.b);
         }
         if (t)
           ++qiss1;
@@ -662,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       const Slot& S = slots[t][slot];
       if (S.item < 0) break;
-      const int n_ent = S.n_ent, b = S.b, h = S.h, tok = S.t0 + row;
+      const int n_ent = S.n_ent, b = S.b, h = S.h, tok = (half ? S.t1 : S.t0) + (row & 63);
       const int n_steps = (n_ent + 1) / 2;
       float m = -INFINITY;  // running max (log2 units) used as the exponent reference
       float l = 0.f;        // row sum of the bf16-rounded weights

@@ -30,6 +30,7 @@ struct AttnArgs {
   float* lse;
   const int32_t* row_ptr;  // null: dense
   const int32_t* col_idx;
+  const int32_t* plan;     // tile plan for 64-token blocks (null: adjacent pairs)
   int B, H, Hkv, L, d, block, nb;
   int64_t qs[3], ks[3], vs[3], os[3];
   float scale_log2;  // scale * log2(e)
@@ -47,5 +48,7 @@ size_t select_workspace_bytes(int B, int H, int nb);
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_plan(const int32_t* row_ptr, const int32_t* col_idx, int B, int H, int nb,
+                        int32_t* plan, cudaStream_t st);
 
 }  // namespace sdl

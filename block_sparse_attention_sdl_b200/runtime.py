@@ -12,7 +12,7 @@ from __future__ import annotations
 import torch
 
 from . import (block_scores, make_shape, mask_budget, scores_workspace_bytes, select_mask,
-               select_workspace_bytes, sparse_attn)
+               select_workspace_bytes, sparse_attn, tile_plan)
 
 
 def is_anchor(step: int, anchor_every: int) -> bool:
@@ -49,6 +49,9 @@ class StepSparseAttention:
                                      device=dev)
         self.row_ptr = torch.empty(B * H * self.nb + 1, dtype=torch.int32, device=dev)
         self.col_idx = torch.empty(self.budget, dtype=torch.int32, device=dev)
+        # 64-token blocks: which two query blocks share a 128-row tile (rebuilt with the mask)
+        self.plan = (torch.empty((B, H, (self.nb + 1) // 2, 2), dtype=torch.int32, device=dev)
+                     if block == 64 else None)
         self.mask_step = None  # anchor step whose mask is current
 
     def refresh(self, q, k, step: int, stream=None):
@@ -56,10 +59,13 @@ class StepSparseAttention:
                      stream=stream)
         select_mask(self.scores, self.sparsity, self.block, self.L, row_ptr=self.row_ptr,
                     col_idx=self.col_idx, workspace=self.ws_select, stream=stream)
+        if self.plan is not None:
+            tile_plan(self.row_ptr, self.col_idx, self.B, self.H, self.L, self.block,
+                      plan=self.plan, stream=stream)
         self.mask_step = step
 
     def __call__(self, q, k, v, step: int, out=None, lse=None, stream=None):
         if is_anchor(step, self.anchor_every) or self.mask_step is None:
             self.refresh(q, k, anchor_of(step, self.anchor_every), stream)
         return sparse_attn(q, k, v, self.row_ptr, self.col_idx, self.block, out=out, lse=lse,
-                           stream=stream)
+                           plan=self.plan, stream=stream)

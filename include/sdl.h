@@ -136,6 +136,30 @@ sdl_status sdl_sparse_attn(const void* q, const void* k, const void* v, const sd
                            const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
                            float* lse, void* stream);
 
+/* Tile plan for 64-token blocks (a scheduling aid with no counterpart in the
+ * abstract): the attention kernels run 128-row tensor-core tiles, each holding
+ * two query blocks and walking the union of their kept lists, so pairing
+ * blocks whose lists overlap saves work.  Writes plan, int32
+ * [B, H, ceil(nb/2), 2] (device, caller-owned): tile p of head (b, h) holds
+ * query blocks plan[..., p, 0] and plan[..., p, 1] (-1 for the single block
+ * left when nb is odd).  Per head, blocks are taken in order of descending
+ * list length (ties: lower index) and each unpaired block is paired with the
+ * unpaired block whose kept list shares the most entries (ties: lower index).
+ * Heads with more than 256 blocks get adjacent pairs.  Only block == 64;
+ * other block sizes return SDL_ERR_UNSUPPORTED. */
+sdl_status sdl_tile_plan(const int32_t* row_ptr, const int32_t* col_idx, const sdl_shape* shape,
+                         int32_t* plan, void* stream);
+
+/* sdl_sparse_attn with a tile plan from sdl_tile_plan (NULL: adjacent pairs,
+ * which is what sdl_sparse_attn uses).  Same results up to fp32 summation
+ * order.  The plan must pair every query block of every head exactly once;
+ * entries outside [0, nb) are skipped and reported as SDL_ERR_BAD_MASK.  Used
+ * for bf16 with block == 64 only (fp32 and 128-token blocks ignore it). */
+sdl_status sdl_sparse_attn_planned(const void* q, const void* k, const void* v,
+                                   const sdl_shape* shape, const int32_t* row_ptr,
+                                   const int32_t* col_idx, const int32_t* plan, float scale,
+                                   void* o, float* lse, void* stream);
+
 /* Dense bidirectional attention, the baseline of the same abstract: the
  * sparse call with every block of every row kept. */
 sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,

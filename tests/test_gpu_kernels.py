@@ -228,6 +228,83 @@ def test_sparse_attention_many_tiles_per_cta(bs, density):
     assert np.abs(lg - lw).max() <= TOL["bf16"]["lse"]
 
 
+def _greedy_plan(M):
+    """The tile-plan rule restated: blocks by descending list length (ties: lower
+    index), each unpaired block paired with the unpaired block of largest list
+    intersection (ties: lower index); adjacent pairs above 256 blocks."""
+    nb = M.shape[0]
+    n_qt = (nb + 1) // 2
+    if nb > 256:
+        return np.array([[2 * p, 2 * p + 1 if 2 * p + 1 < nb else -1] for p in range(n_qt)])
+    ln = M.sum(1)
+    ov = (M[:, None, :].astype(np.int64) & M[None, :, :]).sum(-1)
+    used = np.zeros(nb, bool)
+    pairs = []
+    for i in sorted(range(nb), key=lambda i: (-ln[i], i)):
+        if used[i]:
+            continue
+        used[i] = True
+        cand = [j for j in range(nb) if not used[j]]
+        best = max(cand, key=lambda j: (ov[i, j], -j)) if cand else -1
+        if best >= 0:
+            used[best] = True
+        pairs.append((i, best))
+    return np.array(pairs)
+
+
+@pytest.mark.parametrize("nb,density", [(9, 0.4), (32, 0.2), (128, 0.1), (300, 0.05)])
+def test_tile_plan_follows_the_greedy_rule(nb, density):
+    B, H = 1, 3
+    rng = np.random.default_rng(nb)
+    mask = _random_mask(B, H, nb, density, rng)
+    rp, ci = _mask_to_csr(mask)
+    plan = sdl.tile_plan(rp, ci, B, H, nb * 64, 64).cpu().numpy()
+    for h in range(H):
+        want = _greedy_plan(mask[0, h].astype(bool))
+        assert np.array_equal(plan[0, h], want), h
+        got = plan[0, h].ravel()
+        assert sorted(got[got >= 0].tolist()) == list(range(nb))  # every block exactly once
+
+
+@pytest.mark.parametrize("L,H,Hkv,density,kind", [(1024, 4, 2, 0.3, "greedy"),
+                                                 (1088, 3, 1, 0.25, "random"),
+                                                 (2048, 2, 2, 0.15, "random")])
+def test_sparse_attention_with_tile_plan(L, H, Hkv, density, kind):
+    """Any pairing of query blocks into tiles gives the oracle's result."""
+    w = synth.small_workload(L=L, H=H, H_kv=Hkv, d=128, bs=64)
+    host, dev = _inputs(w)
+    nb = L // 64
+    rng = np.random.default_rng(L + H)
+    mask = _random_mask(1, H, nb, density, rng)
+    rp, ci = _mask_to_csr(mask)
+    if kind == "greedy":
+        plan = sdl.tile_plan(rp, ci, 1, H, L, 64)
+    else:
+        n_qt = (nb + 1) // 2
+        pl = np.full((1, H, n_qt, 2), -1, np.int32)
+        for h in range(H):
+            perm = rng.permutation(nb)
+            flat = np.full(2 * n_qt, -1)
+            flat[:nb] = perm
+            pl[0, h] = flat.reshape(n_qt, 2)
+        plan = torch.from_numpy(pl).cuda()
+    O, lse = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, want_lse=True, plan=plan)
+    assert sdl.last_device_status() == sdl.SDL_OK
+    Ow, lw = oracle.attention(host["q"], host["k"], host["v"], 64, mask=mask)
+    check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, "bf16")
+    assert np.abs(lse.cpu().numpy() - lw).max() <= TOL["bf16"]["lse"]
+
+
+def test_bad_tile_plan_entry_is_reported():
+    w = synth.small_workload(L=256, H=1, H_kv=1, d=128)
+    _, dev = _inputs(w)
+    mask = np.ones((1, 1, 4, 4), np.uint8)
+    rp, ci = _mask_to_csr(mask)
+    plan = torch.tensor([[[[0, 1], [2, 77]]]], dtype=torch.int32, device="cuda")  # 77 >= nb
+    sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, plan=plan)
+    assert sdl.last_device_status() == sdl.SDL_ERR_BAD_MASK
+
+
 def test_repeated_launches_on_two_streams_are_identical():
     """The attention kernel's CTAs take tiles from a per-launch counter that the
     last CTA resets; 150 launches, alternating over two streams, must all give
