@@ -55,6 +55,14 @@ def parse():
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--variant", choices=["step-dllm", "uniform-head", "sparsed"],
+                   default="step-dllm",
+                   help="step-dllm: head-adaptive global budget, mask refreshed every anchor "
+                        "interval (the headline); uniform-head: the same schedule with a "
+                        "uniform per-head budget; sparsed: dense attention for the first "
+                        "--dense-steps steps, then one mask reused for every later step")
+    p.add_argument("--dense-steps", type=int, default=32,
+                   help="dense warm-up steps of the sparsed variant")
     p.add_argument("--profile", choices=["sparse", "dense"], default=None,
                    help="launch only this attention kernel (warmup + steps times, one input) "
                         "and print its event-timed average; for profiler captures")
@@ -136,34 +144,46 @@ class ClockSampler:
 class Runner:
     """The library's step loop over per-step device inputs, with per-launch events."""
 
-    def __init__(self, w, seed, device):
+    def __init__(self, w, seed, device, variant="step-dllm", dense_steps=0):
         import block_sparse_attention_sdl_b200 as sdl
-        from block_sparse_attention_sdl_b200.runtime import StepSparseAttention
-        self.sdl, self.w = sdl, w
-        self.att = StepSparseAttention(w.B, w.H, w.H_kv, w.L, w.d, w.bs, w.sparsity,
-                                       w.anchor_every, device=device)
+        from block_sparse_attention_sdl_b200 import runtime
+        self.sdl, self.w, self.rt = sdl, w, runtime
+        sparsed = variant == "sparsed"
+        self.interval = None if sparsed else w.anchor_every
+        self.dense_steps = dense_steps if sparsed else 0
+        self.att = runtime.StepSparseAttention(
+            w.B, w.H, w.H_kv, w.L, w.d, w.bs, w.sparsity, self.interval, device=device,
+            budget="head" if variant == "uniform-head" else "sequence",
+            dense_steps=self.dense_steps)
         self.out = torch.empty((w.B, w.L, w.H, w.d), dtype=torch.bfloat16, device=device)
         self.seed = seed
+        self.kinds = []  # per attention launch: "sparse" or "dense"
 
     def make_inputs(self, steps):
         import synth
         return [synth.device_inputs(self.w, s, self.seed) for s in steps]
 
     def step(self, x, s, ev=None):
-        att, w = self.att, self.w
-        if s % w.anchor_every == 0 or att.mask_step is None:
+        att, w, rt = self.att, self.w, self.rt
+        dense = rt.is_dense(s, self.dense_steps)
+        if not dense and (rt.is_anchor(s, self.interval, self.dense_steps) or
+                          att.mask_step is None):
             if ev is not None:
                 ev["a0"].append(torch.cuda.Event(enable_timing=True))
                 ev["a0"][-1].record()
-            att.refresh(x["q"], x["k"], s)
+            att.refresh(x["q"], x["k"], rt.anchor_of(s, self.interval, self.dense_steps))
             if ev is not None:
                 ev["a1"].append(torch.cuda.Event(enable_timing=True))
                 ev["a1"][-1].record()
         if ev is not None:
             ev["s0"].append(torch.cuda.Event(enable_timing=True))
             ev["s0"][-1].record()
-        self.sdl.sparse_attn(x["q"], x["k"], x["v"], att.row_ptr, att.col_idx, w.bs, out=self.out,
-                             plan=att.plan)
+            self.kinds.append("dense" if dense else "sparse")
+        if dense:
+            self.sdl.dense_attn(x["q"], x["k"], x["v"], w.bs, out=self.out)
+        else:
+            self.sdl.sparse_attn(x["q"], x["k"], x["v"], att.row_ptr, att.col_idx, w.bs,
+                                 out=self.out, plan=att.plan)
         if ev is not None:
             ev["s1"].append(torch.cuda.Event(enable_timing=True))
             ev["s1"][-1].record()
@@ -379,7 +399,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     w = synth.WORKLOADS[args.workload]
     seed = rank_seed(args.seed, rank)  # each rank: its own independent sequence
-    runner = Runner(w, seed, device)
+    runner = Runner(w, seed, device, args.variant, args.dense_steps)
     if args.profile:
         profile_kernel(runner, args)
         return
@@ -402,10 +422,17 @@ def main():
     pk, pk_kind = peaks()
     budget = runner.att.budget
     flop_step = 4.0 * w.bs * w.bs * w.d * budget
-    value = job_rate(flop_step, len(steps), world, ms_max)
-    sparse_ms = [a.elapsed_time(b) for a, b in zip(ev["s0"], ev["s1"])]
+    dense_flop = 4.0 * w.B * w.H * w.L * w.L * w.d
+    kinds = runner.kinds[-len(steps):]
+    n_dense_steps = kinds.count("dense")
+    # algorithmic work of the timed steps: kept blocks on sparse steps, L^2 on dense ones
+    value = job_rate((flop_step * (len(steps) - n_dense_steps) + dense_flop * n_dense_steps) /
+                     len(steps), len(steps), world, ms_max)
+    attn_ms = [a.elapsed_time(b) for a, b in zip(ev["s0"], ev["s1"])]
+    sparse_ms = [t for t, k in zip(attn_ms, kinds) if k == "sparse"]
     anchor_ms = [a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])]
     sp_avg = statistics.mean(sparse_ms)
+    sp_q = statistics.quantiles(sparse_ms, n=10) if len(sparse_ms) > 1 else [sp_avg] * 9
     kernel_tflops = flop_step / (sp_avg * 1e-3) / 1e12
     peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
 
@@ -429,7 +456,7 @@ def main():
                                              workspace=att.ws_scores))
     se_ms = ev_time(lambda: sdl.select_mask(att.scores, w.sparsity, w.bs, w.L,
                                             row_ptr=att.row_ptr, col_idx=att.col_idx,
-                                            workspace=att.ws_select))
+                                            workspace=att.ws_select, per_head=att.per_head))
     score_bytes = 2 * w.B * w.L * (w.H + w.H_kv) * w.d + 4 * w.B * w.H * w.nb * w.nb
     # dense baseline on distinct inputs per launch (larger than L2 in total)
     de = []
@@ -467,10 +494,15 @@ def main():
                 "per step)",
         "config": {"workload": args.workload, "global_batch": w.B * world, "seq_len": w.L,
                    "heads": w.H, "kv_heads": w.H_kv, "head_dim": w.d, "block": w.bs,
-                   "sparsity": w.sparsity, "anchor_every": w.anchor_every,
+                   "sparsity": w.sparsity, "anchor_every": runner.interval,
+                   "dense_steps": runner.dense_steps,
+                   "budget": "per head" if runner.att.per_head else "per sequence, across heads",
                    "parallelism": f"independent sequences x{world}",
                    "l2": "inputs larger than L2 (192 MiB per step, distinct per step)"},
+        "variant": args.variant,
         "sparse_attn_ms": sp_avg, "sparse_attn_tflops": kernel_tflops,
+        "sparse_attn_ms_p10_p50_p90": [sp_q[0], statistics.median(sparse_ms), sp_q[-1]],
+        "dense_steps_timed": n_dense_steps,
         "pct_bf16_peak": kernel_tflops / peak,
         "dense_attn_ms": dense_ms, "dense_attn_tflops": dense_flop / (dense_ms * 1e-3) / 1e12,
         "speedup_vs_dense": dense_ms / sp_avg,

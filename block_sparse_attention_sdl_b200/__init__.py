@@ -26,6 +26,7 @@ SDL_ERR_WORKSPACE, SDL_ERR_CUDA, SDL_ERR_TIMEOUT, SDL_ERR_BAD_MASK = 4, 5, 6, 7
 SDL_BF16, SDL_FP32 = 0, 1
 
 EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspace_bytes",
+           "sdl_mask_budget_scoped", "sdl_select_workspace_bytes_scoped", "sdl_select_mask_scoped",
            "sdl_block_scores", "sdl_select_mask", "sdl_select_mask_noalloc", "sdl_sparse_attn",
            "sdl_tile_plan", "sdl_sparse_attn_planned", "sdl_dense_attn",
            "sdl_last_device_status", "sdl_last_cuda_error", "sdl_status_string")
@@ -67,6 +68,11 @@ def _lib():
         L.sdl_scores_workspace_bytes.restype = SZ
         L.sdl_select_workspace_bytes.argtypes = [SP]
         L.sdl_select_workspace_bytes.restype = SZ
+        L.sdl_mask_budget_scoped.argtypes = [SP, D, ctypes.c_int]
+        L.sdl_mask_budget_scoped.restype = I64
+        L.sdl_select_workspace_bytes_scoped.argtypes = [SP, ctypes.c_int]
+        L.sdl_select_workspace_bytes_scoped.restype = SZ
+        L.sdl_select_mask_scoped.argtypes = [P, SP, D, ctypes.c_int, P, P, I64, P, P, SZ, P]
         L.sdl_block_scores.argtypes = [P, P, SP, F, P, P, SZ, P]
         L.sdl_select_mask.argtypes = [P, SP, D, P, P, I64, P, P, SZ, P]
         L.sdl_sparse_attn.argtypes = [P, P, P, SP, P, P, F, P, P, P]
@@ -77,7 +83,8 @@ def _lib():
         L.sdl_last_cuda_error.argtypes = []
         L.sdl_status_string.argtypes = [ctypes.c_int]
         L.sdl_status_string.restype = ctypes.c_char_p
-        for f in ("sdl_block_scores", "sdl_select_mask", "sdl_sparse_attn", "sdl_tile_plan",
+        for f in ("sdl_block_scores", "sdl_select_mask", "sdl_select_mask_scoped",
+                  "sdl_sparse_attn", "sdl_tile_plan",
                   "sdl_sparse_attn_planned", "sdl_dense_attn",
                   "sdl_last_device_status", "sdl_last_cuda_error"):
             getattr(L, f).restype = ctypes.c_int
@@ -132,7 +139,14 @@ def _stream(stream):
     return stream.cuda_stream
 
 
-def mask_budget(shape: Shape, sparsity: float) -> int:
+SDL_BUDGET_SEQUENCE, SDL_BUDGET_HEAD = 0, 1
+
+
+def mask_budget(shape: Shape, sparsity: float, per_head: bool = False) -> int:
+    """Kept blocks of a call: head-adaptive budget per sequence, or uniform per head."""
+    if per_head:
+        return int(_lib().sdl_mask_budget_scoped(ctypes.byref(shape), float(sparsity),
+                                                 SDL_BUDGET_HEAD))
     return int(_lib().sdl_mask_budget(ctypes.byref(shape), float(sparsity)))
 
 
@@ -140,7 +154,9 @@ def scores_workspace_bytes(shape: Shape) -> int:
     return int(_lib().sdl_scores_workspace_bytes(ctypes.byref(shape)))
 
 
-def select_workspace_bytes(shape: Shape) -> int:
+def select_workspace_bytes(shape: Shape, per_head: bool = False) -> int:
+    if per_head:
+        return int(_lib().sdl_select_workspace_bytes_scoped(ctypes.byref(shape), SDL_BUDGET_HEAD))
     return int(_lib().sdl_select_workspace_bytes(ctypes.byref(shape)))
 
 
@@ -167,15 +183,17 @@ def block_scores(q, k, block: int, scale: float = 0.0, scores=None, workspace=No
 
 
 def select_mask(scores, sparsity: float, block: int, L: int, row_ptr=None, col_idx=None,
-                mask=None, want_mask: bool = False, workspace=None, stream=None):
-    """(row_ptr int32 [B*H*nb+1], col_idx int32 [budget], mask uint8 or None)."""
+                mask=None, want_mask: bool = False, workspace=None, per_head: bool = False,
+                stream=None):
+    """(row_ptr int32 [B*H*nb+1], col_idx int32 [budget], mask uint8 or None); ``per_head``
+    takes a uniform budget per head instead of the head-adaptive one per sequence."""
     import torch
     B, H, nb, _ = scores.shape
     s = Shape()
     s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, H, L, 64, block, SDL_FP32
     if nb != L // block:
         raise ValueError("scores shape does not match L / block")
-    total = mask_budget(s, sparsity)
+    total = mask_budget(s, sparsity, per_head)
     if total < 0:
         raise SdlError(SDL_ERR_INVALID_ARG, "sdl_mask_budget")
     dev = scores.device
@@ -185,12 +203,19 @@ def select_mask(scores, sparsity: float, block: int, L: int, row_ptr=None, col_i
         col_idx = torch.empty(total, dtype=torch.int32, device=dev)
     if mask is None and want_mask:
         mask = torch.empty((B, H, nb, nb), dtype=torch.uint8, device=dev)
-    workspace = _workspace(select_workspace_bytes(s), dev, workspace)
-    _check(_lib().sdl_select_mask(scores.data_ptr(), ctypes.byref(s), float(sparsity),
-                                  row_ptr.data_ptr(), col_idx.data_ptr(), col_idx.numel(),
-                                  None if mask is None else mask.data_ptr(),
-                                  workspace.data_ptr(), workspace.numel(), _stream(stream)),
-           "sdl_select_mask")
+    workspace = _workspace(select_workspace_bytes(s, per_head), dev, workspace)
+    mask_ptr = None if mask is None else mask.data_ptr()
+    if per_head:
+        _check(_lib().sdl_select_mask_scoped(scores.data_ptr(), ctypes.byref(s), float(sparsity),
+                                             SDL_BUDGET_HEAD, row_ptr.data_ptr(),
+                                             col_idx.data_ptr(), col_idx.numel(), mask_ptr,
+                                             workspace.data_ptr(), workspace.numel(),
+                                             _stream(stream)), "sdl_select_mask_scoped")
+    else:
+        _check(_lib().sdl_select_mask(scores.data_ptr(), ctypes.byref(s), float(sparsity),
+                                      row_ptr.data_ptr(), col_idx.data_ptr(), col_idx.numel(),
+                                      mask_ptr, workspace.data_ptr(), workspace.numel(),
+                                      _stream(stream)), "sdl_select_mask")
     return row_ptr, col_idx, mask
 
 

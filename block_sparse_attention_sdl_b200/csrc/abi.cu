@@ -190,6 +190,23 @@ size_t sdl_select_workspace_bytes(const sdl_shape* shape) {
   return select_workspace_bytes(shape->B, shape->H, shape->L / shape->block);
 }
 
+size_t sdl_select_workspace_bytes_scoped(const sdl_shape* shape, int scope) {
+  if (scope == SDL_BUDGET_SEQUENCE) return sdl_select_workspace_bytes(shape);
+  if (scope != SDL_BUDGET_HEAD || check_shape(shape) != SDL_OK) return 0;
+  // every head is its own single-head sequence
+  return select_workspace_bytes(shape->B * shape->H, 1, shape->L / shape->block);
+}
+
+int64_t sdl_mask_budget_scoped(const sdl_shape* shape, double sparsity, int scope) {
+  if (scope == SDL_BUDGET_SEQUENCE) return sdl_mask_budget(shape, sparsity);
+  if (scope != SDL_BUDGET_HEAD || check_shape(shape) != SDL_OK) return -1;
+  if (!(sparsity >= 0.0 && sparsity < 1.0)) return -1;
+  const int64_t nb = shape->L / shape->block;
+  const int64_t kb = (int64_t)floor((1.0 - sparsity) * (double)nb * (double)nb + 0.5);
+  if (kb < nb) return -1;
+  return kb * shape->B * shape->H;
+}
+
 sdl_status sdl_block_scores(const void* q, const void* k, const sdl_shape* shape, float scale,
                             float* scores, void* workspace, size_t workspace_bytes,
                             void* stream) {
@@ -230,6 +247,32 @@ sdl_status sdl_select_mask(const float* scores, const sdl_shape* shape, double s
   const int nb = shape->L / shape->block;
   cudaError_t ce = launch_select(scores, shape->B, shape->H, nb, total / shape->B, row_ptr,
                                  col_idx, mask_u8, workspace, static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_select_mask_scoped(const float* scores, const sdl_shape* shape, double sparsity,
+                                  int scope, int32_t* row_ptr, int32_t* col_idx,
+                                  int64_t col_capacity, uint8_t* mask_u8, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (scope == SDL_BUDGET_SEQUENCE)
+    return sdl_select_mask(scores, shape, sparsity, row_ptr, col_idx, col_capacity, mask_u8,
+                           workspace, workspace_bytes, stream);
+  if (scope != SDL_BUDGET_HEAD) return SDL_ERR_INVALID_ARG;
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  if (!scores || !row_ptr || !col_idx) return SDL_ERR_INVALID_ARG;
+  if (!aligned16(scores)) return SDL_ERR_INVALID_ARG;
+  const int64_t total = sdl_mask_budget_scoped(shape, sparsity, scope);
+  if (total < 0) return SDL_ERR_INVALID_ARG;
+  if (col_capacity < total) return SDL_ERR_CAPACITY;
+  const size_t need = sdl_select_workspace_bytes_scoped(shape, scope);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SDL_ERR_WORKSPACE;
+  const int nb = shape->L / shape->block;
+  // every head is its own single-head sequence: same layouts, B*H sequences of H = 1
+  const int seqs = shape->B * shape->H;
+  cudaError_t ce = launch_select(scores, seqs, 1, nb, total / seqs, row_ptr, col_idx, mask_u8,
+                                 workspace, static_cast<cudaStream_t>(stream));
   if (ce != cudaSuccess) return cuda_fail(ce);
   return SDL_OK;
 }

@@ -1,4 +1,4 @@
-"""Anchor-step schedule around the four library calls (host logic only).
+"""Step schedules around the library calls (host logic only).
 
 Step-dLLM (abstract) refreshes the block-sparse mask at anchor steps of the
 denoising trajectory and reuses it within each interval.  Here step ``s`` is an
@@ -6,47 +6,70 @@ anchor when ``s % anchor_every == 0`` (step 0 always is); at an anchor the mask
 is rebuilt from that step's Q and K before the step's own sparse attention
 runs, so every step, anchors included, attends with the mask of its anchor
 ``(s // anchor_every) * anchor_every``.
+
+Two variants of the prior methods the abstract compares against (SparseD
+abstract) are selectable: a uniform budget per head instead of the
+head-adaptive global one (``budget="head"``), and dense attention for the first
+``dense_steps`` steps followed by a single mask, built at step
+``dense_steps`` and reused for every later step (``anchor_every=None``).
 """
 from __future__ import annotations
 
 import torch
 
-from . import (block_scores, make_shape, mask_budget, scores_workspace_bytes, select_mask,
-               select_workspace_bytes, sparse_attn, tile_plan)
+from . import (block_scores, dense_attn, make_shape, mask_budget, scores_workspace_bytes,
+               select_mask, select_workspace_bytes, sparse_attn, tile_plan)
 
 
-def is_anchor(step: int, anchor_every: int) -> bool:
-    return step % anchor_every == 0
+def is_dense(step: int, dense_steps: int = 0) -> bool:
+    return step < dense_steps
 
 
-def anchor_of(step: int, anchor_every: int) -> int:
-    return (step // anchor_every) * anchor_every
+def is_anchor(step: int, anchor_every, dense_steps: int = 0) -> bool:
+    """Whether the mask is rebuilt at `step` (anchor_every None: only at dense_steps)."""
+    if step < dense_steps:
+        return False
+    if anchor_every is None:
+        return step == dense_steps
+    return (step - dense_steps) % anchor_every == 0
+
+
+def anchor_of(step: int, anchor_every, dense_steps: int = 0):
+    """The step whose mask `step` attends with, or None for a dense step."""
+    if step < dense_steps:
+        return None
+    if anchor_every is None:
+        return dense_steps
+    return dense_steps + ((step - dense_steps) // anchor_every) * anchor_every
 
 
 class StepSparseAttention:
     """One attention layer's block-sparse state across denoising steps.
 
-    All device buffers (scores, workspaces, CSR lists) are allocated once here,
-    so the per-step calls allocate nothing.
+    All device buffers (scores, workspaces, CSR lists, tile plan) are allocated
+    once here, so the per-step calls allocate nothing.
     """
 
     def __init__(self, B, H, H_kv, L, d, block, sparsity, anchor_every, dtype=torch.bfloat16,
-                 device="cuda"):
+                 device="cuda", budget: str = "sequence", dense_steps: int = 0):
+        if budget not in ("sequence", "head"):
+            raise ValueError("budget must be 'sequence' or 'head'")
         self.B, self.H, self.H_kv, self.L, self.d, self.block = B, H, H_kv, L, d, block
         self.sparsity, self.anchor_every = sparsity, anchor_every
+        self.per_head, self.dense_steps = budget == "head", dense_steps
         self.nb = L // block
         probe_q = torch.empty((B, L, H, d), dtype=dtype, device="meta")
         probe_k = torch.empty((B, L, H_kv, d), dtype=dtype, device="meta")
         shape = make_shape(probe_q, probe_k, block)
-        self.budget = mask_budget(shape, sparsity)
+        self.budget = mask_budget(shape, sparsity, self.per_head)
         if self.budget < 0:
             raise ValueError("sparsity outside [0, 1) or budget below the diagonal blocks")
         dev = torch.device(device)
         self.scores = torch.empty((B, H, self.nb, self.nb), dtype=torch.float32, device=dev)
         self.ws_scores = torch.empty(max(scores_workspace_bytes(shape), 16), dtype=torch.uint8,
                                      device=dev)
-        self.ws_select = torch.empty(max(select_workspace_bytes(shape), 16), dtype=torch.uint8,
-                                     device=dev)
+        self.ws_select = torch.empty(max(select_workspace_bytes(shape, self.per_head), 16),
+                                     dtype=torch.uint8, device=dev)
         self.row_ptr = torch.empty(B * H * self.nb + 1, dtype=torch.int32, device=dev)
         self.col_idx = torch.empty(self.budget, dtype=torch.int32, device=dev)
         # 64-token blocks: which two query blocks share a 128-row tile (rebuilt with the mask)
@@ -58,14 +81,17 @@ class StepSparseAttention:
         block_scores(q, k, self.block, scores=self.scores, workspace=self.ws_scores,
                      stream=stream)
         select_mask(self.scores, self.sparsity, self.block, self.L, row_ptr=self.row_ptr,
-                    col_idx=self.col_idx, workspace=self.ws_select, stream=stream)
+                    col_idx=self.col_idx, workspace=self.ws_select, per_head=self.per_head,
+                    stream=stream)
         if self.plan is not None:
             tile_plan(self.row_ptr, self.col_idx, self.B, self.H, self.L, self.block,
                       plan=self.plan, stream=stream)
         self.mask_step = step
 
     def __call__(self, q, k, v, step: int, out=None, lse=None, stream=None):
-        if is_anchor(step, self.anchor_every) or self.mask_step is None:
-            self.refresh(q, k, anchor_of(step, self.anchor_every), stream)
+        if is_dense(step, self.dense_steps):
+            return dense_attn(q, k, v, self.block, out=out, lse=lse, stream=stream)
+        if is_anchor(step, self.anchor_every, self.dense_steps) or self.mask_step is None:
+            self.refresh(q, k, anchor_of(step, self.anchor_every, self.dense_steps), stream)
         return sparse_attn(q, k, v, self.row_ptr, self.col_idx, self.block, out=out, lse=lse,
                            plan=self.plan, stream=stream)

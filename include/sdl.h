@@ -106,6 +106,30 @@ sdl_status sdl_select_mask(const float* scores, const sdl_shape* shape, double s
                            uint8_t* mask_u8, void* workspace, size_t workspace_bytes,
                            void* stream);
 
+/* Scope of the mask budget.  SDL_BUDGET_SEQUENCE is the Step-dLLM abstract's
+ * head-adaptive global budget (sdl_select_mask).  SDL_BUDGET_HEAD is the uniform
+ * per-head budget of the prior methods the abstract compares against (SparseD
+ * abstract): every head keeps floor((1 - s) * nb^2 + 0.5) blocks of its own. */
+typedef enum { SDL_BUDGET_SEQUENCE = 0, SDL_BUDGET_HEAD = 1 } sdl_budget_scope;
+
+/* Total kept blocks of a call under `scope` (the sum over sequences or heads),
+ * or -1 when sparsity is outside [0, 1) or a budget is below its diagonal. */
+int64_t sdl_mask_budget_scoped(const sdl_shape* shape, double sparsity, int scope);
+
+/* Workspace bytes sdl_select_mask_scoped needs under `scope` (0 on a bad shape
+ * or scope); for SDL_BUDGET_SEQUENCE it equals sdl_select_workspace_bytes. */
+size_t sdl_select_workspace_bytes_scoped(const sdl_shape* shape, int scope);
+
+/* sdl_select_mask with the budget taken per `scope`: for SDL_BUDGET_HEAD each
+ * head's largest scores are taken among that head's own entries (the same rule
+ * as sdl_select_mask applied to every head alone); outputs as sdl_select_mask,
+ * with sdl_mask_budget_scoped entries, and a workspace of
+ * sdl_select_workspace_bytes_scoped bytes. */
+sdl_status sdl_select_mask_scoped(const float* scores, const sdl_shape* shape, double sparsity,
+                                  int scope, int32_t* row_ptr, int32_t* col_idx,
+                                  int64_t col_capacity, uint8_t* mask_u8, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 /* Allocation-free variant of sdl_select_mask (no counterpart in the paper; it
  * exists for callers that cannot allocate device memory, such as code running
  * inside a device-memory pool's own callbacks or a serving process that reserves

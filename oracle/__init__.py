@@ -107,9 +107,17 @@ def block_scores(q: np.ndarray, k: np.ndarray, bs: int, scale: float | None = No
     return out
 
 
-def select(P: np.ndarray, sparsity: float):
-    """(mask uint8 [B,H,nb,nb], tau float64 [B], kept blocks)."""
+def select(P: np.ndarray, sparsity: float, per_head: bool = False):
+    """(mask uint8 [B,H,nb,nb], tau float64 [B] (or [B*H] per head), kept blocks).
+
+    per_head: the uniform per-head budget of the prior methods the Step-dLLM abstract
+    compares against (SparseD abstract): the same selection rule applied to every head
+    as a sequence of its own."""
     P = np.ascontiguousarray(P, dtype=np.float64)
+    if per_head:
+        B0, H0, nb0, _ = P.shape
+        m, tau, kept = select(P.reshape(B0 * H0, 1, nb0, nb0), sparsity)
+        return m.reshape(B0, H0, nb0, nb0), tau, kept
     B, H, nb, _ = P.shape
     mask = np.empty(P.shape, dtype=np.uint8)
     tau = np.empty(B, dtype=np.float64)

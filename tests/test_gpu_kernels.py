@@ -93,6 +93,25 @@ def test_select_matches_oracle(B, H, nb, s):
     assert np.array_equal(got, want)  # identical fp32 inputs: no excuse needed
 
 
+@pytest.mark.parametrize("B,H,nb,s", [(1, 4, 16, 0.7), (2, 3, 32, 0.9), (1, 32, 128, 0.9)])
+def test_select_per_head_budget_matches_oracle(B, H, nb, s):
+    """Uniform per-head budget: the same rule applied to every head alone."""
+    rng = np.random.default_rng(nb * 5 + H)
+    logits = rng.standard_normal((B, H, nb, nb)) * rng.uniform(0.2, 3.0, (1, H, 1, 1))
+    P32 = (np.exp(logits) / np.exp(logits).sum(-1, keepdims=True)).astype(np.float32)
+    want, tau, kept = oracle.select(P32.astype(np.float64), s, per_head=True)
+    row_ptr, col_idx, mask = sdl.select_mask(torch.from_numpy(P32).cuda(), s, 64, nb * 64,
+                                             want_mask=True, per_head=True)
+    torch.cuda.synchronize()
+    rp, ci = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
+    check_csr(rp, ci, B, H, nb, kept)
+    got = csr_to_mask(rp, ci, B, H, nb)
+    assert np.array_equal(got, mask.cpu().numpy())
+    assert np.array_equal(got, want)
+    per = got.reshape(B * H, -1).sum(-1)
+    assert (per == per[0]).all() and per.sum() == kept
+
+
 def test_select_exact_ties_follow_flat_index():
     B, H, nb = 1, 3, 16
     P = np.full((B, H, nb, nb), 1.0 / nb, dtype=np.float32)

@@ -69,6 +69,41 @@ def test_schedule_full_parity(name, steps):
     assert sdl.last_device_status() == sdl.SDL_OK
 
 
+def test_prior_method_variants_schedule_and_parity():
+    """The comparison variants: SparseD's dense warm-up then one reused mask, with
+    the uniform per-head budget, on the 2K workload."""
+    w = synth.WORKLOADS["bf16-L2048-H32-s80"]
+    att = StepSparseAttention(w.B, w.H, w.H_kv, w.L, w.d, w.bs, w.sparsity, None,
+                              budget="head", dense_steps=2)
+    csr = None
+    for step in range(5):
+        dev = synth.device_inputs(w, step)
+        out = att(dev["q"], dev["k"], dev["v"], step)
+        host = synth.host_inputs(w, step)
+        if step < 2:
+            assert att.mask_step is None
+            ref = sdl.dense_attn(dev["q"], dev["k"], dev["v"])
+            assert torch.equal(out, ref)
+            continue
+        assert att.mask_step == 2
+        if step == 2:
+            P_or = oracle.block_scores(host["q"], host["k"], w.bs)
+            want, tau, kept = oracle.select(P_or, w.sparsity, per_head=True)
+            rp, ci = att.row_ptr.cpu().numpy(), att.col_idx.cpu().numpy()
+            check_csr(rp, ci, w.B, w.H, w.nb, kept)
+            got = csr_to_mask(rp, ci, w.B, w.H, w.nb)
+            shp = (w.B * w.H, 1, w.nb, w.nb)
+            compare_masks(got.reshape(shp), want.reshape(shp), P_or.reshape(shp), tau)
+            csr = (att.row_ptr.clone(), att.col_idx.clone())
+        else:  # the one mask is reused for every later step
+            assert torch.equal(att.row_ptr, csr[0]) and torch.equal(att.col_idx, csr[1])
+        mask = csr_to_mask(att.row_ptr.cpu().numpy(), att.col_idx.cpu().numpy(), w.B, w.H, w.nb)
+        rows = sample_rows(w.B, w.H, w.L, w.bs, mask.sum(-1), n_blocks=4, rows_per_block=8)
+        Ow, _ = oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=mask, rows=rows)
+        check_close(bf16_to_f64(out)[rows[:, 0], rows[:, 2], rows[:, 1]], Ow, "bf16")
+    assert sdl.last_device_status() == sdl.SDL_OK
+
+
 @pytest.mark.parametrize("name,step", [("bf16-L8192-H32-s90", 0), ("bf16-L8192-H32-s90", 64),
                                        ("bf16-L16384-H28kv4-s90", 16),
                                        ("bf16-L65536-H32-bs128-s95", 0)])

@@ -222,6 +222,43 @@ def test_select_single_head_is_per_head_topk():
     assert np.array_equal(mask[0, 0][off], want)
 
 
+def test_select_per_head_brute_force_and_counts():
+    """Uniform per-head budget (the prior methods' rule): in every head, the kept
+    off-diagonal set is the one of largest total score among all subsets of that
+    head's per-head size, the diagonal is kept, and each head keeps the same count."""
+    rng = np.random.default_rng(11)
+    H, nb = 3, 3
+    P = rng.random((1, H, nb, nb))
+    free_h = [(i, j) for i in range(nb) for j in range(nb) if i != j]
+    for k in range(0, len(free_h) + 1):
+        s = 1.0 - (nb + k) / (nb * nb)
+        mask, tau, kept = oracle.select(P, s, per_head=True)
+        assert kept == H * (nb + k)
+        for h in range(H):
+            assert mask[0, h].sum() == nb + k
+            assert all(mask[0, h, i, i] == 1 for i in range(nb))
+            best, best_set = -1.0, None
+            for sub in itertools.combinations(range(len(free_h)), k):
+                tot = sum(P[0, h, free_h[x][0], free_h[x][1]] for x in sub)
+                if tot > best:
+                    best, best_set = tot, set(sub)
+            got = {x for x, (i, j) in enumerate(free_h) if mask[0, h, i, j]}
+            assert got == best_set
+
+
+def test_select_per_head_differs_from_global_on_skewed_heads():
+    """A head with a concentrated row distribution gets fewer blocks under the global
+    budget than under the per-head one; per head, every head gets the same count."""
+    nb = 8
+    P = np.full((1, 2, nb, nb), 1.0 / nb)
+    P[0, 0] = 1e-3
+    np.fill_diagonal(P[0, 0], 1.0)
+    mask_g, _, _ = oracle.select(P, 0.5)
+    mask_h, _, _ = oracle.select(P, 0.5, per_head=True)
+    assert mask_h[0, 0].sum() == mask_h[0, 1].sum()
+    assert mask_g[0, 0].sum() < mask_g[0, 1].sum()
+
+
 def test_select_is_head_adaptive():
     """A concentrated head keeps few blocks; a flat head with larger entries keeps many."""
     nb = 16
