@@ -75,9 +75,12 @@ EncodeTiledFn encode_fn() {
 }
 
 // 4-D map over a [B, L, heads, d] bf16 tensor: dims (d, t, h, b), box of
-// 64 d-columns x 64 tokens, 128-byte swizzle, zero fill out of range.
+// `box_d` d-columns x `box_t` tokens, zero fill out of range.  Loads use
+// 64 x 64 boxes with 128-byte swizzle, the output stores 32 x 32 with 64-byte
+// swizzle.
 bool encode_bf16_map(CUtensorMap* map, const void* base, const sdl_shape& s, int heads,
-                     const int64_t* st) {
+                     const int64_t* st, cuuint32_t box_d = 64, cuuint32_t box_t = 64,
+                     CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)s.L, (cuuint64_t)heads, (cuuint64_t)s.B};
@@ -85,10 +88,10 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, const sdl_shape& s, int
   // a zero stride (broadcast) is not expressible: use the dimension's natural size
   for (int i = 0; i < 3; ++i)
     if (strides[i] == 0) strides[i] = 16;
-  cuuint32_t box[4] = {64, 64, 1, 1};
+  cuuint32_t box[4] = {box_d, box_t, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -135,12 +138,13 @@ sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_sh
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t ce;
   if (s.dtype == SDL_BF16) {
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!encode_bf16_map(&tq, q, s, s.H, s.q_strides) ||
         !encode_bf16_map(&tk, k, s, s.H_kv, s.k_strides) ||
-        !encode_bf16_map(&tv, v, s, s.H_kv, s.v_strides))
+        !encode_bf16_map(&tv, v, s, s.H_kv, s.v_strides) ||
+        !encode_bf16_map(&to, o, s, s.H, s.o_strides, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
       return cuda_fail(cudaErrorInvalidValue);
-    ce = launch_attn_tc(a, &tq, &tk, &tv, st);
+    ce = launch_attn_tc(a, &tq, &tk, &tv, &to, st);
   } else {
     ce = launch_attn_simt(a, st);
   }

@@ -34,9 +34,10 @@
 //                 Online softmax in the log2 domain; the running max is raised
 //                 only when it grows by more than 8 (a factor 256), and O_t is
 //                 rescaled in TMEM only then; P written back as bf16, the row
-//                 sum taken over those rounded weights; 2 of every 8
-//                 exponentials on the FMA pipe.  Epilogue per item: O / l
-//                 rounded to bf16, LSE.
+//                 sum taken over those rounded weights (the LSE's over the
+//                 fp32 weights).  Epilogue per item: O / l rounded to bf16
+//                 and written by TMA tensor stores from a per-warp
+//                 shared-memory box, LSE.
 //
 // Merged step order: the producers and the MMA issuer take the steps of the
 // two streams alternately (0, 1, 0, 1, ...); once a stream has no more items
@@ -66,13 +67,17 @@ constexpr int kBM = 128;         // query rows per item
 constexpr int kBN = 128;         // key rows per step
 constexpr int kStages = 2;       // K and V ring depth
 constexpr int kStreams = 2;
-constexpr int kSlots = 2;        // list slots per stream
+constexpr int kSlots = 2;        // list slots per stream (at most 4)
 constexpr int kMaxSub = 1024;    // 64-token sub-blocks per sequence (L <= 65536)
 constexpr int kThreads = 384;    // 12 warps
 constexpr int kKWarp = 0, kMmaWarp = 1, kVWarp = 2, kItemWarp = 3, kSoftWarp0 = 4;
 constexpr int kBox = 64 * 128;   // bytes of one 64-row x 64-column bf16 box
+constexpr int kOBoxBytes = 32 * 64;  // one 32-row x 32-column bf16 output box
 constexpr uint32_t kTmemCols = 512;
-constexpr int kPolyPer8 = 2;     // of every 8 weights, how many take exp2_poly (FMA pipe)
+// Of every 8 weights, how many take exp2_poly on the FMA pipe instead of
+// MUFU.EX2 (even values; the step is issue-bound more than MUFU-bound here,
+// and 0 measured fastest).
+constexpr int kPolyPer8 = 0;
 
 __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * (uint32_t)t; }
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * (uint32_t)t; }
@@ -87,7 +92,10 @@ struct Layout {
   static constexpr int kOffQ = 0;                  // one Q tile per stream
   static constexpr int kOffK = kStreams * kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKVBytes;
-  static constexpr int kBytes = kOffV + kStages * kKVBytes;
+  // output staging: per softmax warp one 32-row x 32-column bf16 box
+  // (64-byte rows, 64-byte swizzle) for the tensor stores of O
+  static constexpr int kOffO = kOffV + kStages * kKVBytes;
+  static constexpr int kBytes = kOffO + 8 * kOBoxBytes;
   static constexpr int kSmem = kBytes + 1024;      // + alignment slack
 };
 
@@ -120,7 +128,7 @@ struct Slot {
 // Step records, written by the K producer for the MMA issuer, one per step
 // of the merged order (ring position g % kCmdRing):
 //   bit 0 stream, bit 1 first step of its item, bit 2 last step of its item,
-//   bit 3 the item's list slot, bits 4-5 distance back to the stream's
+//   bits 3-4 the item's list slot, bits 5-6 distance back to the stream's
 //   previous step in the merged order (0: none), bit 7 end of the order.
 constexpr int kCmdRing = 8;
 constexpr uint32_t kCmdEnd = 0x80u;
@@ -198,7 +206,8 @@ __device__ __forceinline__ void write_empty_tile(const AttnArgs& a, int b, int h
 template <int D, bool kLse>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                   const __grid_constant__ CUtensorMap tmv, AttnArgs a, int sched_slot) {
+                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                   AttnArgs a, int sched_slot) {
   using Lay = Layout<D>;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
@@ -485,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (isk) {
           const int prev = t ? last_g1 : last_g0;
           const uint32_t rec = (uint32_t)t | (jj == 0 ? 2u : 0u) | (C.at_end(t) ? 4u : 0u) |
-                               ((uint32_t)slot << 3) | ((uint32_t)(prev < 0 ? 0 : g - prev) << 4);
+                               ((uint32_t)slot << 3) | ((uint32_t)(prev < 0 ? 0 : g - prev) << 5);
           if (t)
             last_g1 = g;
           else
@@ -572,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             return 0;
           }
         }
-        const int gap = (int)((s_rec >> 4) & 3u);
+        const int gap = (int)((s_rec >> 5) & 3u);
         if (gap > 0 && s - gap >= p) return 0;  // that stream's PV is not issued yet
         const int t = (int)(s_rec & 1u);
         if (s_rec & 2u) {  // first step of an item: its Q tile
@@ -636,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(&bars.vempty[st]);
           if (rec & 4u) {
             tc_commit(&bars.o_full[t]);
-            mbar_arrive(&bars.list_empty[t][(rec >> 3) & 1u]);
+            mbar_arrive(&bars.list_empty[t][(rec >> 3) & 3u]);
           }
         }
         ++p;
@@ -666,6 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t scol = trow + col_s(t);
     const uint32_t ocol = trow + col_o(t);
+    uint8_t* ostage = dsm + Lay::kOffO + (warp - kSoftWarp0) * kOBoxBytes;
     const float sl2 = a.scale_log2;
     int n = 0;  // steps of this stream so far
     bool ok = true;
@@ -786,25 +796,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
-      __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(a.o) + b * a.os[0] +
-                          (int64_t)tok * a.os[1] + h * a.os[2];
+      // O / l as bf16, 32 columns at a time through this warp's staging box
+      // (row `lane` holds its 64 bytes as four 16-byte chunks, chunk x at
+      // x ^ ((lane / 2) % 4): the 64-byte swizzle), then one tensor store per
+      // box; rows past L are clipped by the store
+      const int tok0 = tok - lane;  // first token of this warp's 32 rows
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
         tmem_ld32(ocol + c * 32, ov);
         tmem_wait_ld();
-        if (tok < a.L) {
-          uint32_t pk[16];
+        uint32_t pk[16];
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(ov[2 * x]) * inv,
-                                                     __uint_as_float(ov[2 * x + 1]) * inv);
-            pk[x] = *reinterpret_cast<uint32_t*>(&v);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(op + c * 32);
+        for (int x = 0; x < 16; ++x) {
+          __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(ov[2 * x]) * inv,
+                                                   __uint_as_float(ov[2 * x + 1]) * inv);
+          pk[x] = *reinterpret_cast<uint32_t*>(&v);
+        }
+        if (lane == 0) bulk_wait_read_all();  // the previous box has been read out
+        __syncwarp();
+        uint4* row_sm = reinterpret_cast<uint4*>(ostage + lane * 64);
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        for (int x = 0; x < 4; ++x)
+          row_sm[x ^ ((lane >> 1) & 3)] =
+              make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && tok0 < a.L) {
+          tma_store_4d(&tmo, ostage, c * 32, tok0, h, b);
+          bulk_commit_group();
         }
       }
       tc_fence_before();
@@ -814,6 +834,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         a.lse[((int64_t)b * a.H + h) * a.L + tok] =
             lx > 0.f ? (m + log2f(lx)) * 0.69314718055994531f : -INFINITY;
     }
+    if (lane == 0) bulk_wait_all();  // this warp's output stores have completed
+    __syncwarp();
     if (!ok) raise_timeout(&abort_sh, a.status);
   }
 
@@ -839,20 +861,20 @@ std::atomic<unsigned> g_launches{0};
 
 template <int D, bool kLse>
 cudaError_t launch_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
-                      const CUtensorMap* tv, cudaStream_t st, int grid) {
+                      const CUtensorMap* tv, const CUtensorMap* to, cudaStream_t st, int grid) {
   using Lay = Layout<D>;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, kLse>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmem);
   if (e != cudaSuccess) return e;
   const int slot = (int)(g_launches.fetch_add(1u) % kSchedRing);
-  attn_tc_kernel<D, kLse><<<grid, kThreads, Lay::kSmem, st>>>(*tq, *tk, *tv, a, slot);
+  attn_tc_kernel<D, kLse><<<grid, kThreads, Lay::kSmem, st>>>(*tq, *tk, *tv, *to, a, slot);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
-                           const CUtensorMap* tv, cudaStream_t st) {
+                           const CUtensorMap* tv, const CUtensorMap* to, cudaStream_t st) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -867,10 +889,10 @@ cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUten
   const int64_t want = (n_items + kStreams - 1) / kStreams;
   const int grid = (int)(want < g_num_sms[dev] ? want : g_num_sms[dev]);
   if (a.d == 128)
-    return a.lse ? launch_tc<128, true>(a, tq, tk, tv, st, grid)
-                 : launch_tc<128, false>(a, tq, tk, tv, st, grid);
-  return a.lse ? launch_tc<64, true>(a, tq, tk, tv, st, grid)
-               : launch_tc<64, false>(a, tq, tk, tv, st, grid);
+    return a.lse ? launch_tc<128, true>(a, tq, tk, tv, to, st, grid)
+                 : launch_tc<128, false>(a, tq, tk, tv, to, st, grid);
+  return a.lse ? launch_tc<64, true>(a, tq, tk, tv, to, st, grid)
+               : launch_tc<64, false>(a, tq, tk, tv, to, st, grid);
 }
 
 }  // namespace sdl

@@ -46,7 +46,7 @@ cudaError_t launch_select(const float* scores, int B, int H, int nb, int64_t kb,
                           int32_t* col_idx, uint8_t* mask, void* ws, cudaStream_t st);
 size_t select_workspace_bytes(int B, int H, int nb);
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
-                           const CUtensorMap* tv, cudaStream_t st);
+                           const CUtensorMap* tv, const CUtensorMap* to, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_plan(const int32_t* row_ptr, const int32_t* col_idx, int B, int H, int nb,
                         int32_t* plan, cudaStream_t st);
