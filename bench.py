@@ -408,6 +408,14 @@ def main():
     warm = [inputs[i % len(inputs)] for i in range(args.warmup)]
     for x, s in zip(warm, range(args.warmup)):
         runner.step(x, s)
+    # A schedule that starts with dense steps launches no anchor or sparse kernel
+    # while warming up: run each once, untimed, so that none is loaded inside the
+    # timed region.  The timed schedule then builds its own masks.
+    x0 = inputs[0]
+    runner.att.refresh(x0["q"], x0["k"], 0)
+    runner.sdl.sparse_attn(x0["q"], x0["k"], x0["v"], runner.att.row_ptr, runner.att.col_idx,
+                           w.bs, out=runner.out, plan=runner.att.plan)
+    runner.att.mask_step = None
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
