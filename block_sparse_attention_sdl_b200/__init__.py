@@ -29,7 +29,11 @@ EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspac
            "sdl_mask_budget_scoped", "sdl_select_workspace_bytes_scoped", "sdl_select_mask_scoped",
            "sdl_block_scores", "sdl_select_mask", "sdl_select_mask_noalloc", "sdl_sparse_attn",
            "sdl_tile_plan", "sdl_sparse_attn_planned", "sdl_dense_attn",
+           "sdl_select_shard_workspace_bytes", "sdl_select_shard_hist",
+           "sdl_select_shard_capacity", "sdl_select_shard_pass", "sdl_select_shard_count",
+           "sdl_select_shard_finish",
            "sdl_last_device_status", "sdl_last_cuda_error", "sdl_status_string")
+SDL_SELECT_PASSES = 3
 
 
 class Shape(ctypes.Structure):
@@ -79,11 +83,23 @@ def _lib():
         L.sdl_tile_plan.argtypes = [P, P, SP, P, P]
         L.sdl_sparse_attn_planned.argtypes = [P, P, P, SP, P, P, P, F, P, P, P]
         L.sdl_dense_attn.argtypes = [P, P, P, SP, F, P, P, P]
+        L.sdl_select_shard_workspace_bytes.argtypes = [SP]
+        L.sdl_select_shard_workspace_bytes.restype = SZ
+        L.sdl_select_shard_hist.argtypes = [SP, ctypes.c_int, ctypes.POINTER(SZ),
+                                            ctypes.POINTER(SZ)]
+        L.sdl_select_shard_capacity.argtypes = [SP, ctypes.c_int32, D]
+        L.sdl_select_shard_capacity.restype = I64
+        L.sdl_select_shard_pass.argtypes = [P, SP, ctypes.c_int32, D, ctypes.c_int, P, SZ, P]
+        L.sdl_select_shard_count.argtypes = [P, SP, ctypes.c_int32, D, P, SZ, P, P]
+        L.sdl_select_shard_finish.argtypes = [P, SP, ctypes.c_int32, D, P, P, P, I64, P, P, SZ,
+                                              P]
         L.sdl_last_device_status.argtypes = [P]
         L.sdl_last_cuda_error.argtypes = []
         L.sdl_status_string.argtypes = [ctypes.c_int]
         L.sdl_status_string.restype = ctypes.c_char_p
         for f in ("sdl_block_scores", "sdl_select_mask", "sdl_select_mask_scoped",
+                  "sdl_select_shard_hist", "sdl_select_shard_pass", "sdl_select_shard_count",
+                  "sdl_select_shard_finish",
                   "sdl_sparse_attn", "sdl_tile_plan",
                   "sdl_sparse_attn_planned", "sdl_dense_attn",
                   "sdl_last_device_status", "sdl_last_cuda_error"):
@@ -216,6 +232,89 @@ def select_mask(scores, sparsity: float, block: int, L: int, row_ptr=None, col_i
                                       row_ptr.data_ptr(), col_idx.data_ptr(), col_idx.numel(),
                                       mask_ptr, workspace.data_ptr(), workspace.numel(),
                                       _stream(stream)), "sdl_select_mask")
+    return row_ptr, col_idx, mask
+
+
+def _score_shape(scores, block: int, L: int) -> Shape:
+    B, H, nb, _ = scores.shape
+    if nb != L // block:
+        raise ValueError("scores shape does not match L / block")
+    s = Shape()
+    s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, H, L, 64, block, SDL_FP32
+    return s
+
+
+def select_shard_workspace_bytes(scores, block: int, L: int) -> int:
+    """Workspace bytes of the staged selection for this rank's part of the heads."""
+    return int(_lib().sdl_select_shard_workspace_bytes(ctypes.byref(_score_shape(scores, block, L))))
+
+
+def select_shard_hist(workspace, scores, block: int, L: int, p: int):
+    """int32 view of the pass-``p`` histogram inside the workspace (summed over ranks
+    in place between passes)."""
+    import torch
+    off, cnt = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib().sdl_select_shard_hist(ctypes.byref(_score_shape(scores, block, L)), int(p),
+                                        ctypes.byref(off), ctypes.byref(cnt)),
+           "sdl_select_shard_hist")
+    return workspace[off.value: off.value + 4 * cnt.value].view(torch.int32)
+
+
+def select_shard_capacity(scores, sparsity: float, block: int, L: int, heads_total: int) -> int:
+    n = int(_lib().sdl_select_shard_capacity(ctypes.byref(_score_shape(scores, block, L)),
+                                             int(heads_total), float(sparsity)))
+    if n < 0:
+        raise SdlError(SDL_ERR_INVALID_ARG, "sdl_select_shard_capacity")
+    return n
+
+
+def select_shard_pass(scores, sparsity: float, block: int, L: int, heads_total: int, p: int,
+                      workspace, stream=None):
+    s = _score_shape(scores, block, L)
+    _check(_lib().sdl_select_shard_pass(scores.data_ptr(), ctypes.byref(s), int(heads_total),
+                                        float(sparsity), int(p), workspace.data_ptr(),
+                                        workspace.numel(), _stream(stream)),
+           "sdl_select_shard_pass")
+
+
+def select_shard_count(scores, sparsity: float, block: int, L: int, heads_total: int,
+                       workspace, totals=None, stream=None):
+    """int64 [B, 2]: this rank's keys above and equal to the threshold, per sequence."""
+    import torch
+    s = _score_shape(scores, block, L)
+    if totals is None:
+        totals = torch.empty((s.B, 2), dtype=torch.int64, device=scores.device)
+    _check(_lib().sdl_select_shard_count(scores.data_ptr(), ctypes.byref(s), int(heads_total),
+                                         float(sparsity), workspace.data_ptr(),
+                                         workspace.numel(), totals.data_ptr(), _stream(stream)),
+           "sdl_select_shard_count")
+    return totals
+
+
+def select_shard_finish(scores, sparsity: float, block: int, L: int, heads_total: int,
+                        offsets, workspace, row_ptr=None, col_idx=None, mask=None,
+                        want_mask: bool = False, stream=None):
+    """This rank's CSR (row_ptr, col_idx with ``select_shard_capacity`` room, mask)."""
+    import torch
+    s = _score_shape(scores, block, L)
+    nb = L // block
+    dev = scores.device
+    if row_ptr is None:
+        row_ptr = torch.empty(s.B * s.H * nb + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty(select_shard_capacity(scores, sparsity, block, L, heads_total),
+                              dtype=torch.int32, device=dev)
+    if mask is None and want_mask:
+        mask = torch.empty((s.B, s.H, nb, nb), dtype=torch.uint8, device=dev)
+    if offsets.dtype != torch.int64 or not offsets.is_contiguous():
+        raise ValueError("offsets must be a contiguous int64 [B, 2] tensor")
+    _check(_lib().sdl_select_shard_finish(scores.data_ptr(), ctypes.byref(s), int(heads_total),
+                                          float(sparsity), offsets.data_ptr(),
+                                          row_ptr.data_ptr(), col_idx.data_ptr(),
+                                          col_idx.numel(),
+                                          None if mask is None else mask.data_ptr(),
+                                          workspace.data_ptr(), workspace.numel(),
+                                          _stream(stream)), "sdl_select_shard_finish")
     return row_ptr, col_idx, mask
 
 

@@ -281,6 +281,106 @@ sdl_status sdl_select_mask_scoped(const float* scores, const sdl_shape* shape, d
   return SDL_OK;
 }
 
+// ------------------------------------------------- heads split over ranks
+
+namespace {
+// Free picks per sequence under the global budget of all `heads_total` heads
+// (-1 if the arguments are invalid).
+int64_t shard_kfree(const sdl_shape* local, int32_t heads_total, double sparsity) {
+  if (check_shape(local) != SDL_OK) return -1;
+  if (heads_total < local->H) return -1;
+  if (!(sparsity >= 0.0 && sparsity < 1.0)) return -1;
+  const int64_t nb = local->L / local->block;
+  const int64_t kb =
+      (int64_t)floor((1.0 - sparsity) * (double)heads_total * (double)nb * (double)nb + 0.5);
+  const int64_t forced = (int64_t)heads_total * nb;
+  if (kb < forced) return -1;
+  return kb - forced;
+}
+
+sdl_status shard_args(const float* scores, const sdl_shape* local, int32_t heads_total,
+                      double sparsity, void* workspace, size_t workspace_bytes, int64_t* kfree) {
+  sdl_status e = check_shape(local);
+  if (e) return e;
+  *kfree = shard_kfree(local, heads_total, sparsity);
+  if (*kfree < 0) return SDL_ERR_INVALID_ARG;
+  if (!scores || !aligned16(scores)) return SDL_ERR_INVALID_ARG;
+  const size_t need = sdl_select_shard_workspace_bytes(local);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SDL_ERR_WORKSPACE;
+  return SDL_OK;
+}
+}  // namespace
+
+size_t sdl_select_shard_workspace_bytes(const sdl_shape* local) {
+  return sdl_select_workspace_bytes(local);
+}
+
+sdl_status sdl_select_shard_hist(const sdl_shape* local, int pass, size_t* offset_bytes,
+                                 size_t* count) {
+  sdl_status e = check_shape(local);
+  if (e) return e;
+  if (pass < 0 || pass >= SDL_SELECT_PASSES || !offset_bytes || !count) return SDL_ERR_INVALID_ARG;
+  *offset_bytes = select_hist_offset(local->B, pass);
+  *count = select_hist_count(local->B);
+  return SDL_OK;
+}
+
+int64_t sdl_select_shard_capacity(const sdl_shape* local, int32_t heads_total, double sparsity) {
+  const int64_t kfree = shard_kfree(local, heads_total, sparsity);
+  if (kfree < 0) return -1;
+  const int64_t nb = local->L / local->block;
+  const int64_t rows = (int64_t)local->H * nb;
+  const int64_t free_here = rows * (nb - 1) < kfree ? rows * (nb - 1) : kfree;
+  return (rows + free_here) * local->B;
+}
+
+sdl_status sdl_select_shard_pass(const float* scores, const sdl_shape* local, int32_t heads_total,
+                                 double sparsity, int pass, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  int64_t kfree = 0;
+  sdl_status e = shard_args(scores, local, heads_total, sparsity, workspace, workspace_bytes, &kfree);
+  if (e) return e;
+  if (pass < 0 || pass >= SDL_SELECT_PASSES) return SDL_ERR_INVALID_ARG;
+  cudaError_t ce = launch_select_shard_pass(scores, local->B, local->H, local->L / local->block,
+                                            kfree, pass, workspace,
+                                            static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_select_shard_count(const float* scores, const sdl_shape* local, int32_t heads_total,
+                                  double sparsity, void* workspace, size_t workspace_bytes,
+                                  int64_t* totals, void* stream) {
+  int64_t kfree = 0;
+  sdl_status e = shard_args(scores, local, heads_total, sparsity, workspace, workspace_bytes, &kfree);
+  if (e) return e;
+  if (!totals) return SDL_ERR_INVALID_ARG;
+  cudaError_t ce = launch_select_shard_count(scores, local->B, local->H, local->L / local->block,
+                                             kfree, workspace, totals,
+                                             static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_select_shard_finish(const float* scores, const sdl_shape* local,
+                                   int32_t heads_total, double sparsity, const int64_t* offsets,
+                                   int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                   uint8_t* mask_u8, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  int64_t kfree = 0;
+  sdl_status e = shard_args(scores, local, heads_total, sparsity, workspace, workspace_bytes, &kfree);
+  if (e) return e;
+  if (!offsets || !row_ptr || !col_idx) return SDL_ERR_INVALID_ARG;
+  if (col_capacity < sdl_select_shard_capacity(local, heads_total, sparsity))
+    return SDL_ERR_CAPACITY;
+  cudaError_t ce = launch_select_shard_finish(scores, local->B, local->H,
+                                              local->L / local->block, kfree, offsets, workspace,
+                                              row_ptr, col_idx, mask_u8,
+                                              static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
 sdl_status sdl_sparse_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,
                            const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
                            float* lse, void* stream) {

@@ -45,6 +45,16 @@ cudaError_t launch_scores(const float* qbar, const float* kbar, const sdl_shape&
 cudaError_t launch_select(const float* scores, int B, int H, int nb, int64_t kb, int32_t* row_ptr,
                           int32_t* col_idx, uint8_t* mask, void* ws, cudaStream_t st);
 size_t select_workspace_bytes(int B, int H, int nb);
+// staged selection for heads split over ranks (select.cu)
+cudaError_t launch_select_shard_pass(const float* scores, int B, int H, int nb, int64_t kfree,
+                                     int pass, void* ws, cudaStream_t st);
+cudaError_t launch_select_shard_count(const float* scores, int B, int H, int nb, int64_t kfree,
+                                      void* ws, int64_t* totals, cudaStream_t st);
+cudaError_t launch_select_shard_finish(const float* scores, int B, int H, int nb, int64_t kfree,
+                                       const int64_t* offs, void* ws, int32_t* row_ptr,
+                                       int32_t* col_idx, uint8_t* mask, cudaStream_t st);
+size_t select_hist_offset(int B, int pass);
+size_t select_hist_count(int B);
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, const CUtensorMap* to, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t st);

@@ -218,8 +218,12 @@ __global__ void __launch_bounds__(kThreads) count_kernel(const float* __restrict
 
 // One CTA of 1024 threads: per batch element, the ties are handed out to rows
 // in flat order (the tie-break), then the kept counts are scanned into row_ptr.
+// With `offs` (heads split over ranks; [B][2]: keys above the threshold over
+// all ranks, threshold ties held by lower ranks) the tie quota and its start
+// come from there instead of from this call's rows alone.
 __global__ void __launch_bounds__(1024) scan_kernel(int B, int H, int nb, uint32_t kfree,
-                                                    SelWs ws, int32_t* __restrict__ row_ptr) {
+                                                    SelWs ws, int32_t* __restrict__ row_ptr,
+                                                    const int64_t* __restrict__ offs) {
   __shared__ int s_warp[32];
   __shared__ int s_carry;
   const int rows = H * nb;
@@ -238,10 +242,14 @@ __global__ void __launch_bounds__(1024) scan_kernel(int B, int H, int nb, uint32
       for (int r = threadIdx.x; r < rows; r += 1024) g += ws.gt[(int64_t)b * rows + r];
       atomicAdd(&s_gt, g);
       __syncthreads();
-      krem = kfree - (uint32_t)s_gt;
+      krem = kfree - (uint32_t)(offs ? offs[2 * b] : (int64_t)s_gt);
     }
     __shared__ int s_eqcarry;
-    if (threadIdx.x == 0) s_eqcarry = 0;
+    if (threadIdx.x == 0) {
+      // ties held by lower ranks come first; more than the quota means none here
+      const int64_t before = offs ? offs[2 * b + 1] : 0;
+      s_eqcarry = before > (int64_t)krem ? (int)krem : (int)before;
+    }
     __syncthreads();
     for (int r0 = 0; r0 < rows; r0 += 1024) {
       const int r = r0 + threadIdx.x;
@@ -348,6 +356,29 @@ __global__ void __launch_bounds__(kThreads) write_kernel(const float* __restrict
   }
 }
 
+// grid: B; per batch element this call's keys above the threshold and equal to
+// it (totals[2b], totals[2b+1]).
+__global__ void __launch_bounds__(kThreads) totals_kernel(int B, int H, int nb, SelWs ws,
+                                                          int64_t* __restrict__ totals) {
+  __shared__ unsigned long long s[2];
+  const int b = blockIdx.x;
+  if (threadIdx.x == 0) s[0] = s[1] = 0;
+  __syncthreads();
+  unsigned long long g = 0, e = 0;
+  const int rows = H * nb;
+  for (int r = threadIdx.x; r < rows; r += kThreads) {
+    g += ws.gt[(int64_t)b * rows + r];
+    e += ws.eq[(int64_t)b * rows + r];
+  }
+  atomicAdd(&s[0], g);
+  atomicAdd(&s[1], e);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    totals[2 * b] = (int64_t)s[0];
+    totals[2 * b + 1] = (int64_t)s[1];
+  }
+}
+
 }  // namespace
 
 size_t select_workspace_bytes(int B, int H, int nb) {
@@ -372,10 +403,60 @@ cudaError_t launch_select(const float* scores, int B, int H, int nb, int64_t kb,
   int rchunks = (H * nb + (kThreads / 32) - 1) / (kThreads / 32);
   if (rchunks > 148 * 8) rchunks = 148 * 8;
   count_kernel<<<dim3(rchunks, B), kThreads, 0, st>>>(scores, B, H, nb, kfree, ws);
-  scan_kernel<<<1, 1024, 0, st>>>(B, H, nb, kfree, ws, row_ptr);
+  scan_kernel<<<1, 1024, 0, st>>>(B, H, nb, kfree, ws, row_ptr, nullptr);
   write_kernel<<<dim3(rchunks, B), kThreads, 0, st>>>(scores, B, H, nb, ws, row_ptr, col_idx,
                                                       mask);
   return cudaGetLastError();
 }
+
+// ------------------------------------------------- heads split over ranks
+// The same selection in stages, for a sequence whose heads are split over
+// ranks (contiguous head ranges in rank order, so flat order is rank order).
+// Between the stages the caller sums the pass histograms over ranks and
+// exchanges the per-rank totals; every stage re-derives the threshold from the
+// summed histograms, so all ranks agree on it.
+
+cudaError_t launch_select_shard_pass(const float* scores, int B, int H, int nb, int64_t kfree,
+                                     int pass, void* ws_raw, cudaStream_t st) {
+  const int R = B * H * nb;
+  SelWs ws = carve(ws_raw, B, R);
+  if (pass == 0) {
+    const size_t nh = (size_t)kPasses * B * kBins;
+    zero_kernel<<<(unsigned)((nh + 255) / 256), 256, 0, st>>>(ws.hist, nh);
+  }
+  const int64_t per_b = (int64_t)H * nb * nb;
+  int chunks = (int)((per_b / 4 + kThreads - 1) / kThreads);
+  if (chunks < 1) chunks = 1;
+  if (chunks > 148 * 4) chunks = 148 * 4;
+  hist_kernel<<<dim3(chunks, B), kThreads, 0, st>>>(scores, B, H, nb, (uint32_t)kfree, pass, ws);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_shard_count(const float* scores, int B, int H, int nb, int64_t kfree,
+                                      void* ws_raw, int64_t* totals, cudaStream_t st) {
+  const int R = B * H * nb;
+  SelWs ws = carve(ws_raw, B, R);
+  int rchunks = (H * nb + (kThreads / 32) - 1) / (kThreads / 32);
+  if (rchunks > 148 * 8) rchunks = 148 * 8;
+  count_kernel<<<dim3(rchunks, B), kThreads, 0, st>>>(scores, B, H, nb, (uint32_t)kfree, ws);
+  totals_kernel<<<B, kThreads, 0, st>>>(B, H, nb, ws, totals);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_shard_finish(const float* scores, int B, int H, int nb, int64_t kfree,
+                                       const int64_t* offs, void* ws_raw, int32_t* row_ptr,
+                                       int32_t* col_idx, uint8_t* mask, cudaStream_t st) {
+  const int R = B * H * nb;
+  SelWs ws = carve(ws_raw, B, R);
+  scan_kernel<<<1, 1024, 0, st>>>(B, H, nb, (uint32_t)kfree, ws, row_ptr, offs);
+  int rchunks = (H * nb + (kThreads / 32) - 1) / (kThreads / 32);
+  if (rchunks > 148 * 8) rchunks = 148 * 8;
+  write_kernel<<<dim3(rchunks, B), kThreads, 0, st>>>(scores, B, H, nb, ws, row_ptr, col_idx,
+                                                      mask);
+  return cudaGetLastError();
+}
+
+size_t select_hist_offset(int B, int pass) { return sizeof(int) * (size_t)pass * B * kBins; }
+size_t select_hist_count(int B) { return (size_t)B * kBins; }
 
 }  // namespace sdl

@@ -130,6 +130,49 @@ sdl_status sdl_select_mask_scoped(const float* scores, const sdl_shape* shape, d
                                   int64_t col_capacity, uint8_t* mask_u8, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/* ---- Mask selection with the heads of a sequence split over ranks ----------
+ * The global budget of the Step-dLLM abstract (and the rule of sdl_select_mask)
+ * when rank r of W holds the contiguous head range [h_r, h_r + H_local) of
+ * every sequence (ranks in head order, so flat index order is rank order), as
+ * when attention is sharded over GPUs by heads.  `local` describes this
+ * rank's part (H = H_local heads; its scores are fp32 [B, H_local, nb, nb]);
+ * `heads_total` is the sequence's head count, the budget is
+ * floor((1 - sparsity) * heads_total * nb^2 + 0.5) per sequence.  Steps, every
+ * rank in the same order:
+ *   1. for pass p = 0, 1, ..., SDL_SELECT_PASSES - 1:
+ *        sdl_select_shard_pass(p); then sum the pass-p histogram over ranks in
+ *        place (int32, `count` elements at `offset_bytes` into the workspace,
+ *        from sdl_select_shard_hist), e.g. one all-reduce;
+ *   2. sdl_select_shard_count: writes int64 totals[2 b] (keys above the
+ *      threshold on this rank) and totals[2 b + 1] (keys equal to it);
+ *   3. gather the totals of all ranks and pass offsets[2 b] = the sum over all
+ *      ranks of totals[2 b], offsets[2 b + 1] = the sum of totals[2 b + 1] over
+ *      the ranks before this one;
+ *   4. sdl_select_shard_finish: this rank's CSR (row_ptr over its B * H_local * nb
+ *      rows, starting at 0; col_idx ascending per row; optional mask_u8), its
+ *      part of the global selection exactly.
+ * The workspace (caller-owned, sdl_select_shard_workspace_bytes) must persist
+ * across the steps; offsets must stay valid until finish has run on the stream.
+ * col_capacity must be at least sdl_select_shard_capacity (an upper bound on
+ * this rank's kept blocks).  Errors as sdl_select_mask; SDL_ERR_INVALID_ARG also
+ * when heads_total < H_local. */
+#define SDL_SELECT_PASSES 3
+size_t sdl_select_shard_workspace_bytes(const sdl_shape* local);
+sdl_status sdl_select_shard_hist(const sdl_shape* local, int pass, size_t* offset_bytes,
+                                 size_t* count);
+int64_t sdl_select_shard_capacity(const sdl_shape* local, int32_t heads_total, double sparsity);
+sdl_status sdl_select_shard_pass(const float* scores, const sdl_shape* local, int32_t heads_total,
+                                 double sparsity, int pass, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+sdl_status sdl_select_shard_count(const float* scores, const sdl_shape* local, int32_t heads_total,
+                                  double sparsity, void* workspace, size_t workspace_bytes,
+                                  int64_t* totals, void* stream);
+sdl_status sdl_select_shard_finish(const float* scores, const sdl_shape* local,
+                                   int32_t heads_total, double sparsity, const int64_t* offsets,
+                                   int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                   uint8_t* mask_u8, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
 /* Allocation-free variant of sdl_select_mask (no counterpart in the paper; it
  * exists for callers that cannot allocate device memory, such as code running
  * inside a device-memory pool's own callbacks or a serving process that reserves

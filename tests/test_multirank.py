@@ -81,3 +81,62 @@ def test_reference_arm_runs_on_rank_zero_only():
                        text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def _scores_np(B, H, nb, seed, ties):
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal((B, H, nb, nb)) * rng.uniform(0.3, 4.0, size=(1, H, 1, 1))
+    if ties:
+        z = np.round(z)  # many equal logits, hence equal scores, within a row
+    e = np.exp(z - z.max(-1, keepdims=True))
+    return (e / e.sum(-1, keepdims=True)).astype(np.float32)
+
+
+SHARD_CASES = [(2, 8, 16, 0.8, False, 11), (1, 8, 12, 0.6, True, 12),
+               (2, 4, 8, 1.0 - 1.0 / 8, False, 13)]  # the last: diagonal only
+
+
+def _shard_rank_main(rank, world, port, out_dir):
+    import datetime
+
+    from block_sparse_attention_sdl_b200.sharded import head_range, select_mask_sharded
+    from shard_stages_np import NumpyStages
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        for n, (B, H, nb, s, ties, seed) in enumerate(SHARD_CASES):
+            P = _scores_np(B, H, nb, seed, ties)
+            h0, h1 = head_range(H, H, rank, world)
+            st = NumpyStages(P[:, h0:h1], s, H)
+            rp, ci, mask = select_mask_sharded(None, s, 64, nb * 64, H, rank, stages=st)
+            parts = [torch.zeros_like(mask) for _ in range(world)]
+            dist.all_gather(parts, mask)
+            np.save(os.path.join(out_dir, f"shard{n}_rank{rank}.npy"),
+                    torch.cat(parts, dim=1).numpy())
+            np.save(os.path.join(out_dir, f"shard{n}_csr{rank}.npy"),
+                    np.concatenate([rp.numpy(), ci.numpy()]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_gloo_head_sharded_selection(tmp_path):
+    """Heads split over two ranks: the histogram sums and tie offsets exchanged with
+    gloo reproduce the oracle's global selection exactly, on every rank."""
+    import oracle
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_shard_rank_main, args=(r, 2, port, str(tmp_path)))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    for n, (B, H, nb, s, ties, seed) in enumerate(SHARD_CASES):
+        want, _, kept = oracle.select(_scores_np(B, H, nb, seed, ties).astype(np.float64), s)
+        for r in range(2):
+            got = np.load(tmp_path / f"shard{n}_rank{r}.npy")
+            assert np.array_equal(got, want), (n, r)
+        total = sum(int(np.load(tmp_path / f"shard{n}_csr{r}.npy")[B * (H // 2) * nb])
+                    for r in range(2))
+        assert total == kept
