@@ -61,6 +61,11 @@ def parse():
                         "interval (the headline); uniform-head: the same schedule with a "
                         "uniform per-head budget; sparsed: dense attention for the first "
                         "--dense-steps steps, then one mask reused for every later step")
+    p.add_argument("--shard", choices=["sequences", "heads"], default="sequences",
+                   help="sequences: every rank its own independent sequence (weak scaling, no "
+                        "collective); heads: the ranks split the heads of one sequence, the "
+                        "mask's global budget met by the staged selection with NCCL "
+                        "exchanges (strong scaling)")
     p.add_argument("--dense-steps", type=int, default=32,
                    help="dense warm-up steps of the sparsed variant")
     p.add_argument("--profile", choices=["sparse", "dense"], default=None,
@@ -144,24 +149,37 @@ class ClockSampler:
 class Runner:
     """The library's step loop over per-step device inputs, with per-launch events."""
 
-    def __init__(self, w, seed, device, variant="step-dllm", dense_steps=0):
+    def __init__(self, w, seed, device, variant="step-dllm", dense_steps=0, shard=None,
+                 rank=0):
+        """shard: None (every head here) or (h0, h1, kv0, kv1), this rank's query- and
+        KV-head ranges of a head-sharded sequence."""
         import block_sparse_attention_sdl_b200 as sdl
         from block_sparse_attention_sdl_b200 import runtime
         self.sdl, self.w, self.rt = sdl, w, runtime
         sparsed = variant == "sparsed"
         self.interval = None if sparsed else w.anchor_every
         self.dense_steps = dense_steps if sparsed else 0
+        self.shard = shard
+        self.H, self.H_kv = (w.H, w.H_kv) if shard is None else (shard[1] - shard[0],
+                                                                 shard[3] - shard[2])
         self.att = runtime.StepSparseAttention(
-            w.B, w.H, w.H_kv, w.L, w.d, w.bs, w.sparsity, self.interval, device=device,
+            w.B, self.H, self.H_kv, w.L, w.d, w.bs, w.sparsity, self.interval, device=device,
             budget="head" if variant == "uniform-head" else "sequence",
-            dense_steps=self.dense_steps)
-        self.out = torch.empty((w.B, w.L, w.H, w.d), dtype=torch.bfloat16, device=device)
+            dense_steps=self.dense_steps, heads_total=None if shard is None else w.H,
+            rank=rank)
+        self.out = torch.empty((w.B, w.L, self.H, w.d), dtype=torch.bfloat16, device=device)
         self.seed = seed
         self.kinds = []  # per attention launch: "sparse" or "dense"
 
     def make_inputs(self, steps):
         import synth
-        return [synth.device_inputs(self.w, s, self.seed) for s in steps]
+        xs = [synth.device_inputs(self.w, s, self.seed) for s in steps]
+        if self.shard is not None:
+            # this rank's heads only, as a head-sharded projection would hand them over
+            h0, h1, kv0, kv1 = self.shard
+            xs = [{"q": x["q"][:, :, h0:h1].contiguous(), "k": x["k"][:, :, kv0:kv1].contiguous(),
+                   "v": x["v"][:, :, kv0:kv1].contiguous()} for x in xs]
+        return xs
 
     def step(self, x, s, ev=None):
         att, w, rt = self.att, self.w, self.rt
@@ -230,9 +248,10 @@ def time_steps(runner, inputs, steps, dist_on, device, with_events=True):
     return ms, ev
 
 
-def launches_per_anchor(block: int):
-    # pool, score; select: zero, 3 histogram passes, count, scan, write; tile plan (64-token blocks)
-    return 2 + 7 + (1 if block == 64 else 0)
+def launches_per_anchor(block: int, sharded: bool = False):
+    # pool, score; select: zero, 3 histogram passes, count, scan, write (+ the per-rank
+    # totals when the heads are sharded); tile plan (64-token blocks)
+    return 2 + 7 + (1 if sharded else 0) + (1 if block == 64 else 0)
 
 
 def e2e_measure(runner, inputs, steps, device):
@@ -398,8 +417,16 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     w = synth.WORKLOADS[args.workload]
-    seed = rank_seed(args.seed, rank)  # each rank: its own independent sequence
-    runner = Runner(w, seed, device, args.variant, args.dense_steps)
+    heads = args.shard == "heads"
+    if heads:
+        # one sequence, its heads split over the ranks (whole KV-head groups)
+        from block_sparse_attention_sdl_b200.sharded import head_range
+        h0, h1 = head_range(w.H, w.H_kv, rank, world)
+        g = w.H // w.H_kv
+        shard, seed = (h0, h1, h0 // g, h1 // g), args.seed
+    else:
+        shard, seed = None, rank_seed(args.seed, rank)  # each rank: its own sequence
+    runner = Runner(w, seed, device, args.variant, args.dense_steps, shard, rank)
     if args.profile:
         profile_kernel(runner, args)
         return
@@ -428,20 +455,25 @@ def main():
     ms_max = max_over_ranks(ms, dist_on, device)
 
     pk, pk_kind = peaks()
-    budget = runner.att.budget
+    budget = runner.att.budget  # kept blocks of the whole sequence
     flop_step = 4.0 * w.bs * w.bs * w.d * budget
     dense_flop = 4.0 * w.B * w.H * w.L * w.L * w.d
     kinds = runner.kinds[-len(steps):]
     n_dense_steps = kinds.count("dense")
+    # sequences counted per rank (weak scaling) or once, split over the ranks (heads)
+    seqs = 1 if heads else world
     # algorithmic work of the timed steps: kept blocks on sparse steps, L^2 on dense ones
     value = job_rate((flop_step * (len(steps) - n_dense_steps) + dense_flop * n_dense_steps) /
-                     len(steps), len(steps), world, ms_max)
+                     len(steps), len(steps), seqs, ms_max)
+    # this rank's launches: its own kept blocks and heads
+    local_blocks = int(runner.att.row_ptr[-1].item()) if heads else budget
+    flop_local = 4.0 * w.bs * w.bs * w.d * local_blocks
     attn_ms = [a.elapsed_time(b) for a, b in zip(ev["s0"], ev["s1"])]
     sparse_ms = [t for t, k in zip(attn_ms, kinds) if k == "sparse"]
     anchor_ms = [a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])]
     sp_avg = statistics.mean(sparse_ms)
     sp_q = statistics.quantiles(sparse_ms, n=10) if len(sparse_ms) > 1 else [sp_avg] * 9
-    kernel_tflops = flop_step / (sp_avg * 1e-3) / 1e12
+    kernel_tflops = flop_local / (sp_avg * 1e-3) / 1e12
     peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
 
     # anchor-step kernels, timed apart: scoring bandwidth and selection latency
@@ -462,10 +494,9 @@ def main():
     att = runner.att
     sc_ms = ev_time(lambda: sdl.block_scores(x0["q"], x0["k"], w.bs, scores=att.scores,
                                              workspace=att.ws_scores))
-    se_ms = ev_time(lambda: sdl.select_mask(att.scores, w.sparsity, w.bs, w.L,
-                                            row_ptr=att.row_ptr, col_idx=att.col_idx,
-                                            workspace=att.ws_select, per_head=att.per_head))
-    score_bytes = 2 * w.B * w.L * (w.H + w.H_kv) * w.d + 4 * w.B * w.H * w.nb * w.nb
+    se_ms = ev_time(att.select)
+    score_bytes = (2 * w.B * w.L * (runner.H + runner.H_kv) * w.d +
+                   4 * w.B * runner.H * w.nb * w.nb)
     # dense baseline on distinct inputs per launch (larger than L2 in total)
     de = []
     for i in range(min(6, len(inputs))):
@@ -478,13 +509,13 @@ def main():
     torch.cuda.synchronize()
     dense_ms = statistics.median([a.elapsed_time(b) for a, b in de[1:]] or
                                  [de[0][0].elapsed_time(de[0][1])])
-    dense_flop = 4.0 * w.B * w.H * w.L * w.L * w.d
+    dense_flop = 4.0 * w.B * runner.H * w.L * w.L * w.d  # this rank's heads
 
     e2e = None
     if not args.no_e2e:
         e_ms, bi, bo = e2e_measure(runner, inputs, steps, device)
         e_ms = max_over_ranks(e_ms, dist_on, device)
-        e2e = {"value": job_rate(flop_step, len(steps), world, e_ms), "unit": "TFLOP/s",
+        e2e = {"value": job_rate(flop_step, len(steps), seqs, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e_ms / len(steps)}
 
     cpu = None
@@ -497,15 +528,17 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": len(steps), "warmup": args.warmup, "ms_per_step": ms_max / len(steps),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if heads else "weak", "vs_baseline": None,
+        "dtype": "bf16",
         "data": "synthetic (seeded Philox inputs shaped like the 8K/90% workload, regenerated "
                 "per step)",
-        "config": {"workload": args.workload, "global_batch": w.B * world, "seq_len": w.L,
+        "config": {"workload": args.workload, "global_batch": w.B * seqs, "seq_len": w.L,
                    "heads": w.H, "kv_heads": w.H_kv, "head_dim": w.d, "block": w.bs,
                    "sparsity": w.sparsity, "anchor_every": runner.interval,
                    "dense_steps": runner.dense_steps,
                    "budget": "per head" if runner.att.per_head else "per sequence, across heads",
-                   "parallelism": f"independent sequences x{world}",
+                   "parallelism": (f"heads split over {world} ranks" if heads else
+                                   f"independent sequences x{world}"),
                    "l2": "inputs larger than L2 (192 MiB per step, distinct per step)"},
         "variant": args.variant,
         "sparse_attn_ms": sp_avg, "sparse_attn_tflops": kernel_tflops,
@@ -525,7 +558,7 @@ def main():
                      "traffic": traffic},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": len(steps) + n_anchor * launches_per_anchor(w.bs),
+        "gpu_launches": len(steps) + n_anchor * launches_per_anchor(w.bs, runner.att.sharded),
         "clocks": sampler.summary(),
     }
     if rank == 0:

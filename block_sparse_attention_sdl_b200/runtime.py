@@ -12,13 +12,21 @@ abstract) are selectable: a uniform budget per head instead of the
 head-adaptive global one (``budget="head"``), and dense attention for the first
 ``dense_steps`` steps followed by a single mask, built at step
 ``dense_steps`` and reused for every later step (``anchor_every=None``).
+
+With ``heads_total`` the layer is one rank's part of a head-sharded attention
+layer: its tensors hold ``H`` of the sequence's ``heads_total`` query heads
+(whole KV-head groups, ranks in head order), and the global budget is met with
+the staged selection of ``sharded.py`` (histogram sums and totals exchanged
+over ``group``); scores, attention and the tile plan stay local.
 """
 from __future__ import annotations
 
 import torch
 
 from . import (block_scores, dense_attn, make_shape, mask_budget, scores_workspace_bytes,
-               select_mask, select_workspace_bytes, sparse_attn, tile_plan)
+               select_mask, select_shard_capacity, select_workspace_bytes, sparse_attn,
+               tile_plan)
+from .sharded import CudaStages, select_mask_sharded, torch_collectives
 
 
 def is_dense(step: int, dense_steps: int = 0) -> bool:
@@ -51,9 +59,15 @@ class StepSparseAttention:
     """
 
     def __init__(self, B, H, H_kv, L, d, block, sparsity, anchor_every, dtype=torch.bfloat16,
-                 device="cuda", budget: str = "sequence", dense_steps: int = 0):
+                 device="cuda", budget: str = "sequence", dense_steps: int = 0,
+                 heads_total=None, rank: int = 0, group=None, collectives=None):
         if budget not in ("sequence", "head"):
             raise ValueError("budget must be 'sequence' or 'head'")
+        # a head-sharded layer needs the exchange only for the budget across heads
+        self.sharded = heads_total is not None and budget == "sequence"
+        self.heads_total = H if heads_total is None else heads_total
+        self.rank, self.group = rank, group
+        self.collectives = collectives
         self.B, self.H, self.H_kv, self.L, self.d, self.block = B, H, H_kv, L, d, block
         self.sparsity, self.anchor_every = sparsity, anchor_every
         self.per_head, self.dense_steps = budget == "head", dense_steps
@@ -61,17 +75,25 @@ class StepSparseAttention:
         probe_q = torch.empty((B, L, H, d), dtype=dtype, device="meta")
         probe_k = torch.empty((B, L, H_kv, d), dtype=dtype, device="meta")
         shape = make_shape(probe_q, probe_k, block)
-        self.budget = mask_budget(shape, sparsity, self.per_head)
+        full = make_shape(torch.empty((B, L, self.heads_total, d), dtype=dtype, device="meta"),
+                          torch.empty((B, L, self.heads_total, d), dtype=dtype, device="meta"),
+                          block)
+        # kept blocks of the whole sequence (every rank's heads)
+        self.budget = mask_budget(full, sparsity, self.per_head)
         if self.budget < 0:
             raise ValueError("sparsity outside [0, 1) or budget below the diagonal blocks")
         dev = torch.device(device)
         self.scores = torch.empty((B, H, self.nb, self.nb), dtype=torch.float32, device=dev)
+        if self.sharded:
+            capacity = select_shard_capacity(self.scores, sparsity, block, L, self.heads_total)
+        else:
+            capacity = mask_budget(shape, sparsity, self.per_head)
         self.ws_scores = torch.empty(max(scores_workspace_bytes(shape), 16), dtype=torch.uint8,
                                      device=dev)
         self.ws_select = torch.empty(max(select_workspace_bytes(shape, self.per_head), 16),
                                      dtype=torch.uint8, device=dev)
         self.row_ptr = torch.empty(B * H * self.nb + 1, dtype=torch.int32, device=dev)
-        self.col_idx = torch.empty(self.budget, dtype=torch.int32, device=dev)
+        self.col_idx = torch.empty(capacity, dtype=torch.int32, device=dev)
         # 64-token blocks: which two query blocks share a 128-row tile (rebuilt with the mask)
         self.plan = (torch.empty((B, H, (self.nb + 1) // 2, 2), dtype=torch.int32, device=dev)
                      if block == 64 else None)
@@ -80,13 +102,31 @@ class StepSparseAttention:
     def refresh(self, q, k, step: int, stream=None):
         block_scores(q, k, self.block, scores=self.scores, workspace=self.ws_scores,
                      stream=stream)
-        select_mask(self.scores, self.sparsity, self.block, self.L, row_ptr=self.row_ptr,
-                    col_idx=self.col_idx, workspace=self.ws_select, per_head=self.per_head,
-                    stream=stream)
+        self.select(stream)
         if self.plan is not None:
             tile_plan(self.row_ptr, self.col_idx, self.B, self.H, self.L, self.block,
                       plan=self.plan, stream=stream)
         self.mask_step = step
+
+    def select(self, stream=None):
+        """The mask from the current scores (every rank of a sharded layer calls it)."""
+        if self.sharded:
+            if self.collectives is not None:
+                all_reduce, all_gather = self.collectives
+            elif torch.distributed.is_available() and torch.distributed.is_initialized():
+                all_reduce, all_gather = torch_collectives(self.group)
+            else:  # a single rank holds every head
+                all_reduce, all_gather = (lambda t: None), (lambda t: [t])
+            stages = CudaStages(self.scores, self.sparsity, self.block, self.L, self.heads_total,
+                                workspace=self.ws_select, stream=stream)
+            select_mask_sharded(self.scores, self.sparsity, self.block, self.L,
+                                self.heads_total, self.rank, all_reduce=all_reduce,
+                                all_gather=all_gather, stages=stages, row_ptr=self.row_ptr,
+                                col_idx=self.col_idx)
+        else:
+            select_mask(self.scores, self.sparsity, self.block, self.L, row_ptr=self.row_ptr,
+                        col_idx=self.col_idx, workspace=self.ws_select,
+                        per_head=self.per_head, stream=stream)
 
     def __call__(self, q, k, v, step: int, out=None, lse=None, stream=None):
         if is_dense(step, self.dense_steps):
