@@ -248,10 +248,14 @@ def time_steps(runner, inputs, steps, dist_on, device, with_events=True):
     return ms, ev
 
 
-def launches_per_anchor(block: int, sharded: bool = False):
-    # pool, score; select: zero, 3 histogram passes, count, scan, write (+ the per-rank
-    # totals when the heads are sharded); tile plan (64-token blocks)
-    return 2 + 7 + (1 if sharded else 0) + (1 if block == 64 else 0)
+def launches_per_anchor(block: int, sharded: bool = False, fused: bool = False):
+    # fused: scores and selection in one launch; else pool, score; select: zero, 3
+    # histogram passes, count, scan, write (+ the per-rank totals when the heads are
+    # sharded); tile plan (64-token blocks)
+    plan = 1 if block == 64 else 0
+    if fused:
+        return 1 + plan
+    return 2 + 7 + (1 if sharded else 0) + plan
 
 
 def e2e_measure(runner, inputs, steps, device):
@@ -558,7 +562,8 @@ def main():
                      "traffic": traffic},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": len(steps) + n_anchor * launches_per_anchor(w.bs, runner.att.sharded),
+        "gpu_launches": len(steps) + n_anchor * launches_per_anchor(w.bs, runner.att.sharded,
+                                                                    runner.att.fused),
         "clocks": sampler.summary(),
     }
     if rank == 0:

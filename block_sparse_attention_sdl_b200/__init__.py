@@ -29,6 +29,7 @@ EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspac
            "sdl_mask_budget_scoped", "sdl_select_workspace_bytes_scoped", "sdl_select_mask_scoped",
            "sdl_block_scores", "sdl_select_mask", "sdl_select_mask_noalloc", "sdl_sparse_attn",
            "sdl_tile_plan", "sdl_sparse_attn_planned", "sdl_dense_attn",
+           "sdl_anchor_workspace_bytes", "sdl_anchor_refresh",
            "sdl_select_shard_workspace_bytes", "sdl_select_shard_hist",
            "sdl_select_shard_capacity", "sdl_select_shard_pass", "sdl_select_shard_count",
            "sdl_select_shard_finish",
@@ -83,6 +84,9 @@ def _lib():
         L.sdl_tile_plan.argtypes = [P, P, SP, P, P]
         L.sdl_sparse_attn_planned.argtypes = [P, P, P, SP, P, P, P, F, P, P, P]
         L.sdl_dense_attn.argtypes = [P, P, P, SP, F, P, P, P]
+        L.sdl_anchor_workspace_bytes.argtypes = [SP]
+        L.sdl_anchor_workspace_bytes.restype = SZ
+        L.sdl_anchor_refresh.argtypes = [P, P, SP, F, D, P, P, P, I64, P, P, SZ, P]
         L.sdl_select_shard_workspace_bytes.argtypes = [SP]
         L.sdl_select_shard_workspace_bytes.restype = SZ
         L.sdl_select_shard_hist.argtypes = [SP, ctypes.c_int, ctypes.POINTER(SZ),
@@ -98,6 +102,7 @@ def _lib():
         L.sdl_status_string.argtypes = [ctypes.c_int]
         L.sdl_status_string.restype = ctypes.c_char_p
         for f in ("sdl_block_scores", "sdl_select_mask", "sdl_select_mask_scoped",
+                  "sdl_anchor_refresh",
                   "sdl_select_shard_hist", "sdl_select_shard_pass", "sdl_select_shard_count",
                   "sdl_select_shard_finish",
                   "sdl_sparse_attn", "sdl_tile_plan",
@@ -233,6 +238,40 @@ def select_mask(scores, sparsity: float, block: int, L: int, row_ptr=None, col_i
                                       mask_ptr, workspace.data_ptr(), workspace.numel(),
                                       _stream(stream)), "sdl_select_mask")
     return row_ptr, col_idx, mask
+
+
+def anchor_workspace_bytes(q, k, block: int) -> int:
+    return int(_lib().sdl_anchor_workspace_bytes(ctypes.byref(make_shape(q, k, block))))
+
+
+def anchor_refresh(q, k, block: int, sparsity: float, scores=None, row_ptr=None, col_idx=None,
+                   plan=None, want_plan: bool = True, workspace=None, scale: float = 0.0,
+                   stream=None):
+    """Block scores, mask selection and (64-token blocks) the tile plan in one launch
+    (see ``sdl_anchor_refresh``); returns (scores, row_ptr, col_idx, plan or None)."""
+    import torch
+    s = make_shape(q, k, block)
+    nb = s.L // block
+    dev = q.device
+    total = mask_budget(s, sparsity)
+    if total < 0:
+        raise SdlError(SDL_ERR_INVALID_ARG, "sdl_mask_budget")
+    if scores is None:
+        scores = torch.empty((s.B, s.H, nb, nb), dtype=torch.float32, device=dev)
+    if row_ptr is None:
+        row_ptr = torch.empty(s.B * s.H * nb + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty(total, dtype=torch.int32, device=dev)
+    if plan is None and want_plan and block == 64:
+        plan = torch.empty((s.B, s.H, (nb + 1) // 2, 2), dtype=torch.int32, device=dev)
+    workspace = _workspace(anchor_workspace_bytes(q, k, block), dev, workspace)
+    _check(_lib().sdl_anchor_refresh(q.data_ptr(), k.data_ptr(), ctypes.byref(s), float(scale),
+                                     float(sparsity), scores.data_ptr(), row_ptr.data_ptr(),
+                                     col_idx.data_ptr(), col_idx.numel(),
+                                     None if plan is None else plan.data_ptr(),
+                                     workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "sdl_anchor_refresh")
+    return scores, row_ptr, col_idx, plan
 
 
 def _score_shape(scores, block: int, L: int) -> Shape:

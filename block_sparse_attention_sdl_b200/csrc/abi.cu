@@ -281,6 +281,46 @@ sdl_status sdl_select_mask_scoped(const float* scores, const sdl_shape* shape, d
   return SDL_OK;
 }
 
+// ------------------------------------------------- fused anchor step
+
+size_t sdl_anchor_workspace_bytes(const sdl_shape* shape) {
+  if (check_shape(shape) != SDL_OK) return 0;
+  return align256(sdl_scores_workspace_bytes(shape)) +
+         align256(sdl_select_workspace_bytes(shape)) + anchor_barrier_bytes();
+}
+
+sdl_status sdl_anchor_refresh(const void* q, const void* k, const sdl_shape* shape, float scale,
+                              double sparsity, float* scores, int32_t* row_ptr,
+                              int32_t* col_idx, int64_t col_capacity, int32_t* plan,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  const sdl_shape& s = *shape;
+  if (!q || !k || !scores || !row_ptr || !col_idx) return SDL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(scores)) return SDL_ERR_INVALID_ARG;
+  if ((e = check_strides(s.q_strides, s.dtype)) || (e = check_strides(s.k_strides, s.dtype)))
+    return e;
+  if (plan && s.block != 64) return SDL_ERR_INVALID_ARG;
+  const int64_t total = sdl_mask_budget(shape, sparsity);
+  if (total < 0) return SDL_ERR_INVALID_ARG;
+  if (col_capacity < total) return SDL_ERR_CAPACITY;
+  const size_t need = sdl_anchor_workspace_bytes(shape);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SDL_ERR_WORKSPACE;
+  int* status = device_status_ptr();
+  if (!status) return SDL_ERR_CUDA;
+  const size_t nb = s.L / s.block;
+  char* w = static_cast<char*>(workspace);
+  float* qbar = reinterpret_cast<float*>(w);
+  float* kbar = reinterpret_cast<float*>(w + align256(sizeof(float) * s.B * s.H * nb * s.d));
+  char* sel = w + align256(sdl_scores_workspace_bytes(shape));
+  unsigned* bar = reinterpret_cast<unsigned*>(sel + align256(sdl_select_workspace_bytes(shape)));
+  cudaError_t ce = launch_anchor(q, k, s, resolve_scale(scale, s.d), total / s.B, qbar, kbar,
+                                 scores, sel, row_ptr, col_idx, plan, bar, status,
+                                 static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
 // ------------------------------------------------- heads split over ranks
 
 namespace {

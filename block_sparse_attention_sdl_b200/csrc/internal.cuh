@@ -53,6 +53,13 @@ cudaError_t launch_select_shard_count(const float* scores, int B, int H, int nb,
 cudaError_t launch_select_shard_finish(const float* scores, int B, int H, int nb, int64_t kfree,
                                        const int64_t* offs, void* ws, int32_t* row_ptr,
                                        int32_t* col_idx, uint8_t* mask, cudaStream_t st);
+// fused anchor step (anchor.cu): scores, selection and (plan != nullptr) the
+// tile plan in one cooperative launch; `bar` holds anchor_barrier_bytes()
+cudaError_t launch_anchor(const void* q, const void* k, const sdl_shape& s, float scale,
+                          int64_t kb, float* qbar, float* kbar, float* scores, void* sel_ws,
+                          int32_t* row_ptr, int32_t* col_idx, int32_t* plan, unsigned* bar,
+                          int* status, cudaStream_t st);
+size_t anchor_barrier_bytes();
 size_t select_hist_offset(int B, int pass);
 size_t select_hist_count(int B);
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,

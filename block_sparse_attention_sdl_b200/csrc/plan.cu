@@ -13,22 +13,12 @@
 // The plan is a schedule only: attention results do not depend on it beyond
 // fp32 summation order.
 #include "internal.cuh"
+#include "plan_impl.cuh"
 
 namespace sdl {
 namespace {
 
-constexpr int kPlanThreads = 256;
-constexpr int kPlanMaxNb = 256;
-
-struct PlanSmem {
-  static size_t bytes(int nb) {
-    const int nw = (nb + 31) / 32;
-    return sizeof(uint32_t) * (size_t)nb * nw      // kept-list bitmaps
-           + sizeof(uint16_t) * (size_t)nb * nb    // pairwise intersections
-           + sizeof(int) * 2 * (size_t)nb          // list lengths, visiting order
-           + (size_t)nb + 16;                      // paired flags
-  }
-};
+using namespace planimpl;
 
 // grid (H, B); dynamic shared memory PlanSmem::bytes(nb)
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ row_ptr,
@@ -36,81 +26,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
                                                             int H, int nb, int n_qt,
                                                             int32_t* __restrict__ plan) {
   extern __shared__ __align__(16) uint8_t psm[];
-  const int nw = (nb + 31) / 32;
-  uint32_t* bits = reinterpret_cast<uint32_t*>(psm);
-  uint16_t* ov = reinterpret_cast<uint16_t*>(bits + (size_t)nb * nw);
-  int* len = reinterpret_cast<int*>(ov + (size_t)nb * nb + ((nb * nb) & 1));
-  int* order = len + nb;
-  volatile uint8_t* used = reinterpret_cast<uint8_t*>(order + nb);
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
-  const int64_t r0 = ((int64_t)b * H + h) * nb;
-  int32_t* out = plan + ((int64_t)b * H + h) * n_qt * 2;
-
-  for (int x = tid; x < nb * nw; x += kPlanThreads) bits[x] = 0u;
-  for (int x = tid; x < nb; x += kPlanThreads) used[x] = 0;
-  __syncthreads();
-  for (int i = warp; i < nb; i += kPlanThreads / 32) {
-    const int beg = row_ptr[r0 + i], end = row_ptr[r0 + i + 1];
-    for (int x = beg + lane; x < end; x += 32) {
-      const int j = col_idx[x];
-      if (j >= 0 && j < nb) atomicOr(&bits[i * nw + j / 32], 1u << (j % 32));
-    }
-  }
-  __syncthreads();
-  for (int i = tid; i < nb; i += kPlanThreads) {
-    int c = 0;
-    for (int w = 0; w < nw; ++w) c += __popc(bits[i * nw + w]);
-    len[i] = c;
-  }
-  for (int x = tid; x < nb * nb; x += kPlanThreads) {
-    const int i = x / nb, j = x % nb;
-    int c = 0;
-    for (int w = 0; w < nw; ++w) c += __popc(bits[i * nw + w] & bits[j * nw + w]);
-    ov[x] = (uint16_t)c;
-  }
-  __syncthreads();
-  for (int i = tid; i < nb; i += kPlanThreads) {
-    int rank = 0;
-    for (int j = 0; j < nb; ++j) rank += (len[j] > len[i]) || (len[j] == len[i] && j < i);
-    order[rank] = i;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    int p = 0;
-    for (int k = 0; k < nb; ++k) {
-      const int i = order[k];
-      if (used[i]) continue;
-      __syncwarp();
-      if (lane == 0) used[i] = 1;
-      __syncwarp();
-      // unpaired partner of largest intersection, lowest index on ties
-      int best = -1, bv = -1;
-      for (int j = lane; j < nb; j += 32) {
-        if (used[j]) continue;
-        const int v = ov[i * nb + j];
-        if (v > bv) {
-          bv = v;
-          best = j;
-        }
-      }
-      for (int o = 16; o > 0; o >>= 1) {
-        const int v2 = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int b2 = __shfl_xor_sync(0xffffffffu, best, o);
-        if (v2 > bv || (v2 == bv && b2 >= 0 && (best < 0 || b2 < best))) {
-          bv = v2;
-          best = b2;
-        }
-      }
-      if (lane == 0) {
-        if (best >= 0) used[best] = 1;
-        out[2 * p] = i;
-        out[2 * p + 1] = best;
-      }
-      __syncwarp();
-      ++p;
-    }
-  }
+  plan_body(row_ptr, col_idx, H, nb, n_qt, plan, blockIdx.x, blockIdx.y, psm);
 }
 
 // Adjacent pairs (2p, 2p+1), for heads too long for the greedy plan.

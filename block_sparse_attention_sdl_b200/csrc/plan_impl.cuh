@@ -1,0 +1,121 @@
+// Device code of the tile plan (pairing 64-token query blocks into 128-row
+// tiles by kept-list overlap), shared by plan.cu and the fused anchor kernel
+// of anchor.cu.  See plan.cu for the rule.
+#pragma once
+#include "internal.cuh"
+
+namespace sdl {
+namespace planimpl {
+namespace {  // internal linkage in every translation unit that includes this
+
+
+constexpr int kPlanThreads = 512;
+constexpr int kPlanMaxNb = 256;
+
+struct PlanSmem {
+  static size_t bytes(int nb) {
+    const int nw = (nb + 31) / 32;
+    return sizeof(uint32_t) * (size_t)nb * nw      // kept-list bitmaps, word-major
+           + sizeof(uint16_t) * (size_t)nb * nb    // pairwise intersections
+           + sizeof(int) * 2 * (size_t)nb          // list lengths, visiting order
+           + sizeof(int) * ((size_t)nb + 1)        // the head's row offsets
+           + 16;
+  }
+};
+
+// Block (head h, batch element b), any multiple of 32 threads; shared memory
+// `psm` of PlanSmem::bytes(nb), 16-byte aligned.
+__device__ __forceinline__ void plan_body(const int32_t* __restrict__ row_ptr,
+                                          const int32_t* __restrict__ col_idx, int H, int nb,
+                                          int n_qt, int32_t* __restrict__ plan, int h, int b,
+                                          uint8_t* psm) {
+  const int nthr = blockDim.x;
+  const int nw = (nb + 31) / 32;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(psm);
+  uint16_t* ov = reinterpret_cast<uint16_t*>(bits + (size_t)nb * nw);
+  int* len = reinterpret_cast<int*>(ov + (size_t)nb * nb + ((nb * nb) & 1));
+  int* order = len + nb;
+  int* rp = order + nb;
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  const int64_t r0 = ((int64_t)b * H + h) * nb;
+  int32_t* out = plan + ((int64_t)b * H + h) * n_qt * 2;
+
+  for (int x = tid; x < nb * nw; x += nthr) bits[x] = 0u;
+  for (int x = tid; x <= nb; x += nthr) rp[x] = row_ptr[r0 + x];
+  __syncthreads();
+  // the head's entries as one flat range; an entry's row by binary search in rp
+  {
+    const int base = rp[0], n = rp[nb] - rp[0];
+    for (int x = tid; x < n; x += nthr) {
+      int lo = 0, hi = nb - 1;  // last row whose start is <= base + x
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (rp[mid] <= base + x)
+          lo = mid;
+        else
+          hi = mid - 1;
+      }
+      const int j = col_idx[base + x];
+      if (j >= 0 && j < nb) atomicOr(&bits[(j / 32) * nb + lo], 1u << (j % 32));
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < nb; i += nthr) {
+    int c = 0;
+    for (int w = 0; w < nw; ++w) c += __popc(bits[w * nb + i]);
+    len[i] = c;
+  }
+  // intersections of every unordered pair once: (i, i + d mod nb), 1 <= d <= nb / 2
+  const int half = nb / 2;
+  for (int x = tid; x < nb * half; x += nthr) {
+    const int i = x / half, dd = x % half + 1, j = (i + dd) % nb;
+    if (2 * dd == nb && i > j) continue;  // that pair comes from its other end
+    int c = 0;
+    for (int w = 0; w < nw; ++w) c += __popc(bits[w * nb + i] & bits[w * nb + j]);
+    ov[i * nb + j] = ov[j * nb + i] = (uint16_t)c;
+  }
+  __syncthreads();
+  for (int i = tid; i < nb; i += nthr) {
+    int rank = 0;
+    for (int j = 0; j < nb; ++j) rank += (len[j] > len[i]) || (len[j] == len[i] && j < i);
+    order[rank] = i;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // lane owns the blocks j = lane + 32 c; bit c of `unpaired`: that block exists
+    // and is not paired yet
+    const int nc = (nb + 31) / 32;
+    uint32_t unpaired = 0;
+    for (int c = 0; c < nc; ++c)
+      if (lane + 32 * c < nb) unpaired |= 1u << c;
+    int p = 0;
+    for (int k = 0; k < nb; ++k) {
+      const int i = order[k];
+      if (!((__shfl_sync(0xffffffffu, unpaired, i & 31) >> (i >> 5)) & 1u)) continue;
+      if (lane == (i & 31)) unpaired &= ~(1u << (i >> 5));
+      // unpaired partner of largest intersection, lowest index on ties: the
+      // largest key (intersection + 1) << 16 | (0xFFFF - j); 0 when none is left
+      uint32_t key = 0;
+#pragma unroll
+      for (int c = 0; c < kPlanMaxNb / 32; ++c)
+        if (c < nc && ((unpaired >> c) & 1u)) {
+          const int j = lane + 32 * c;
+          const uint32_t kj = ((uint32_t)ov[i * nb + j] + 1u) << 16 | (0xFFFFu - (uint32_t)j);
+          key = kj > key ? kj : key;
+        }
+      key = __reduce_max_sync(0xffffffffu, key);
+      const int best = key ? (int)(0xFFFFu - (key & 0xFFFFu)) : -1;
+      if (best >= 0 && lane == (best & 31)) unpaired &= ~(1u << (best >> 5));
+      if (lane == 0) {
+        out[2 * p] = i;
+        out[2 * p + 1] = best;
+      }
+      ++p;
+    }
+  }
+  __syncthreads();  // shared memory may be reused by the block's next item
+}
+
+}  // namespace
+}  // namespace planimpl
+}  // namespace sdl

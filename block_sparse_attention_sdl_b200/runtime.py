@@ -23,9 +23,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (block_scores, dense_attn, make_shape, mask_budget, scores_workspace_bytes,
-               select_mask, select_shard_capacity, select_workspace_bytes, sparse_attn,
-               tile_plan)
+from . import (anchor_refresh, anchor_workspace_bytes, block_scores, dense_attn, make_shape,
+               mask_budget, scores_workspace_bytes, select_mask, select_shard_capacity,
+               select_workspace_bytes, sparse_attn, tile_plan)
 from .sharded import CudaStages, select_mask_sharded, torch_collectives
 
 
@@ -98,11 +98,21 @@ class StepSparseAttention:
         self.plan = (torch.empty((B, H, (self.nb + 1) // 2, 2), dtype=torch.int32, device=dev)
                      if block == 64 else None)
         self.mask_step = None  # anchor step whose mask is current
+        # the head-adaptive budget on one device: scores and selection in one launch
+        self.fused = not self.sharded and not self.per_head
+        self.ws_anchor = (torch.empty(max(anchor_workspace_bytes(probe_q, probe_k, block), 16),
+                                      dtype=torch.uint8, device=dev) if self.fused else None)
 
     def refresh(self, q, k, step: int, stream=None):
-        block_scores(q, k, self.block, scores=self.scores, workspace=self.ws_scores,
-                     stream=stream)
-        self.select(stream)
+        if self.fused:
+            # the tile plan runs apart: its own kernel is wider than the fused grid's blocks
+            anchor_refresh(q, k, self.block, self.sparsity, scores=self.scores,
+                           row_ptr=self.row_ptr, col_idx=self.col_idx, want_plan=False,
+                           workspace=self.ws_anchor, stream=stream)
+        else:
+            block_scores(q, k, self.block, scores=self.scores, workspace=self.ws_scores,
+                         stream=stream)
+            self.select(stream)
         if self.plan is not None:
             tile_plan(self.row_ptr, self.col_idx, self.B, self.H, self.L, self.block,
                       plan=self.plan, stream=stream)

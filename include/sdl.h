@@ -130,6 +130,21 @@ sdl_status sdl_select_mask_scoped(const float* scores, const sdl_shape* shape, d
                                   int64_t col_capacity, uint8_t* mask_u8, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/* ---- Fused anchor step ------------------------------------------------------
+ * sdl_block_scores, then sdl_select_mask (global budget per sequence, no
+ * mask_u8), then, when `plan` is not NULL (64-token blocks only),
+ * sdl_tile_plan, as one launch: the mask refresh of the Step-dLLM abstract's
+ * anchor steps.  Outputs are bit for bit those of the three calls.  `scores`
+ * (fp32 [B,H,nb,nb]) is written as well.  Arguments and errors as the three
+ * calls; one caller-owned workspace of sdl_anchor_workspace_bytes bytes.  The
+ * launch is cooperative (all its blocks resident at once); its grid barriers
+ * are bounded and a timeout raises SDL_ERR_TIMEOUT in sdl_last_device_status. */
+size_t sdl_anchor_workspace_bytes(const sdl_shape* shape);
+sdl_status sdl_anchor_refresh(const void* q, const void* k, const sdl_shape* shape, float scale,
+                              double sparsity, float* scores, int32_t* row_ptr,
+                              int32_t* col_idx, int64_t col_capacity, int32_t* plan,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- Mask selection with the heads of a sequence split over ranks ----------
  * The global budget of the Step-dLLM abstract (and the rule of sdl_select_mask)
  * when rank r of W holds the contiguous head range [h_r, h_r + H_local) of
