@@ -8,7 +8,9 @@ Every function takes numpy arrays laid out [B, L, heads, d] (uint16 holding
 bf16 bits, or float32) and returns float64 results.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-against closed forms, invariants, brute force or an independent library routine.
+(block-sparse path) and ``tests/test_oracle_col_pins.py`` (the column-sparse
+path of the PulseCol abstract) against closed forms, invariants, brute force or
+an independent library routine.
 """
 from __future__ import annotations
 
@@ -50,6 +52,13 @@ def lib():
         l.oracle_select.restype = _L
         l.oracle_attention.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P,
                                        _D, _P, _L, _P, _P, _I]
+        l.oracle_col_budget.argtypes = [_I, _D]
+        l.oracle_col_budget.restype = _L
+        l.oracle_col_scores.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _D, _P]
+        l.oracle_col_select.argtypes = [_P, _I, _I, _I, _D, _P]
+        l.oracle_col_select.restype = _L
+        l.oracle_col_attention.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P,
+                                           _I, _D, _P, _L, _P, _P, _I]
         _lib = l
     return _lib
 
@@ -155,6 +164,76 @@ def attention(q, k, v, bs, mask=None, scale=None, rows=None, nthreads=None):
                                 lse.ctypes.data, nthreads or os.cpu_count() or 1)
     if rc:
         raise ValueError("oracle_attention rejected its arguments")
+    if rows is None:
+        return O.reshape(B, H, L, d), lse.reshape(B, H, L)
+    return O, lse
+
+
+# ------------------------------------------------ column-sparse (PulseCol)
+
+def col_budget(L: int, sparsity: float) -> int:
+    """Columns kept per head: 64 * floor((1 - s) * L / 64 + 0.5), at least 64 (-1 if invalid)."""
+    return int(lib().oracle_col_budget(int(L), float(sparsity)))
+
+
+def col_scores(q: np.ndarray, k: np.ndarray, bs: int, scale: float | None = None) -> np.ndarray:
+    """S[b, h, u]: the mean over query blocks of softmax_u(scale * Qbar . k_u), fp64 [B, H, L]."""
+    B, L, H, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    code = _dtype_code(q)
+    assert _dtype_code(k) == code
+    S = np.empty((B, H, L), dtype=np.float64)
+    qs, ks = _strides(q), _strides(k)
+    rc = lib().oracle_col_scores(q.ctypes.data, k.ctypes.data, code, B, H, Hkv, L, d, bs,
+                                 qs.ctypes.data, ks.ctypes.data, float(scale), S.ctypes.data)
+    if rc:
+        raise ValueError("oracle_col_scores rejected its arguments")
+    return S
+
+
+def col_select(S: np.ndarray, sparsity: float) -> np.ndarray:
+    """int32 [B, H, Lc]: each head's Lc best columns (ties: lower index), ascending."""
+    S = np.ascontiguousarray(S, dtype=np.float64)
+    B, H, L = S.shape
+    Lc = col_budget(L, sparsity)
+    if Lc < 0:
+        raise ValueError("sparsity outside [0, 1) or L not a multiple of 64")
+    cols = np.empty((B, H, Lc), dtype=np.int32)
+    if lib().oracle_col_select(S.ctypes.data, B, H, L, float(sparsity), cols.ctypes.data) != Lc:
+        raise ValueError("oracle_col_select failed")
+    return cols
+
+
+def col_attention(q, k, v, cols, scale=None, rows=None, nthreads=None):
+    """Attention of every query row of head h over the columns cols[b, h, :] only:
+    O [B, H, L, d] and LSE [B, H, L] (or [n, d] / [n] for rows = int64 [n, 3] of (b, h, t))."""
+    B, L, H, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    code = _dtype_code(q)
+    assert _dtype_code(k) == code and _dtype_code(v) == code
+    cols = np.ascontiguousarray(cols, dtype=np.int32)
+    assert cols.shape[:2] == (B, H)
+    Lc = cols.shape[2]
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+        n = rows.shape[0]
+    else:
+        n = B * H * L
+    O = np.empty((n, d), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64)
+    qs, ks, vs = _strides(q), _strides(k), _strides(v)
+    rc = lib().oracle_col_attention(q.ctypes.data, k.ctypes.data, v.ctypes.data, code, B, H,
+                                    Hkv, L, d, qs.ctypes.data, ks.ctypes.data, vs.ctypes.data,
+                                    cols.ctypes.data, Lc, float(scale),
+                                    None if rows is None else rows.ctypes.data, n,
+                                    O.ctypes.data, lse.ctypes.data,
+                                    nthreads or os.cpu_count() or 1)
+    if rc:
+        raise ValueError("oracle_col_attention rejected its arguments")
     if rows is None:
         return O.reshape(B, H, L, d), lse.reshape(B, H, L)
     return O, lse

@@ -282,3 +282,209 @@ int oracle_attention(const void* q, const void* k, const void* v, int dtype, int
   }
   return err;
 }
+
+/* ---------------------------------------------- column-sparse attention */
+/*
+ * The PulseCol abstract ("PulseCol: periodically refreshed column-sparse
+ * attention for diffusion language models", same site, abstract): instead of
+ * blocks, a column-sparse pattern -- the key tokens (columns of the attention
+ * matrix) a query head keeps for all of its query rows -- found at an early
+ * denoising step and refreshed at a few later ones.  The abstract gives no
+ * estimator or budget; the reading written out here:
+ *
+ *   score:   S[b,h,u] = (1/nb) * sum over query blocks i of
+ *            softmax over u of (scale * Qbar[b,h,i,:] . k[b,u,h/g,:])
+ *            (block-mean queries against every key token)
+ *   budget:  Lc = 64 * floor((1 - s) * L / 64 + 0.5) columns per head, at
+ *            least 64 (whole 64-key tiles)
+ *   select:  the Lc largest S[b,h,u] of each head, ties by the lower u,
+ *            listed in ascending u
+ *   attend:  for every query token t of head h, softmax over the selected
+ *            keys only of (scale * q_t . k_u), times v_u (non-causal)
+ */
+
+int64_t oracle_col_budget(int L, double sparsity) {
+  if (!(sparsity >= 0.0 && sparsity < 1.0) || L <= 0 || L % 64) return -1;
+  int64_t c = 64 * (int64_t)floor((1.0 - sparsity) * (double)L / 64.0 + 0.5);
+  if (c < 64) c = 64;
+  return c;
+}
+
+int oracle_col_scores(const void* q, const void* k, int dtype, int B, int H, int Hkv, int L,
+                      int d, int bs, const int64_t* qs, const int64_t* ks, double scale,
+                      double* S) {
+  if (!q || !k || !S || Hkv <= 0 || H % Hkv || bs <= 0 || L % bs) return -1;
+  int nb = L / bs, g = H / Hkv;
+  double* qb = (double*)malloc(sizeof(double) * (size_t)B * H * nb * d);
+  double* z = (double*)malloc(sizeof(double) * (size_t)L);
+  if (!qb || !z) {
+    free(qb);
+    free(z);
+    return -2;
+  }
+  oracle_pool(q, dtype, B, L, H, d, bs, qs, qb);
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      int kh = h / g;
+      double* row = S + ((int64_t)b * H + h) * L;
+      for (int u = 0; u < L; ++u) row[u] = 0.0;
+      for (int i = 0; i < nb; ++i) {
+        const double* qi = qb + (((int64_t)b * H + h) * nb + i) * d;
+        double m = -INFINITY;
+        for (int u = 0; u < L; ++u) {
+          double s = 0.0;
+          int64_t ko = offs(ks, b, u, kh);
+          for (int c = 0; c < d; ++c) s += qi[c] * load_elem(k, dtype, ko + c);
+          z[u] = scale * s;
+          if (z[u] > m) m = z[u];
+        }
+        double sum = 0.0;
+        for (int u = 0; u < L; ++u) {
+          z[u] = exp(z[u] - m);
+          sum += z[u];
+        }
+        for (int u = 0; u < L; ++u) row[u] += z[u] / sum / (double)nb;
+      }
+    }
+  free(qb);
+  free(z);
+  return 0;
+}
+
+typedef struct {
+  double s;
+  int u;
+} colcand;
+
+/* larger score first, then the lower column */
+static int colcand_cmp(const void* a, const void* b) {
+  const colcand* x = (const colcand*)a;
+  const colcand* y = (const colcand*)b;
+  if (x->s > y->s) return -1;
+  if (x->s < y->s) return 1;
+  return (x->u > y->u) - (x->u < y->u);
+}
+
+static int int_cmp(const void* a, const void* b) {
+  int x = *(const int*)a, y = *(const int*)b;
+  return (x > y) - (x < y);
+}
+
+/* cols[b, h, 0 .. Lc) ascending; returns Lc or -1 */
+int64_t oracle_col_select(const double* S, int B, int H, int L, double sparsity, int32_t* cols) {
+  int64_t Lc = oracle_col_budget(L, sparsity);
+  if (Lc < 0 || !S || !cols || Lc > L) return -1;
+  colcand* c = (colcand*)malloc(sizeof(colcand) * (size_t)L);
+  int* pick = (int*)malloc(sizeof(int) * (size_t)Lc);
+  if (!c || !pick) {
+    free(c);
+    free(pick);
+    return -1;
+  }
+  for (int64_t r = 0; r < (int64_t)B * H; ++r) {
+    for (int u = 0; u < L; ++u) {
+      c[u].s = S[r * L + u];
+      c[u].u = u;
+    }
+    qsort(c, (size_t)L, sizeof(colcand), colcand_cmp);
+    for (int64_t x = 0; x < Lc; ++x) pick[x] = c[x].u;
+    qsort(pick, (size_t)Lc, sizeof(int), int_cmp);
+    for (int64_t x = 0; x < Lc; ++x) cols[r * Lc + x] = pick[x];
+  }
+  free(c);
+  free(pick);
+  return Lc;
+}
+
+typedef struct {
+  const void *q, *k, *v;
+  int dtype, B, H, Hkv, L, d;
+  const int64_t *qs, *ks, *vs;
+  const int32_t* cols;
+  int Lc;
+  double scale;
+  const int64_t* rows;
+  int64_t r0, r1;
+  double *O, *lse;
+  int err;
+} colattn_job;
+
+static void* colattn_worker(void* arg) {
+  colattn_job* j = (colattn_job*)arg;
+  int g = j->H / j->Hkv, d = j->d;
+  double* x = (double*)malloc(sizeof(double) * (size_t)j->Lc);
+  double* qv = (double*)malloc(sizeof(double) * (size_t)d);
+  double* acc = (double*)malloc(sizeof(double) * (size_t)d);
+  if (!x || !qv || !acc) {
+    j->err = -2;
+    free(x);
+    free(qv);
+    free(acc);
+    return NULL;
+  }
+  for (int64_t r = j->r0; r < j->r1; ++r) {
+    int b, h, t;
+    if (j->rows) {
+      b = (int)j->rows[3 * r];
+      h = (int)j->rows[3 * r + 1];
+      t = (int)j->rows[3 * r + 2];
+    } else {
+      b = (int)(r / ((int64_t)j->H * j->L));
+      h = (int)((r / j->L) % j->H);
+      t = (int)(r % j->L);
+    }
+    int kh = h / g;
+    const int32_t* cl = j->cols + ((int64_t)b * j->H + h) * j->Lc;
+    for (int c = 0; c < d; ++c) qv[c] = load_elem(j->q, j->dtype, offs(j->qs, b, t, h) + c);
+    double m = -INFINITY;
+    for (int x_ = 0; x_ < j->Lc; ++x_) {
+      double s = 0.0;
+      int64_t ko = offs(j->ks, b, cl[x_], kh);
+      for (int c = 0; c < d; ++c) s += qv[c] * load_elem(j->k, j->dtype, ko + c);
+      x[x_] = j->scale * s;
+      if (x[x_] > m) m = x[x_];
+    }
+    double l = 0.0;
+    for (int c = 0; c < d; ++c) acc[c] = 0.0;
+    for (int x_ = 0; x_ < j->Lc; ++x_) {
+      double p = exp(x[x_] - m);
+      l += p;
+      int64_t vo = offs(j->vs, b, cl[x_], kh);
+      for (int c = 0; c < d; ++c) acc[c] += p * load_elem(j->v, j->dtype, vo + c);
+    }
+    for (int c = 0; c < d; ++c) j->O[r * d + c] = acc[c] / l;
+    if (j->lse) j->lse[r] = m + log(l);
+  }
+  free(x);
+  free(qv);
+  free(acc);
+  return NULL;
+}
+
+/* O[r, :] and lse[r] for each requested row r = (b, h, t) (NULL: all, in
+ * (b, h, t) order), attending to the Lc columns cols[b, h, :] of each head. */
+int oracle_col_attention(const void* q, const void* k, const void* v, int dtype, int B, int H,
+                         int Hkv, int L, int d, const int64_t* qs, const int64_t* ks,
+                         const int64_t* vs, const int32_t* cols, int Lc, double scale,
+                         const int64_t* rows, int64_t n_rows, double* O, double* lse,
+                         int nthreads) {
+  if (!q || !k || !v || !O || !cols || Lc <= 0 || Hkv <= 0 || H % Hkv) return -1;
+  if (!rows) n_rows = (int64_t)B * H * L;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  if (nthreads > n_rows) nthreads = (int)(n_rows > 0 ? n_rows : 1);
+  pthread_t th[256];
+  colattn_job jobs[256];
+  for (int i = 0; i < nthreads; ++i) {
+    colattn_job jb = {q, k, v, dtype, B, H, Hkv, L, d, qs, ks, vs, cols, Lc, scale, rows,
+                      n_rows * i / nthreads, n_rows * (i + 1) / nthreads, O, lse, 0};
+    jobs[i] = jb;
+    pthread_create(&th[i], NULL, colattn_worker, &jobs[i]);
+  }
+  int err = 0;
+  for (int i = 0; i < nthreads; ++i) {
+    pthread_join(th[i], NULL);
+    if (jobs[i].err) err = jobs[i].err;
+  }
+  return err;
+}
