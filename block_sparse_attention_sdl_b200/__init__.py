@@ -30,6 +30,8 @@ EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspac
            "sdl_block_scores", "sdl_select_mask", "sdl_select_mask_noalloc", "sdl_sparse_attn",
            "sdl_tile_plan", "sdl_sparse_attn_planned", "sdl_dense_attn",
            "sdl_anchor_workspace_bytes", "sdl_anchor_refresh",
+           "sdl_col_budget", "sdl_col_scores_workspace_bytes", "sdl_col_scores",
+           "sdl_col_select", "sdl_col_gather", "sdl_col_sparse_attn",
            "sdl_select_shard_workspace_bytes", "sdl_select_shard_hist",
            "sdl_select_shard_capacity", "sdl_select_shard_pass", "sdl_select_shard_count",
            "sdl_select_shard_finish",
@@ -84,6 +86,14 @@ def _lib():
         L.sdl_tile_plan.argtypes = [P, P, SP, P, P]
         L.sdl_sparse_attn_planned.argtypes = [P, P, P, SP, P, P, P, F, P, P, P]
         L.sdl_dense_attn.argtypes = [P, P, P, SP, F, P, P, P]
+        L.sdl_col_budget.argtypes = [SP, D]
+        L.sdl_col_budget.restype = I64
+        L.sdl_col_scores_workspace_bytes.argtypes = [SP]
+        L.sdl_col_scores_workspace_bytes.restype = SZ
+        L.sdl_col_scores.argtypes = [P, P, SP, F, P, P, SZ, P]
+        L.sdl_col_select.argtypes = [P, SP, D, P, I64, P]
+        L.sdl_col_gather.argtypes = [P, P, SP, P, ctypes.c_int32, P, P, P]
+        L.sdl_col_sparse_attn.argtypes = [P, P, P, SP, ctypes.c_int32, F, P, P, P]
         L.sdl_anchor_workspace_bytes.argtypes = [SP]
         L.sdl_anchor_workspace_bytes.restype = SZ
         L.sdl_anchor_refresh.argtypes = [P, P, SP, F, D, P, P, P, I64, P, P, SZ, P]
@@ -102,7 +112,8 @@ def _lib():
         L.sdl_status_string.argtypes = [ctypes.c_int]
         L.sdl_status_string.restype = ctypes.c_char_p
         for f in ("sdl_block_scores", "sdl_select_mask", "sdl_select_mask_scoped",
-                  "sdl_anchor_refresh",
+                  "sdl_anchor_refresh", "sdl_col_scores", "sdl_col_select",
+                  "sdl_col_gather", "sdl_col_sparse_attn",
                   "sdl_select_shard_hist", "sdl_select_shard_pass", "sdl_select_shard_count",
                   "sdl_select_shard_finish",
                   "sdl_sparse_attn", "sdl_tile_plan",
@@ -272,6 +283,75 @@ def anchor_refresh(q, k, block: int, sparsity: float, scores=None, row_ptr=None,
                                      workspace.data_ptr(), workspace.numel(), _stream(stream)),
            "sdl_anchor_refresh")
     return scores, row_ptr, col_idx, plan
+
+
+def col_budget(q, k, block: int, sparsity: float) -> int:
+    """Columns kept per head (``sdl_col_budget``)."""
+    n = int(_lib().sdl_col_budget(ctypes.byref(make_shape(q, k, block)), float(sparsity)))
+    if n < 0:
+        raise SdlError(SDL_ERR_INVALID_ARG, "sdl_col_budget")
+    return n
+
+
+def col_scores(q, k, block: int, scale: float = 0.0, out=None, workspace=None, stream=None):
+    """fp32 [B, H, L] column scores (see ``sdl_col_scores``)."""
+    import torch
+    s = make_shape(q, k, block)
+    if out is None:
+        out = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
+    n = int(_lib().sdl_col_scores_workspace_bytes(ctypes.byref(s)))
+    workspace = _workspace(n, q.device, workspace)
+    _check(_lib().sdl_col_scores(q.data_ptr(), k.data_ptr(), ctypes.byref(s), float(scale),
+                                 out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                 _stream(stream)), "sdl_col_scores")
+    return out
+
+
+def col_select(col_scores_, q, k, block: int, sparsity: float, cols=None, stream=None):
+    """int32 [B, H, Lc]: each head's kept columns, ascending (see ``sdl_col_select``)."""
+    import torch
+    s = make_shape(q, k, block)
+    Lc = col_budget(q, k, block, sparsity)
+    if cols is None:
+        cols = torch.empty((s.B, s.H, Lc), dtype=torch.int32, device=q.device)
+    _check(_lib().sdl_col_select(col_scores_.data_ptr(), ctypes.byref(s), float(sparsity),
+                                 cols.data_ptr(), cols.numel(), _stream(stream)),
+           "sdl_col_select")
+    return cols
+
+
+def col_gather(k, v, cols, q, block: int, k_cols=None, v_cols=None, stream=None):
+    """The kept K and V tokens, [B, Lc, H, d] each (see ``sdl_col_gather``)."""
+    import torch
+    s = make_shape(q, k, block, v=v)
+    Lc = cols.shape[2]
+    if k_cols is None:
+        k_cols = torch.empty((s.B, Lc, s.H, s.d), dtype=k.dtype, device=k.device)
+    if v_cols is None:
+        v_cols = torch.empty((s.B, Lc, s.H, s.d), dtype=v.dtype, device=v.device)
+    _check(_lib().sdl_col_gather(k.data_ptr(), v.data_ptr(), ctypes.byref(s), cols.data_ptr(),
+                                 int(Lc), k_cols.data_ptr(), v_cols.data_ptr(), _stream(stream)),
+           "sdl_col_gather")
+    return k_cols, v_cols
+
+
+def col_sparse_attn(q, k_cols, v_cols, block: int = 64, scale: float = 0.0, out=None,
+                    want_lse: bool = False, lse=None, stream=None):
+    """Attention of every query token over its head's gathered columns
+    (see ``sdl_col_sparse_attn``); returns out, or (out, lse)."""
+    import torch
+    Lc = k_cols.shape[1]
+    s = make_shape(q, q, block, o=out if out is not None else q)
+    if out is None:
+        out = torch.empty_like(q)
+        s.o_strides[:] = _strides(out)
+    if lse is None and want_lse:
+        lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
+    _check(_lib().sdl_col_sparse_attn(q.data_ptr(), k_cols.data_ptr(), v_cols.data_ptr(),
+                                      ctypes.byref(s), int(Lc), float(scale), out.data_ptr(),
+                                      None if lse is None else lse.data_ptr(), _stream(stream)),
+           "sdl_col_sparse_attn")
+    return (out, lse) if want_lse else out
 
 
 def _score_shape(scores, block: int, L: int) -> Shape:

@@ -80,10 +80,11 @@ EncodeTiledFn encode_fn() {
 // swizzle.
 bool encode_bf16_map(CUtensorMap* map, const void* base, const sdl_shape& s, int heads,
                      const int64_t* st, cuuint32_t box_d = 64, cuuint32_t box_t = 64,
-                     CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+                     CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B, int tokens = 0) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)s.L, (cuuint64_t)heads, (cuuint64_t)s.B};
+  cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)(tokens > 0 ? tokens : s.L),
+                        (cuuint64_t)heads, (cuuint64_t)s.B};
   cuuint64_t strides[3] = {(cuuint64_t)st[1] * 2, (cuuint64_t)st[2] * 2, (cuuint64_t)st[0] * 2};
   // a zero stride (broadcast) is not expressible: use the dimension's natural size
   for (int i = 0; i < 3; ++i)
@@ -96,9 +97,10 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, const sdl_shape& s, int
   return r == CUDA_SUCCESS;
 }
 
+// Lk: key and value tokens (0: L, the same as the queries).
 sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_shape* shape,
                        const int32_t* row_ptr, const int32_t* col_idx, const int32_t* plan,
-                       float scale, void* o, float* lse, void* stream) {
+                       float scale, void* o, float* lse, void* stream, int Lk = 0) {
   sdl_status e = check_shape(shape);
   if (e) return e;
   const sdl_shape& s = *shape;
@@ -126,6 +128,7 @@ sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_sh
   a.d = s.d;
   a.block = s.block;
   a.nb = s.L / s.block;
+  a.Lk = Lk > 0 ? Lk : s.L;
   for (int i = 0; i < 3; ++i) {
     a.qs[i] = s.q_strides[i];
     a.ks[i] = s.k_strides[i];
@@ -140,8 +143,10 @@ sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_sh
   if (s.dtype == SDL_BF16) {
     CUtensorMap tq, tk, tv, to;
     if (!encode_bf16_map(&tq, q, s, s.H, s.q_strides) ||
-        !encode_bf16_map(&tk, k, s, s.H_kv, s.k_strides) ||
-        !encode_bf16_map(&tv, v, s, s.H_kv, s.v_strides) ||
+        !encode_bf16_map(&tk, k, s, s.H_kv, s.k_strides, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+                         a.Lk) ||
+        !encode_bf16_map(&tv, v, s, s.H_kv, s.v_strides, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+                         a.Lk) ||
         !encode_bf16_map(&to, o, s, s.H, s.o_strides, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
       return cuda_fail(cudaErrorInvalidValue);
     ce = launch_attn_tc(a, &tq, &tk, &tv, &to, st);
@@ -319,6 +324,95 @@ sdl_status sdl_anchor_refresh(const void* q, const void* k, const sdl_shape* sha
                                  static_cast<cudaStream_t>(stream));
   if (ce != cudaSuccess) return cuda_fail(ce);
   return SDL_OK;
+}
+
+// ------------------------------------------------- column-sparse attention
+
+int64_t sdl_col_budget(const sdl_shape* shape, double sparsity) {
+  if (check_shape(shape) != SDL_OK) return -1;
+  if (!(sparsity >= 0.0 && sparsity < 1.0)) return -1;
+  int64_t c = 64 * (int64_t)floor((1.0 - sparsity) * (double)shape->L / 64.0 + 0.5);
+  if (c < 64) c = 64;
+  return c > shape->L ? shape->L : c;
+}
+
+size_t sdl_col_scores_workspace_bytes(const sdl_shape* shape) {
+  if (check_shape(shape) != SDL_OK) return 0;
+  const size_t nb = shape->L / shape->block;
+  return align256(sdl_scores_workspace_bytes(shape)) +
+         align256(sizeof(float) * 2 * shape->B * shape->H * nb);
+}
+
+sdl_status sdl_col_scores(const void* q, const void* k, const sdl_shape* shape, float scale,
+                          float* col_scores, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  const sdl_shape& s = *shape;
+  if (!q || !k || !col_scores) return SDL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(col_scores)) return SDL_ERR_INVALID_ARG;
+  if ((e = check_strides(s.q_strides, s.dtype)) || (e = check_strides(s.k_strides, s.dtype)))
+    return e;
+  const size_t need = sdl_col_scores_workspace_bytes(shape);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SDL_ERR_WORKSPACE;
+  const size_t nb = s.L / s.block;
+  char* w = static_cast<char*>(workspace);
+  float* qbar = reinterpret_cast<float*>(w);
+  float* kbar = reinterpret_cast<float*>(w + align256(sizeof(float) * s.B * s.H * nb * s.d));
+  float2* stats = reinterpret_cast<float2*>(w + align256(sdl_scores_workspace_bytes(shape)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t ce = launch_pool(q, k, s, qbar, kbar, st);
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  ce = launch_col_scores(k, s, resolve_scale(scale, s.d), qbar, stats, col_scores, st);
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_col_select(const float* col_scores, const sdl_shape* shape, double sparsity,
+                          int32_t* cols, int64_t col_capacity, void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  if (!col_scores || !cols) return SDL_ERR_INVALID_ARG;
+  const int64_t Lc = sdl_col_budget(shape, sparsity);
+  if (Lc < 0) return SDL_ERR_INVALID_ARG;
+  if (col_capacity < Lc * shape->B * shape->H) return SDL_ERR_CAPACITY;
+  cudaError_t ce = launch_col_select(col_scores, shape->B * shape->H, shape->L, (int)Lc, cols,
+                                     static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_col_gather(const void* k, const void* v, const sdl_shape* shape,
+                          const int32_t* cols, int32_t Lc, void* k_cols, void* v_cols,
+                          void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  const sdl_shape& s = *shape;
+  if (!k || !v || !cols || !k_cols || !v_cols || Lc <= 0 || Lc > s.L) return SDL_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cols) || !aligned16(v_cols))
+    return SDL_ERR_INVALID_ARG;
+  if ((e = check_strides(s.k_strides, s.dtype)) || (e = check_strides(s.v_strides, s.dtype)))
+    return e;
+  cudaError_t ce = launch_col_gather(k, v, s, cols, Lc, k_cols, v_cols,
+                                     static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_col_sparse_attn(const void* q, const void* k_cols, const void* v_cols,
+                               const sdl_shape* shape, int32_t Lc, float scale, void* o,
+                               float* lse, void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  if (Lc <= 0 || Lc % 64 || Lc > shape->L) return SDL_ERR_INVALID_ARG;
+  // the gathered tensors: one per query head, contiguous [B, Lc, H, d]
+  sdl_shape loc = *shape;
+  loc.H_kv = shape->H;
+  const int64_t st[3] = {(int64_t)Lc * shape->H * shape->d, (int64_t)shape->H * shape->d,
+                         (int64_t)shape->d};
+  for (int i = 0; i < 3; ++i) loc.k_strides[i] = loc.v_strides[i] = st[i];
+  return attn_common(q, k_cols, v_cols, &loc, nullptr, nullptr, nullptr, scale, o, lse, stream,
+                     Lc);
 }
 
 // ------------------------------------------------- heads split over ranks

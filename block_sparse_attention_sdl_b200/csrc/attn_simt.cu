@@ -27,7 +27,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int t0 = tile * kRows;
   const int kh = h / (a.H / a.Hkv);
-  const int nsub = a.L / kSubBlock;
+  const int nsub = a.Lk / kSubBlock;
   const int tid = threadIdx.x;
 
   // ---- kept 64-token key sub-blocks of this tile's query block, ascending

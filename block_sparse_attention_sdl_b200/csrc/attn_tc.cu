@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kItemWarp) {
     // ====================================================== item producer
-    const int nsub = a.L / kSubBlock;
+    const int nsub = a.Lk / kSubBlock;
     int pub0 = 0, pub1 = 0;  // slots published per stream (end marker included)
     bool ended0 = false, ended1 = false;
     bool exhausted = false;  // the launch's counter ran out

@@ -1,0 +1,348 @@
+// Column-sparse attention of the PulseCol abstract: every query head keeps a
+// set of key tokens (columns of the attention matrix) for all of its query
+// rows, chosen at a refresh step and reused until the next one.
+//
+// The abstract gives no estimator or budget; the reading implemented here:
+//   score:  S[b,h,u] = (1/nb) * sum over query blocks i of
+//           softmax over u of (scale * Qbar[b,h,i,:] . k[b,u,h/g,:])
+//   budget: Lc = 64 * floor((1 - s) * L / 64 + 0.5) columns per head, at
+//           least 64 (whole 64-key tiles)
+//   select: the Lc largest S[b,h,:] of each head, ties to the lower u,
+//           listed in ascending u
+//   attend: softmax over the kept keys only, for every query token of the head
+//
+// Kernels:
+//   col_stats_kernel  per (b, h, 16 query blocks): row max and sum of the
+//                     block-mean queries' logits over every key (fp32 FFMA).
+//   col_sum_kernel    per (b, h, 64 keys): the column sums of the softmax
+//                     weights, over the query blocks in a fixed order (no
+//                     atomics: the same bits on every run).
+//   col_select_kernel per (b, h): radix select of the Lc-th largest score
+//                     (digits of 11, 11, 10 bits), then the kept columns in
+//                     ascending order.
+//   col_gather_kernel the kept K and V tokens into dense [B, Lc, H, d]
+//                     tensors (one per query head); the attention kernel then
+//                     walks them as dense keys (attn_tc.cu, key length Lc).
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "internal.cuh"
+#include "select_impl.cuh"
+
+namespace sdl {
+namespace {
+
+using selimpl::block_excl_scan;
+
+struct ColArgs {
+  int B, H, Hkv, L, d, nb;
+  float scale;
+  int64_t ks[3], vs[3];  // (b, t, h) strides of K and V, in elements
+};
+
+void fill_col_args(ColArgs& c, const sdl_shape& s, float scale) {
+  c.B = s.B;
+  c.H = s.H;
+  c.Hkv = s.H_kv;
+  c.L = s.L;
+  c.d = s.d;
+  c.nb = s.L / s.block;
+  c.scale = scale;
+  for (int i = 0; i < 3; ++i) {
+    c.ks[i] = s.k_strides[i];
+    c.vs[i] = s.v_strides[i];
+  }
+}
+
+constexpr int kCR = 16;   // query blocks per tile
+constexpr int kCK = 64;   // keys per tile
+constexpr int kCThreads = 128;
+
+// qs [kCR][d+4] (block-mean queries), ks [kCK][d+4] (keys as fp32)
+inline size_t col_smem_bytes(int d) { return sizeof(float) * (size_t)(kCR + kCK) * (d + 4); }
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+// Rows i0 .. i0+kCR of Qbar (head h) into qs; zero rows past nb.
+__device__ __forceinline__ void load_q_tile(const float* __restrict__ qsrc, int nb, int d, int i0,
+                                            float* qs) {
+  const int dp = d + 4, d4 = d / 4;
+  for (int x = threadIdx.x; x < kCR * d4; x += kCThreads) {
+    const int r = x / d4, c = (x % d4) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i0 + r < nb) v = *reinterpret_cast<const float4*>(qsrc + (int64_t)(i0 + r) * d + c);
+    *reinterpret_cast<float4*>(qs + r * dp + c) = v;
+  }
+}
+
+// Keys u0 .. u0+kCK of KV head kh into ks (fp32).
+template <typename T>
+__device__ __forceinline__ void load_k_tile(const T* __restrict__ k, const int64_t* ks, int b,
+                                            int kh, int d, int u0, float* kt) {
+  const int dp = d + 4;
+  for (int x = threadIdx.x; x < kCK * d; x += kCThreads) {
+    const int r = x / d, c = x % d;
+    kt[r * dp + c] = to_f<T>(k[b * ks[0] + (int64_t)(u0 + r) * ks[1] + kh * ks[2] + c]);
+  }
+}
+
+// z[a][u] for the thread's 4 rows (ty*4 + a) and 2 keys (tx, tx + 32).
+__device__ __forceinline__ void tile_logits(const float* qs, const float* kt, int d, float scale,
+                                            float (&z)[4][2]) {
+  const int dp = d + 4, ty = threadIdx.x / 32, tx = threadIdx.x % 32;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) z[a][0] = z[a][1] = 0.f;
+  for (int c = 0; c < d; c += 4) {
+    const float4 k0 = *reinterpret_cast<const float4*>(kt + tx * dp + c);
+    const float4 k1 = *reinterpret_cast<const float4*>(kt + (tx + 32) * dp + c);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const float4 q = *reinterpret_cast<const float4*>(qs + (ty * 4 + a) * dp + c);
+      z[a][0] += q.x * k0.x + q.y * k0.y + q.z * k0.z + q.w * k0.w;
+      z[a][1] += q.x * k1.x + q.y * k1.y + q.z * k1.z + q.w * k1.w;
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    z[a][0] *= scale;
+    z[a][1] *= scale;
+  }
+}
+
+// grid (ceil(nb / kCR), H, B): stats[b, h, i] = (max over u of z_iu, sum over u
+// of exp(z_iu - max)).
+template <typename T>
+__global__ void __launch_bounds__(kCThreads) col_stats_kernel(const float* __restrict__ qbar,
+                                                              const T* __restrict__ k, ColArgs c,
+                                                              float2* __restrict__ stats) {
+  extern __shared__ float sm[];
+  float* qs = sm;
+  float* kt = qs + kCR * (c.d + 4);
+  const int b = blockIdx.z, h = blockIdx.y, i0 = blockIdx.x * kCR;
+  const int kh = h / (c.H / c.Hkv);
+  load_q_tile(qbar + ((int64_t)b * c.H + h) * c.nb * c.d, c.nb, c.d, i0, qs);
+  float m[4], l[4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    m[a] = -INFINITY;
+    l[a] = 0.f;
+  }
+  for (int u0 = 0; u0 < c.L; u0 += kCK) {
+    __syncthreads();
+    load_k_tile<T>(k, c.ks, b, kh, c.d, u0, kt);
+    __syncthreads();
+    float z[4][2];
+    tile_logits(qs, kt, c.d, c.scale, z);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const float mt = fmaxf(m[a], fmaxf(z[a][0], z[a][1]));
+      l[a] = l[a] * expf(m[a] - mt) + expf(z[a][0] - mt) + expf(z[a][1] - mt);
+      m[a] = mt;
+    }
+  }
+  // merge the 32 lanes' partial (max, sum) of each row, in a fixed order
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m[a], o);
+      const float l2 = __shfl_xor_sync(0xffffffffu, l[a], o);
+      const float mt = fmaxf(m[a], m2);
+      l[a] = l[a] * expf(m[a] - mt) + l2 * expf(m2 - mt);
+      m[a] = mt;
+    }
+    const int i = i0 + (threadIdx.x / 32) * 4 + a;
+    if (threadIdx.x % 32 == 0 && i < c.nb)
+      stats[((int64_t)b * c.H + h) * c.nb + i] = make_float2(m[a], l[a]);
+  }
+}
+
+// grid (L / kCK, H, B): S[b, h, u] = (1/nb) sum over i of exp(z_iu - max_i) / sum_i.
+template <typename T>
+__global__ void __launch_bounds__(kCThreads) col_sum_kernel(const float* __restrict__ qbar,
+                                                            const T* __restrict__ k, ColArgs c,
+                                                            const float2* __restrict__ stats,
+                                                            float* __restrict__ S) {
+  extern __shared__ float sm[];
+  float* qs = sm;
+  float* kt = qs + kCR * (c.d + 4);
+  __shared__ float part[kCThreads / 32][kCK];
+  const int b = blockIdx.z, h = blockIdx.y, u0 = blockIdx.x * kCK;
+  const int kh = h / (c.H / c.Hkv);
+  const int ty = threadIdx.x / 32, tx = threadIdx.x % 32;
+  load_k_tile<T>(k, c.ks, b, kh, c.d, u0, kt);
+  const float* qsrc = qbar + ((int64_t)b * c.H + h) * c.nb * c.d;
+  const float2* st = stats + ((int64_t)b * c.H + h) * c.nb;
+  float acc0 = 0.f, acc1 = 0.f;
+  for (int i0 = 0; i0 < c.nb; i0 += kCR) {
+    __syncthreads();
+    load_q_tile(qsrc, c.nb, c.d, i0, qs);
+    __syncthreads();
+    float z[4][2];
+    tile_logits(qs, kt, c.d, c.scale, z);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int i = i0 + ty * 4 + a;
+      if (i < c.nb) {
+        const float2 s2 = st[i];
+        const float inv = 1.0f / s2.y;
+        acc0 += expf(z[a][0] - s2.x) * inv;
+        acc1 += expf(z[a][1] - s2.x) * inv;
+      }
+    }
+  }
+  part[ty][tx] = acc0;
+  part[ty][tx + 32] = acc1;
+  __syncthreads();
+  if (threadIdx.x < kCK) {
+    float t = 0.f;
+    for (int w = 0; w < kCThreads / 32; ++w) t += part[w][threadIdx.x];
+    S[((int64_t)b * c.H + h) * c.L + u0 + threadIdx.x] = t / (float)c.nb;
+  }
+}
+
+constexpr int kSelThreads = 1024;
+
+// grid B * H: cols[bh, 0 .. Lc) = the Lc largest S[bh, :] (ties: lower u), ascending.
+__global__ void __launch_bounds__(kSelThreads) col_select_kernel(const float* __restrict__ S,
+                                                                 int L, int Lc,
+                                                                 int32_t* __restrict__ cols) {
+  __shared__ int hist[2048];
+  __shared__ int s_warp[32];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_krem;
+  const int tid = threadIdx.x;
+  const int64_t bh = blockIdx.x;
+  const uint32_t* keys = reinterpret_cast<const uint32_t*>(S + bh * L);  // scores >= 0
+  int32_t* out = cols + bh * Lc;
+  uint32_t prefix = 0;
+  int krem = Lc;  // the Lc-th largest key
+#pragma unroll
+  for (int p = 0; p < 3; ++p) {
+    const int width = p < 2 ? 11 : 10, shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
+    const int nbin = 1 << width, hs = shift + width;
+    for (int x = tid; x < nbin; x += kSelThreads) hist[x] = 0;
+    __syncthreads();
+    for (int u = tid; u < L; u += kSelThreads) {
+      const uint32_t key = keys[u];
+      if (hs >= 32 || (key >> hs) == (prefix >> hs))
+        atomicAdd(&hist[(key >> shift) & (uint32_t)(nbin - 1)], 1);
+    }
+    __syncthreads();
+    // thread t owns bins [nbin - per (t+1), nbin - per t): the top bins first
+    const int per = nbin / kSelThreads;  // 2 or 1
+    const int hi = nbin - per * tid;
+    int cnt[2] = {0, 0}, local = 0;
+    for (int x = 0; x < per; ++x) {
+      cnt[x] = hist[hi - 1 - x];
+      local += cnt[x];
+    }
+    int total = 0;
+    int above = block_excl_scan(local, s_warp, total);
+    for (int x = 0; x < per; ++x) {
+      if (above < krem && above + cnt[x] >= krem) {
+        s_prefix = prefix | ((uint32_t)(hi - 1 - x) << shift);
+        s_krem = krem - above;
+      }
+      above += cnt[x];
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    krem = s_krem;
+    __syncthreads();
+  }
+  // keys above the threshold, then krem of its ties in ascending u
+  const uint32_t tau = prefix;
+  int carry_sel = 0, carry_tie = 0;
+  for (int u0 = 0; u0 < L; u0 += kSelThreads) {
+    const int u = u0 + tid;
+    const uint32_t key = u < L ? keys[u] : 0u;
+    const bool gt = u < L && key > tau;
+    const bool tie = u < L && key == tau;
+    int tot_tie = 0;
+    const int tie_before = carry_tie + block_excl_scan(tie ? 1 : 0, s_warp, tot_tie);
+    const bool sel = gt || (tie && tie_before < krem);
+    int tot_sel = 0;
+    const int pos = carry_sel + block_excl_scan(sel ? 1 : 0, s_warp, tot_sel);
+    if (sel && pos < Lc) out[pos] = u;
+    carry_tie += tot_tie;
+    carry_sel += tot_sel;
+  }
+}
+
+// kc[b, c, h, :] = k[b, cols[b, h, c], h / g, :] and likewise v, 16 bytes per thread.
+__global__ void col_gather_kernel(const uint8_t* __restrict__ k, const uint8_t* __restrict__ v,
+                                  ColArgs c, const int32_t* __restrict__ cols, int Lc,
+                                  int esize, uint8_t* __restrict__ kc, uint8_t* __restrict__ vc) {
+  const int per = 16 / esize;  // elements per 16 bytes
+  const int chunks = c.d / per;
+  const int64_t n = (int64_t)c.B * Lc * c.H * chunks;
+  const int g = c.H / c.Hkv;
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n;
+       x += (int64_t)gridDim.x * blockDim.x) {
+    const int ch = (int)(x % chunks);
+    const int h = (int)((x / chunks) % c.H);
+    const int cc = (int)((x / ((int64_t)chunks * c.H)) % Lc);
+    const int b = (int)(x / ((int64_t)chunks * c.H * Lc));
+    const int u = cols[((int64_t)b * c.H + h) * Lc + cc];
+    const int64_t src_k = (b * c.ks[0] + (int64_t)u * c.ks[1] + (h / g) * c.ks[2]) * esize +
+                          (int64_t)ch * 16;
+    const int64_t src_v = (b * c.vs[0] + (int64_t)u * c.vs[1] + (h / g) * c.vs[2]) * esize +
+                          (int64_t)ch * 16;
+    const int64_t dst = (((int64_t)b * Lc + cc) * c.H + h) * (int64_t)c.d * esize + (int64_t)ch * 16;
+    *reinterpret_cast<uint4*>(kc + dst) = __ldg(reinterpret_cast<const uint4*>(k + src_k));
+    *reinterpret_cast<uint4*>(vc + dst) = __ldg(reinterpret_cast<const uint4*>(v + src_v));
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_col_scores(const void* k, const sdl_shape& s, float scale, const float* qbar,
+                              float2* stats, float* S, cudaStream_t st) {
+  ColArgs c;
+  fill_col_args(c, s, scale);
+  const size_t smem = col_smem_bytes(s.d);
+  const dim3 g1((c.nb + kCR - 1) / kCR, s.H, s.B), g2(s.L / kCK, s.H, s.B);
+  if (s.dtype == SDL_BF16) {
+    col_stats_kernel<__nv_bfloat16><<<g1, kCThreads, smem, st>>>(
+        qbar, static_cast<const __nv_bfloat16*>(k), c, stats);
+    col_sum_kernel<__nv_bfloat16><<<g2, kCThreads, smem, st>>>(
+        qbar, static_cast<const __nv_bfloat16*>(k), c, stats, S);
+  } else {
+    col_stats_kernel<float><<<g1, kCThreads, smem, st>>>(qbar, static_cast<const float*>(k), c,
+                                                          stats);
+    col_sum_kernel<float><<<g2, kCThreads, smem, st>>>(qbar, static_cast<const float*>(k), c,
+                                                        stats, S);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_col_select(const float* S, int BH, int L, int Lc, int32_t* cols,
+                              cudaStream_t st) {
+  col_select_kernel<<<BH, kSelThreads, 0, st>>>(S, L, Lc, cols);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_col_gather(const void* k, const void* v, const sdl_shape& s,
+                              const int32_t* cols, int Lc, void* kc, void* vc, cudaStream_t st) {
+  ColArgs c;
+  fill_col_args(c, s, 0.f);
+  const int esize = s.dtype == SDL_BF16 ? 2 : 4;
+  const int64_t n = (int64_t)s.B * Lc * s.H * (s.d * esize / 16);
+  int64_t grid = (n + 255) / 256;
+  if (grid > 148 * 16) grid = 148 * 16;
+  col_gather_kernel<<<(unsigned)grid, 256, 0, st>>>(
+      static_cast<const uint8_t*>(k), static_cast<const uint8_t*>(v), c, cols, Lc, esize,
+      static_cast<uint8_t*>(kc), static_cast<uint8_t*>(vc));
+  return cudaGetLastError();
+}
+
+}  // namespace sdl

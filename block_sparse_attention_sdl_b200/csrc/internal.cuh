@@ -32,6 +32,7 @@ struct AttnArgs {
   const int32_t* col_idx;
   const int32_t* plan;     // tile plan for 64-token blocks (null: adjacent pairs)
   int B, H, Hkv, L, d, block, nb;
+  int Lk;  // key (and value) tokens: L, or the gathered columns of column-sparse attention
   int64_t qs[3], ks[3], vs[3], os[3];
   float scale_log2;  // scale * log2(e)
   float scale;
@@ -60,6 +61,13 @@ cudaError_t launch_anchor(const void* q, const void* k, const sdl_shape& s, floa
                           int32_t* row_ptr, int32_t* col_idx, int32_t* plan, unsigned* bar,
                           int* status, cudaStream_t st);
 size_t anchor_barrier_bytes();
+// column-sparse attention (col.cu)
+cudaError_t launch_col_scores(const void* k, const sdl_shape& s, float scale, const float* qbar,
+                              float2* stats, float* S, cudaStream_t st);
+cudaError_t launch_col_select(const float* S, int BH, int L, int Lc, int32_t* cols,
+                              cudaStream_t st);
+cudaError_t launch_col_gather(const void* k, const void* v, const sdl_shape& s,
+                              const int32_t* cols, int Lc, void* kc, void* vc, cudaStream_t st);
 size_t select_hist_offset(int B, int pass);
 size_t select_hist_count(int B);
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,

@@ -130,6 +130,41 @@ sdl_status sdl_select_mask_scoped(const float* scores, const sdl_shape* shape, d
                                   int64_t col_capacity, uint8_t* mask_u8, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/* ---- Column-sparse attention (the PulseCol abstract) ------------------------
+ * Every query head keeps a set of key tokens ("columns") for all of its query
+ * rows; the set is chosen at refresh steps and reused between them.  The
+ * abstract gives no estimator or budget; this library's reading:
+ *   sdl_col_scores:  S[b,h,u] = (1/nb) sum over query blocks i of
+ *                    softmax over u of (scale * Qbar[b,h,i,:] . k[b,u,h/g,:]),
+ *                    fp32 [B, H, L], Qbar the block means of Q (block = shape
+ *                    block); workspace sdl_col_scores_workspace_bytes
+ *   sdl_col_budget:  Lc = 64 * floor((1 - s) * L / 64 + 0.5) columns per head,
+ *                    at least 64 and at most L (-1 on bad arguments)
+ *   sdl_col_select:  cols int32 [B, H, Lc]: each head's Lc largest S, ties to
+ *                    the lower u, ascending (col_capacity elements of room, at
+ *                    least B*H*Lc, else SDL_ERR_CAPACITY)
+ *   sdl_col_gather:  k_cols[b,c,h,:] = k[b, cols[b,h,c], h/g, :] and likewise
+ *                    v, contiguous [B, Lc, H, d] of the shape's dtype (K/V
+ *                    duplicated per query head under GQA)
+ *   sdl_col_sparse_attn: O[b,t,h,:] = sum over c of softmax_c(scale * q_t .
+ *                    k_cols[b,c,h,:]) v_cols[b,c,h,:] for every query token t,
+ *                    optional LSE [B,H,L]; Lc a multiple of 64.  Q and O as in
+ *                    sdl_dense_attn (the shape's k/v strides are ignored).
+ * All asynchronous on `stream`; errors as the block-sparse calls. */
+int64_t sdl_col_budget(const sdl_shape* shape, double sparsity);
+size_t sdl_col_scores_workspace_bytes(const sdl_shape* shape);
+sdl_status sdl_col_scores(const void* q, const void* k, const sdl_shape* shape, float scale,
+                          float* col_scores, void* workspace, size_t workspace_bytes,
+                          void* stream);
+sdl_status sdl_col_select(const float* col_scores, const sdl_shape* shape, double sparsity,
+                          int32_t* cols, int64_t col_capacity, void* stream);
+sdl_status sdl_col_gather(const void* k, const void* v, const sdl_shape* shape,
+                          const int32_t* cols, int32_t Lc, void* k_cols, void* v_cols,
+                          void* stream);
+sdl_status sdl_col_sparse_attn(const void* q, const void* k_cols, const void* v_cols,
+                               const sdl_shape* shape, int32_t Lc, float scale, void* o,
+                               float* lse, void* stream);
+
 /* ---- Fused anchor step ------------------------------------------------------
  * sdl_block_scores, then sdl_select_mask (global budget per sequence, no
  * mask_u8), then, when `plan` is not NULL (64-token blocks only),
