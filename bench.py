@@ -55,12 +55,14 @@ def parse():
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--variant", choices=["step-dllm", "uniform-head", "sparsed"],
+    p.add_argument("--variant", choices=["step-dllm", "uniform-head", "sparsed", "pulsecol"],
                    default="step-dllm",
                    help="step-dllm: head-adaptive global budget, mask refreshed every anchor "
                         "interval (the headline); uniform-head: the same schedule with a "
                         "uniform per-head budget; sparsed: dense attention for the first "
-                        "--dense-steps steps, then one mask reused for every later step")
+                        "--dense-steps steps, then one mask reused for every later step; "
+                        "pulsecol: column-sparse attention (key tokens kept per head, "
+                        "refreshed every anchor interval, same FLOP budget)")
     p.add_argument("--shard", choices=["sequences", "heads"], default="sequences",
                    help="sequences: every rank its own independent sequence (weak scaling, no "
                         "collective); heads: the ranks split the heads of one sequence, the "
@@ -162,11 +164,16 @@ class Runner:
         self.shard = shard
         self.H, self.H_kv = (w.H, w.H_kv) if shard is None else (shard[1] - shard[0],
                                                                  shard[3] - shard[2])
-        self.att = runtime.StepSparseAttention(
-            w.B, self.H, self.H_kv, w.L, w.d, w.bs, w.sparsity, self.interval, device=device,
-            budget="head" if variant == "uniform-head" else "sequence",
-            dense_steps=self.dense_steps, heads_total=None if shard is None else w.H,
-            rank=rank)
+        self.pulsecol = variant == "pulsecol"
+        if self.pulsecol:
+            self.att = runtime.ColSparseAttention(w.B, self.H, self.H_kv, w.L, w.d, w.bs,
+                                                  w.sparsity, self.interval, device=device)
+        else:
+            self.att = runtime.StepSparseAttention(
+                w.B, self.H, self.H_kv, w.L, w.d, w.bs, w.sparsity, self.interval,
+                device=device, budget="head" if variant == "uniform-head" else "sequence",
+                dense_steps=self.dense_steps, heads_total=None if shard is None else w.H,
+                rank=rank)
         self.out = torch.empty((w.B, w.L, self.H, w.d), dtype=torch.bfloat16, device=device)
         self.seed = seed
         self.kinds = []  # per attention launch: "sparse" or "dense"
@@ -199,12 +206,24 @@ class Runner:
             self.kinds.append("dense" if dense else "sparse")
         if dense:
             self.sdl.dense_attn(x["q"], x["k"], x["v"], w.bs, out=self.out)
+        elif self.pulsecol:
+            att.attend(x["q"], x["k"], x["v"], out=self.out)
         else:
             self.sdl.sparse_attn(x["q"], x["k"], x["v"], att.row_ptr, att.col_idx, w.bs,
                                  out=self.out, plan=att.plan)
         if ev is not None:
             ev["s1"].append(torch.cuda.Event(enable_timing=True))
             ev["s1"][-1].record()
+
+    def prime(self, x):
+        """Run the anchor and attention kernels once, untimed (see main)."""
+        self.att.refresh(x["q"], x["k"], 0)
+        if self.pulsecol:
+            self.att.attend(x["q"], x["k"], x["v"], out=self.out)
+        else:
+            self.sdl.sparse_attn(x["q"], x["k"], x["v"], self.att.row_ptr, self.att.col_idx,
+                                 self.w.bs, out=self.out, plan=self.att.plan)
+        self.att.mask_step = None
 
 
 def barrier(dist_on):
@@ -442,11 +461,7 @@ def main():
     # A schedule that starts with dense steps launches no anchor or sparse kernel
     # while warming up: run each once, untimed, so that none is loaded inside the
     # timed region.  The timed schedule then builds its own masks.
-    x0 = inputs[0]
-    runner.att.refresh(x0["q"], x0["k"], 0)
-    runner.sdl.sparse_attn(x0["q"], x0["k"], x0["v"], runner.att.row_ptr, runner.att.col_idx,
-                           w.bs, out=runner.out, plan=runner.att.plan)
-    runner.att.mask_step = None
+    runner.prime(inputs[0])
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
@@ -496,8 +511,12 @@ def main():
         return a.elapsed_time(b) / n
 
     att = runner.att
-    sc_ms = ev_time(lambda: sdl.block_scores(x0["q"], x0["k"], w.bs, scores=att.scores,
-                                             workspace=att.ws_scores))
+    if runner.pulsecol:
+        sc_ms = ev_time(lambda: sdl.col_scores(x0["q"], x0["k"], w.bs, out=att.col_scores,
+                                               workspace=att.ws))
+    else:
+        sc_ms = ev_time(lambda: sdl.block_scores(x0["q"], x0["k"], w.bs, scores=att.scores,
+                                                 workspace=att.ws_scores))
     se_ms = ev_time(att.select)
     score_bytes = (2 * w.B * w.L * (runner.H + runner.H_kv) * w.d +
                    4 * w.B * runner.H * w.nb * w.nb)
@@ -528,7 +547,8 @@ def main():
         cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
 
     n_anchor = len(anchor_ms)
-    traffic = traffic_record()
+    # the ncu record covers the block-sparse kernel's launch only
+    traffic = None if runner.pulsecol else traffic_record()
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": len(steps), "warmup": args.warmup, "ms_per_step": ms_max / len(steps),
@@ -540,7 +560,9 @@ def main():
                    "heads": w.H, "kv_heads": w.H_kv, "head_dim": w.d, "block": w.bs,
                    "sparsity": w.sparsity, "anchor_every": runner.interval,
                    "dense_steps": runner.dense_steps,
-                   "budget": "per head" if runner.att.per_head else "per sequence, across heads",
+                   "budget": ("key columns per head" if runner.pulsecol else
+                              "per head" if runner.att.per_head else
+                              "per sequence, across heads"),
                    "parallelism": (f"heads split over {world} ranks" if heads else
                                    f"independent sequences x{world}"),
                    "l2": "inputs larger than L2 (192 MiB per step, distinct per step)"},
@@ -553,8 +575,10 @@ def main():
         "speedup_vs_dense": dense_ms / sp_avg,
         "speedup_vs_dense_amortized": dense_ms / (ms_max / len(steps)),
         "anchor_ms": statistics.mean(anchor_ms) if anchor_ms else None,
-        "block_scores_ms": sc_ms, "block_scores_gbs": score_bytes / (sc_ms * 1e-3) / 1e9,
+        "block_scores_ms": sc_ms,
+        "block_scores_gbs": None if runner.pulsecol else score_bytes / (sc_ms * 1e-3) / 1e9,
         "select_mask_ms": se_ms, "mask_blocks": budget,
+        "columns_per_head": getattr(runner.att, "Lc", None),
         "tokens_steps_per_s": w.B * world * w.L * len(steps) / (ms_max * 1e-3),
         "roofline": {"bound": "tensor", "achieved": kernel_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": kernel_tflops / peak,
@@ -562,8 +586,11 @@ def main():
                      "traffic": traffic},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": len(steps) + n_anchor * launches_per_anchor(w.bs, runner.att.sharded,
-                                                                    runner.att.fused),
+        # pulsecol: gather + attention per step; pool, two score passes and the
+        # selection per refresh
+        "gpu_launches": (2 * len(steps) + 4 * n_anchor if runner.pulsecol else
+                         len(steps) + n_anchor * launches_per_anchor(w.bs, runner.att.sharded,
+                                                                     runner.att.fused)),
         "clocks": sampler.summary(),
     }
     if rank == 0:

@@ -293,14 +293,17 @@ def col_budget(q, k, block: int, sparsity: float) -> int:
     return n
 
 
+def col_scores_workspace_bytes(q, k, block: int) -> int:
+    return int(_lib().sdl_col_scores_workspace_bytes(ctypes.byref(make_shape(q, k, block))))
+
+
 def col_scores(q, k, block: int, scale: float = 0.0, out=None, workspace=None, stream=None):
     """fp32 [B, H, L] column scores (see ``sdl_col_scores``)."""
     import torch
     s = make_shape(q, k, block)
     if out is None:
         out = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
-    n = int(_lib().sdl_col_scores_workspace_bytes(ctypes.byref(s)))
-    workspace = _workspace(n, q.device, workspace)
+    workspace = _workspace(col_scores_workspace_bytes(q, k, block), q.device, workspace)
     _check(_lib().sdl_col_scores(q.data_ptr(), k.data_ptr(), ctypes.byref(s), float(scale),
                                  out.data_ptr(), workspace.data_ptr(), workspace.numel(),
                                  _stream(stream)), "sdl_col_scores")

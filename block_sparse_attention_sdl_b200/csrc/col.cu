@@ -55,7 +55,8 @@ void fill_col_args(ColArgs& c, const sdl_shape& s, float scale) {
 }
 
 constexpr int kCR = 16;   // query blocks per tile
-constexpr int kCK = 64;   // keys per tile
+constexpr int kCK = 128;  // keys per tile
+constexpr int kCJ = kCK / 32;  // keys per thread: tx + 32 j
 constexpr int kCThreads = 128;
 
 // qs [kCR][d+4] (block-mean queries), ks [kCK][d+4] (keys as fp32)
@@ -84,38 +85,52 @@ __device__ __forceinline__ void load_q_tile(const float* __restrict__ qsrc, int 
   }
 }
 
-// Keys u0 .. u0+kCK of KV head kh into ks (fp32).
+// Keys u0 .. u0+kCK of KV head kh into ks (fp32; zero past L), 16 bytes per
+// load (the (b, t, h) strides are multiples of 16 bytes and d of 8 elements).
 template <typename T>
 __device__ __forceinline__ void load_k_tile(const T* __restrict__ k, const int64_t* ks, int b,
-                                            int kh, int d, int u0, float* kt) {
-  const int dp = d + 4;
-  for (int x = threadIdx.x; x < kCK * d; x += kCThreads) {
-    const int r = x / d, c = x % d;
-    kt[r * dp + c] = to_f<T>(k[b * ks[0] + (int64_t)(u0 + r) * ks[1] + kh * ks[2] + c]);
+                                            int kh, int d, int u0, int L, float* kt) {
+  constexpr int V = 16 / sizeof(T);  // elements per load
+  const int dp = d + 4, dv = d / V;
+#pragma unroll 4
+  for (int x = threadIdx.x; x < kCK * dv; x += kCThreads) {
+    const int r = x / dv, c = (x % dv) * V;
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (u0 + r < L)
+      u = __ldg(reinterpret_cast<const uint4*>(k + b * ks[0] + (int64_t)(u0 + r) * ks[1] +
+                                               kh * ks[2] + c));
+    const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+    for (int y = 0; y < V; y += 4)
+      *reinterpret_cast<float4*>(kt + r * dp + c + y) =
+          make_float4(to_f<T>(e[y]), to_f<T>(e[y + 1]), to_f<T>(e[y + 2]), to_f<T>(e[y + 3]));
   }
 }
 
-// z[a][u] for the thread's 4 rows (ty*4 + a) and 2 keys (tx, tx + 32).
+// z[a][j] for the thread's 4 rows (ty*4 + a) and kCJ keys (tx + 32 j).
 __device__ __forceinline__ void tile_logits(const float* qs, const float* kt, int d, float scale,
-                                            float (&z)[4][2]) {
+                                            float (&z)[4][kCJ]) {
   const int dp = d + 4, ty = threadIdx.x / 32, tx = threadIdx.x % 32;
 #pragma unroll
-  for (int a = 0; a < 4; ++a) z[a][0] = z[a][1] = 0.f;
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int j = 0; j < kCJ; ++j) z[a][j] = 0.f;
   for (int c = 0; c < d; c += 4) {
-    const float4 k0 = *reinterpret_cast<const float4*>(kt + tx * dp + c);
-    const float4 k1 = *reinterpret_cast<const float4*>(kt + (tx + 32) * dp + c);
+    float4 kv[kCJ];
+#pragma unroll
+    for (int j = 0; j < kCJ; ++j) kv[j] = *reinterpret_cast<const float4*>(kt + (tx + 32 * j) * dp + c);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const float4 q = *reinterpret_cast<const float4*>(qs + (ty * 4 + a) * dp + c);
-      z[a][0] += q.x * k0.x + q.y * k0.y + q.z * k0.z + q.w * k0.w;
-      z[a][1] += q.x * k1.x + q.y * k1.y + q.z * k1.z + q.w * k1.w;
+#pragma unroll
+      for (int j = 0; j < kCJ; ++j)
+        z[a][j] += q.x * kv[j].x + q.y * kv[j].y + q.z * kv[j].z + q.w * kv[j].w;
     }
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    z[a][0] *= scale;
-    z[a][1] *= scale;
-  }
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int j = 0; j < kCJ; ++j) z[a][j] *= scale;
 }
 
 // grid (ceil(nb / kCR), H, B): stats[b, h, i] = (max over u of z_iu, sum over u
@@ -138,14 +153,24 @@ __global__ void __launch_bounds__(kCThreads) col_stats_kernel(const float* __res
   }
   for (int u0 = 0; u0 < c.L; u0 += kCK) {
     __syncthreads();
-    load_k_tile<T>(k, c.ks, b, kh, c.d, u0, kt);
+    load_k_tile<T>(k, c.ks, b, kh, c.d, u0, c.L, kt);
     __syncthreads();
-    float z[4][2];
+    float z[4][kCJ];
     tile_logits(qs, kt, c.d, c.scale, z);
 #pragma unroll
+    for (int j = 0; j < kCJ; ++j)
+      if (u0 + (int)(threadIdx.x % 32) + 32 * j >= c.L)  // no such key
+#pragma unroll
+        for (int a = 0; a < 4; ++a) z[a][j] = -INFINITY;
+#pragma unroll
     for (int a = 0; a < 4; ++a) {
-      const float mt = fmaxf(m[a], fmaxf(z[a][0], z[a][1]));
-      l[a] = l[a] * expf(m[a] - mt) + expf(z[a][0] - mt) + expf(z[a][1] - mt);
+      float mt = m[a];
+#pragma unroll
+      for (int j = 0; j < kCJ; ++j) mt = fmaxf(mt, z[a][j]);
+      float t = l[a] * expf(m[a] - mt);
+#pragma unroll
+      for (int j = 0; j < kCJ; ++j) t += expf(z[a][j] - mt);
+      l[a] = t;
       m[a] = mt;
     }
   }
@@ -165,7 +190,7 @@ __global__ void __launch_bounds__(kCThreads) col_stats_kernel(const float* __res
   }
 }
 
-// grid (L / kCK, H, B): S[b, h, u] = (1/nb) sum over i of exp(z_iu - max_i) / sum_i.
+// grid (ceil(L / kCK), H, B): S[b, h, u] = (1/nb) sum over i of exp(z_iu - max_i) / sum_i.
 template <typename T>
 __global__ void __launch_bounds__(kCThreads) col_sum_kernel(const float* __restrict__ qbar,
                                                             const T* __restrict__ k, ColArgs c,
@@ -178,15 +203,17 @@ __global__ void __launch_bounds__(kCThreads) col_sum_kernel(const float* __restr
   const int b = blockIdx.z, h = blockIdx.y, u0 = blockIdx.x * kCK;
   const int kh = h / (c.H / c.Hkv);
   const int ty = threadIdx.x / 32, tx = threadIdx.x % 32;
-  load_k_tile<T>(k, c.ks, b, kh, c.d, u0, kt);
+  load_k_tile<T>(k, c.ks, b, kh, c.d, u0, c.L, kt);
   const float* qsrc = qbar + ((int64_t)b * c.H + h) * c.nb * c.d;
   const float2* st = stats + ((int64_t)b * c.H + h) * c.nb;
-  float acc0 = 0.f, acc1 = 0.f;
+  float acc[kCJ];
+#pragma unroll
+  for (int j = 0; j < kCJ; ++j) acc[j] = 0.f;
   for (int i0 = 0; i0 < c.nb; i0 += kCR) {
     __syncthreads();
     load_q_tile(qsrc, c.nb, c.d, i0, qs);
     __syncthreads();
-    float z[4][2];
+    float z[4][kCJ];
     tile_logits(qs, kt, c.d, c.scale, z);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
@@ -194,18 +221,18 @@ __global__ void __launch_bounds__(kCThreads) col_sum_kernel(const float* __restr
       if (i < c.nb) {
         const float2 s2 = st[i];
         const float inv = 1.0f / s2.y;
-        acc0 += expf(z[a][0] - s2.x) * inv;
-        acc1 += expf(z[a][1] - s2.x) * inv;
+#pragma unroll
+        for (int j = 0; j < kCJ; ++j) acc[j] += expf(z[a][j] - s2.x) * inv;
       }
     }
   }
-  part[ty][tx] = acc0;
-  part[ty][tx + 32] = acc1;
+#pragma unroll
+  for (int j = 0; j < kCJ; ++j) part[ty][tx + 32 * j] = acc[j];
   __syncthreads();
-  if (threadIdx.x < kCK) {
+  for (int x = threadIdx.x; x < kCK && u0 + x < c.L; x += kCThreads) {
     float t = 0.f;
-    for (int w = 0; w < kCThreads / 32; ++w) t += part[w][threadIdx.x];
-    S[((int64_t)b * c.H + h) * c.L + u0 + threadIdx.x] = t / (float)c.nb;
+    for (int w = 0; w < kCThreads / 32; ++w) t += part[w][x];
+    S[((int64_t)b * c.H + h) * c.L + u0 + x] = t / (float)c.nb;
   }
 }
 
@@ -310,7 +337,22 @@ cudaError_t launch_col_scores(const void* k, const sdl_shape& s, float scale, co
   ColArgs c;
   fill_col_args(c, s, scale);
   const size_t smem = col_smem_bytes(s.d);
-  const dim3 g1((c.nb + kCR - 1) / kCR, s.H, s.B), g2(s.L / kCK, s.H, s.B);
+  const dim3 g1((c.nb + kCR - 1) / kCR, s.H, s.B), g2((s.L + kCK - 1) / kCK, s.H, s.B);
+  static bool attr_set = false;  // per function; the size needed is at most this
+  if (!attr_set) {
+    const int most = (int)col_smem_bytes(128);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(col_stats_kernel<__nv_bfloat16>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, most)) ||
+        (e = cudaFuncSetAttribute(col_sum_kernel<__nv_bfloat16>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, most)) ||
+        (e = cudaFuncSetAttribute(col_stats_kernel<float>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, most)) ||
+        (e = cudaFuncSetAttribute(col_sum_kernel<float>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, most)))
+      return e;
+    attr_set = true;
+  }
   if (s.dtype == SDL_BF16) {
     col_stats_kernel<__nv_bfloat16><<<g1, kCThreads, smem, st>>>(
         qbar, static_cast<const __nv_bfloat16*>(k), c, stats);

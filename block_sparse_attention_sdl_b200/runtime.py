@@ -13,6 +13,10 @@ head-adaptive global one (``budget="head"``), and dense attention for the first
 ``dense_steps`` steps followed by a single mask, built at step
 ``dense_steps`` and reused for every later step (``anchor_every=None``).
 
+``ColSparseAttention`` is the column-sparse scheme of the PulseCol abstract on
+the same schedule: every query head keeps a set of key tokens, refreshed at
+anchor steps, gathered and attended to at every step.
+
 With ``heads_total`` the layer is one rank's part of a head-sharded attention
 layer: its tensors hold ``H`` of the sequence's ``heads_total`` query heads
 (whole KV-head groups, ranks in head order), and the global budget is met with
@@ -23,9 +27,10 @@ from __future__ import annotations
 
 import torch
 
-from . import (anchor_refresh, anchor_workspace_bytes, block_scores, dense_attn, make_shape,
-               mask_budget, scores_workspace_bytes, select_mask, select_shard_capacity,
-               select_workspace_bytes, sparse_attn, tile_plan)
+from . import (anchor_refresh, anchor_workspace_bytes, block_scores, col_budget, col_gather,
+               col_scores, col_scores_workspace_bytes, col_select, col_sparse_attn, dense_attn,
+               make_shape, mask_budget, scores_workspace_bytes, select_mask,
+               select_shard_capacity, select_workspace_bytes, sparse_attn, tile_plan)
 from .sharded import CudaStages, select_mask_sharded, torch_collectives
 
 
@@ -145,3 +150,57 @@ class StepSparseAttention:
             self.refresh(q, k, anchor_of(step, self.anchor_every, self.dense_steps), stream)
         return sparse_attn(q, k, v, self.row_ptr, self.col_idx, self.block, out=out, lse=lse,
                            plan=self.plan, stream=stream)
+
+
+class ColSparseAttention:
+    """One attention layer's column-sparse state (the PulseCol abstract).
+
+    Every query head keeps Lc key tokens for all of its query rows: chosen from the
+    column scores at refresh steps (step 0 and every ``refresh_every`` steps;
+    ``None``: step 0 only) and reused in between.  Every step gathers the kept K and
+    V tokens of that step's tensors and runs dense attention over them.  Buffers are
+    allocated once here.
+    """
+
+    def __init__(self, B, H, H_kv, L, d, block, sparsity, refresh_every,
+                 dtype=torch.bfloat16, device="cuda"):
+        self.B, self.H, self.H_kv, self.L, self.d, self.block = B, H, H_kv, L, d, block
+        self.sparsity, self.anchor_every = sparsity, refresh_every
+        self.per_head, self.sharded, self.fused, self.dense_steps = True, False, False, 0
+        probe_q = torch.empty((B, L, H, d), dtype=dtype, device="meta")
+        probe_k = torch.empty((B, L, H_kv, d), dtype=dtype, device="meta")
+        self.Lc = col_budget(probe_q, probe_k, block, sparsity)
+        # kept work in 64x64-block equivalents (L and Lc are whole 64-token tiles)
+        self.budget = B * H * (L // 64) * (self.Lc // 64)
+        dev = torch.device(device)
+        self.col_scores = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(max(col_scores_workspace_bytes(probe_q, probe_k, block), 16),
+                              dtype=torch.uint8, device=dev)
+        self.cols = torch.empty((B, H, self.Lc), dtype=torch.int32, device=dev)
+        self.k_cols = torch.empty((B, self.Lc, H, d), dtype=dtype, device=dev)
+        self.v_cols = torch.empty((B, self.Lc, H, d), dtype=dtype, device=dev)
+        self.mask_step = None
+        self._qk = None  # the tensors of the last refresh (shapes for the selection)
+
+    def refresh(self, q, k, step: int, stream=None):
+        col_scores(q, k, self.block, out=self.col_scores, workspace=self.ws, stream=stream)
+        self._qk = (q, k)
+        self.select(stream)
+        self.mask_step = step
+
+    def select(self, stream=None):
+        q, k = self._qk
+        col_select(self.col_scores, q, k, self.block, self.sparsity, cols=self.cols,
+                   stream=stream)
+
+    def attend(self, q, k, v, out=None, lse=None, stream=None):
+        """This step's attention over the kept columns (gather, then attention)."""
+        col_gather(k, v, self.cols, q, self.block, k_cols=self.k_cols, v_cols=self.v_cols,
+                   stream=stream)
+        return col_sparse_attn(q, self.k_cols, self.v_cols, self.block, out=out,
+                               want_lse=lse is not None, lse=lse, stream=stream)
+
+    def __call__(self, q, k, v, step: int, out=None, lse=None, stream=None):
+        if is_anchor(step, self.anchor_every) or self.mask_step is None:
+            self.refresh(q, k, anchor_of(step, self.anchor_every), stream)
+        return self.attend(q, k, v, out=out, lse=lse, stream=stream)

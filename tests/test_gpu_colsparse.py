@@ -22,6 +22,7 @@ CASES = [
     ("bf16", 1, 512, 4, 2, 128, 0.8),       # GQA
     ("bf16", 2, 1024, 2, 2, 64, 0.9),       # two sequences
     ("bf16", 1, 2048, 4, 4, 128, 0.75),
+    ("bf16", 1, 576, 2, 2, 128, 0.7),       # a partial 128-key score tile
 ]
 
 
@@ -96,3 +97,25 @@ def test_col_arguments_are_checked():
     kc = torch.empty((1, 96, 2, 64), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(sdl.SdlError):
         sdl.col_sparse_attn(q, kc, kc, 64)  # 96 columns: not whole 64-key tiles
+
+
+def test_col_schedule_refreshes_at_anchors_only():
+    """The column set changes only at refresh steps; a step in between attends with
+    its anchor's columns over its own inputs."""
+    from block_sparse_attention_sdl_b200.runtime import ColSparseAttention
+    w = synth.small_workload(B=1, H=4, H_kv=2, L=512, d=128, bs=64, sparsity=0.8, planted=2,
+                             steps=4, anchor_every=2)
+    att = ColSparseAttention(w.B, w.H, w.H_kv, w.L, w.d, w.bs, w.sparsity, 2)
+    seen = []
+    for step in range(4):
+        x = synth.device_inputs(w, step)
+        O = att(x["q"], x["k"], x["v"], step)
+        torch.cuda.synchronize()
+        seen.append(att.cols.clone())
+        assert att.mask_step == (step // 2) * 2
+        if step in (1, 3):
+            assert torch.equal(seen[step], seen[step - 1])
+            host = synth.host_inputs(w, step)
+            Ow, _ = oracle.col_attention(host["q"], host["k"], host["v"], att.cols.cpu().numpy())
+            check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, "bf16")
+    assert sdl.last_device_status() == sdl.SDL_OK
