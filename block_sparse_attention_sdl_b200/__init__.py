@@ -35,6 +35,7 @@ EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspac
            "sdl_select_shard_workspace_bytes", "sdl_select_shard_hist",
            "sdl_select_shard_capacity", "sdl_select_shard_pass", "sdl_select_shard_count",
            "sdl_select_shard_finish",
+           "sdl_wait_selfcheck",
            "sdl_last_device_status", "sdl_last_cuda_error", "sdl_status_string")
 SDL_SELECT_PASSES = 3
 
@@ -107,12 +108,14 @@ def _lib():
         L.sdl_select_shard_count.argtypes = [P, SP, ctypes.c_int32, D, P, SZ, P, P]
         L.sdl_select_shard_finish.argtypes = [P, SP, ctypes.c_int32, D, P, P, P, I64, P, P, SZ,
                                               P]
+        L.sdl_wait_selfcheck.argtypes = [ctypes.c_uint64, P]
         L.sdl_last_device_status.argtypes = [P]
         L.sdl_last_cuda_error.argtypes = []
         L.sdl_status_string.argtypes = [ctypes.c_int]
         L.sdl_status_string.restype = ctypes.c_char_p
         for f in ("sdl_block_scores", "sdl_select_mask", "sdl_select_mask_scoped",
                   "sdl_anchor_refresh", "sdl_col_scores", "sdl_col_select",
+                  "sdl_wait_selfcheck",
                   "sdl_col_gather", "sdl_col_sparse_attn",
                   "sdl_select_shard_hist", "sdl_select_shard_pass", "sdl_select_shard_count",
                   "sdl_select_shard_finish",
@@ -493,6 +496,12 @@ def dense_attn(q, k, v, block: int = 64, scale: float = 0.0, out=None, lse=None,
                                  None if lse is None else lse.data_ptr(), _stream(stream)),
            "sdl_dense_attn")
     return (out, lse) if want_lse or lse is not None else out
+
+
+def wait_selfcheck(limit_ns: int = 1_000_000, stream=None):
+    """Runs the bounded-wait self-check (see ``sdl_wait_selfcheck``); the next
+    ``last_device_status`` reports SDL_ERR_TIMEOUT."""
+    _check(_lib().sdl_wait_selfcheck(int(limit_ns), _stream(stream)), "sdl_wait_selfcheck")
 
 
 def last_device_status(stream=None) -> int:

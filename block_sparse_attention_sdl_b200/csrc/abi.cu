@@ -548,6 +548,15 @@ sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl
   return attn_common(q, k, v, shape, nullptr, nullptr, nullptr, scale, o, lse, stream);
 }
 
+sdl_status sdl_wait_selfcheck(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000ull) return SDL_ERR_INVALID_ARG;
+  int* status = device_status_ptr();
+  if (!status) return SDL_ERR_CUDA;
+  cudaError_t ce = launch_wait_check(limit_ns, status, static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
 sdl_status sdl_last_device_status(void* stream) {
   cudaError_t ce = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (ce != cudaSuccess) return cuda_fail(ce);

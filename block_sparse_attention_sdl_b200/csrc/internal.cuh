@@ -68,6 +68,8 @@ cudaError_t launch_col_select(const float* S, int BH, int L, int Lc, int32_t* co
                               cudaStream_t st);
 cudaError_t launch_col_gather(const void* k, const void* v, const sdl_shape& s,
                               const int32_t* cols, int Lc, void* kc, void* vc, cudaStream_t st);
+// self-check of the bounded waits (selfcheck.cu)
+cudaError_t launch_wait_check(uint64_t limit_ns, int* status, cudaStream_t st);
 size_t select_hist_offset(int B, int pass);
 size_t select_hist_count(int B);
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,

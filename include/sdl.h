@@ -287,6 +287,13 @@ sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl
  * list entry was rejected, SDL_OK otherwise. */
 sdl_status sdl_last_device_status(void* stream);
 
+/* Self-check of the failure path: launches one warp that waits, through the
+ * same bounded wait every kernel of the library uses, on an mbarrier phase
+ * that nothing completes, giving up after `limit_ns` (1 us .. 1 s, else
+ * SDL_ERR_INVALID_ARG).  The next sdl_last_device_status then returns
+ * SDL_ERR_TIMEOUT, and the context stays usable. */
+sdl_status sdl_wait_selfcheck(uint64_t limit_ns, void* stream);
+
 /* cudaError_t of the last failed CUDA call in this thread (0 if none). */
 int sdl_last_cuda_error(void);
 

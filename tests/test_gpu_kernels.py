@@ -405,3 +405,24 @@ def test_argument_errors_do_not_launch():
     with pytest.raises(sdl.SdlError) as e:
         sdl.select_mask(P, 0.5, 64, 256, col_idx=torch.empty(3, dtype=torch.int32, device="cuda"))
     assert e.value.status == sdl.SDL_ERR_CAPACITY
+
+
+def test_bounded_wait_times_out_and_the_context_survives():
+    """A wait on a phase nothing completes gives up at its limit and raises the timeout
+    bit, which sdl_last_device_status reports once and clears; kernels still run."""
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    sdl.wait_selfcheck(2_000_000)  # 2 ms
+    t1.record()
+    assert sdl.last_device_status() == sdl.SDL_ERR_TIMEOUT
+    assert 1.5 <= t0.elapsed_time(t1) < 100.0
+    assert sdl.last_device_status() == sdl.SDL_OK
+    with pytest.raises(sdl.SdlError):
+        sdl.wait_selfcheck(10)  # below the smallest limit
+    w = synth.small_workload(L=256, H=2, H_kv=2, d=64, bs=64, sparsity=0.5)
+    host, dev = _inputs(w)
+    O = sdl.dense_attn(dev["q"], dev["k"], dev["v"])
+    assert sdl.last_device_status() == sdl.SDL_OK
+    Ow, _ = oracle.attention(host["q"], host["k"], host["v"], 64)
+    check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, "bf16")
