@@ -210,7 +210,7 @@ class Runner:
             att.attend(x["q"], x["k"], x["v"], out=self.out)
         else:
             self.sdl.sparse_attn(x["q"], x["k"], x["v"], att.row_ptr, att.col_idx, w.bs,
-                                 out=self.out, plan=att.plan)
+                                 out=self.out, plan=att.plan, order=att.order)
         if ev is not None:
             ev["s1"].append(torch.cuda.Event(enable_timing=True))
             ev["s1"][-1].record()
@@ -222,7 +222,8 @@ class Runner:
             self.att.attend(x["q"], x["k"], x["v"], out=self.out)
         else:
             self.sdl.sparse_attn(x["q"], x["k"], x["v"], self.att.row_ptr, self.att.col_idx,
-                                 self.w.bs, out=self.out, plan=self.att.plan)
+                                 self.w.bs, out=self.out, plan=self.att.plan,
+                                 order=self.att.order)
         self.att.mask_step = None
 
 
@@ -270,8 +271,8 @@ def time_steps(runner, inputs, steps, dist_on, device, with_events=True):
 def launches_per_anchor(block: int, sharded: bool = False, fused: bool = False):
     # fused: scores and selection in one launch; else pool, score; select: zero, 3
     # histogram passes, count, scan, write (+ the per-rank totals when the heads are
-    # sharded); tile plan (64-token blocks)
-    plan = 1 if block == 64 else 0
+    # sharded); tile plan and its order (64-token blocks)
+    plan = 2 if block == 64 else 0  # the plan and its take order
     if fused:
         return 1 + plan
     return 2 + 7 + (1 if sharded else 0) + plan
@@ -403,7 +404,7 @@ def profile_kernel(runner, args):
     if args.profile == "sparse":
         fn = lambda: sdl.sparse_attn(x["q"], x["k"], x["v"], runner.att.row_ptr,
                                      runner.att.col_idx, w.bs, out=runner.out,
-                                     plan=runner.att.plan)
+                                     plan=runner.att.plan, order=runner.att.order)
         flop = 4.0 * w.bs * w.bs * w.d * runner.att.budget
     else:
         fn = lambda: sdl.dense_attn(x["q"], x["k"], x["v"], out=runner.out)

@@ -28,7 +28,8 @@ SDL_BF16, SDL_FP32 = 0, 1
 EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspace_bytes",
            "sdl_mask_budget_scoped", "sdl_select_workspace_bytes_scoped", "sdl_select_mask_scoped",
            "sdl_block_scores", "sdl_select_mask", "sdl_select_mask_noalloc", "sdl_sparse_attn",
-           "sdl_tile_plan", "sdl_sparse_attn_planned", "sdl_dense_attn",
+           "sdl_tile_plan", "sdl_sparse_attn_planned", "sdl_tile_order",
+           "sdl_sparse_attn_scheduled", "sdl_dense_attn",
            "sdl_anchor_workspace_bytes", "sdl_anchor_refresh",
            "sdl_col_budget", "sdl_col_scores_workspace_bytes", "sdl_col_scores",
            "sdl_col_select", "sdl_col_gather", "sdl_col_sparse_attn",
@@ -86,6 +87,8 @@ def _lib():
         L.sdl_sparse_attn.argtypes = [P, P, P, SP, P, P, F, P, P, P]
         L.sdl_tile_plan.argtypes = [P, P, SP, P, P]
         L.sdl_sparse_attn_planned.argtypes = [P, P, P, SP, P, P, P, F, P, P, P]
+        L.sdl_tile_order.argtypes = [P, P, SP, P, P]
+        L.sdl_sparse_attn_scheduled.argtypes = [P, P, P, SP, P, P, P, P, F, P, P, P]
         L.sdl_dense_attn.argtypes = [P, P, P, SP, F, P, P, P]
         L.sdl_col_budget.argtypes = [SP, D]
         L.sdl_col_budget.restype = I64
@@ -120,7 +123,8 @@ def _lib():
                   "sdl_select_shard_hist", "sdl_select_shard_pass", "sdl_select_shard_count",
                   "sdl_select_shard_finish",
                   "sdl_sparse_attn", "sdl_tile_plan",
-                  "sdl_sparse_attn_planned", "sdl_dense_attn",
+                  "sdl_sparse_attn_planned", "sdl_tile_order", "sdl_sparse_attn_scheduled",
+                  "sdl_dense_attn",
                   "sdl_last_device_status", "sdl_last_cuda_error"):
             getattr(L, f).restype = ctypes.c_int
         _L = L
@@ -443,6 +447,20 @@ def select_shard_finish(scores, sparsity: float, block: int, L: int, heads_total
     return row_ptr, col_idx, mask
 
 
+def tile_order(row_ptr, plan, B: int, H: int, L: int, block: int = 64, order=None,
+               stream=None):
+    """int32 [B*H*ceil(nb/2)]: the plan's tiles, costliest first (see ``sdl_tile_order``)."""
+    import torch
+    nb = L // block
+    s = Shape()
+    s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, H, L, 64, block, SDL_BF16
+    if order is None:
+        order = torch.empty(B * H * ((nb + 1) // 2), dtype=torch.int32, device=plan.device)
+    _check(_lib().sdl_tile_order(row_ptr.data_ptr(), plan.data_ptr(), ctypes.byref(s),
+                                 order.data_ptr(), _stream(stream)), "sdl_tile_order")
+    return order
+
+
 def tile_plan(row_ptr, col_idx, B: int, H: int, L: int, block: int = 64, plan=None,
               stream=None):
     """int32 [B, H, ceil(nb/2), 2] tile plan for 64-token blocks (see ``sdl_tile_plan``)."""
@@ -458,16 +476,24 @@ def tile_plan(row_ptr, col_idx, B: int, H: int, L: int, block: int = 64, plan=No
 
 
 def sparse_attn(q, k, v, row_ptr, col_idx, block: int, scale: float = 0.0, out=None, lse=None,
-                want_lse: bool = False, plan=None, stream=None):
+                want_lse: bool = False, plan=None, order=None, stream=None):
     """O like q (and LSE fp32 [B,H,L] when asked) over the kept blocks; ``plan`` is an
-    optional tile plan from :func:`tile_plan` (results equal up to fp32 summation order)."""
+    optional tile plan from :func:`tile_plan` (results equal up to fp32 summation order),
+    ``order`` the order of taking its tiles from :func:`tile_order` (same bits)."""
     import torch
     if out is None:
         out = torch.empty_like(q)
     s = make_shape(q, k, block, v, out)
     if lse is None and want_lse:
         lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
-    if plan is None:
+    if plan is not None and order is not None:
+        _check(_lib().sdl_sparse_attn_scheduled(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                ctypes.byref(s), row_ptr.data_ptr(),
+                                                col_idx.data_ptr(), plan.data_ptr(),
+                                                order.data_ptr(), float(scale), out.data_ptr(),
+                                                None if lse is None else lse.data_ptr(),
+                                                _stream(stream)), "sdl_sparse_attn_scheduled")
+    elif plan is None:
         _check(_lib().sdl_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(s),
                                       row_ptr.data_ptr(), col_idx.data_ptr(), float(scale),
                                       out.data_ptr(), None if lse is None else lse.data_ptr(),

@@ -100,7 +100,8 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, const sdl_shape& s, int
 // Lk: key and value tokens (0: L, the same as the queries).
 sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_shape* shape,
                        const int32_t* row_ptr, const int32_t* col_idx, const int32_t* plan,
-                       float scale, void* o, float* lse, void* stream, int Lk = 0) {
+                       float scale, void* o, float* lse, void* stream, int Lk = 0,
+                       const int32_t* order = nullptr) {
   sdl_status e = check_shape(shape);
   if (e) return e;
   const sdl_shape& s = *shape;
@@ -121,6 +122,7 @@ sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_sh
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
   a.plan = (row_ptr && s.block == 64) ? plan : nullptr;
+  a.order = a.plan ? order : nullptr;
   a.B = s.B;
   a.H = s.H;
   a.Hkv = s.H_kv;
@@ -541,6 +543,28 @@ sdl_status sdl_tile_plan(const int32_t* row_ptr, const int32_t* col_idx, const s
                                      static_cast<cudaStream_t>(stream));
   if (ce != cudaSuccess) return cuda_fail(ce);
   return SDL_OK;
+}
+
+sdl_status sdl_tile_order(const int32_t* row_ptr, const int32_t* plan, const sdl_shape* shape,
+                          int32_t* order, void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  if (!row_ptr || !plan || !order) return SDL_ERR_INVALID_ARG;
+  if (shape->block != 64) return SDL_ERR_UNSUPPORTED;
+  const cudaError_t ce = launch_tile_order(row_ptr, plan, shape->B, shape->H,
+                                           shape->L / shape->block, order,
+                                           static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_sparse_attn_scheduled(const void* q, const void* k, const void* v,
+                                     const sdl_shape* shape, const int32_t* row_ptr,
+                                     const int32_t* col_idx, const int32_t* plan,
+                                     const int32_t* order, float scale, void* o, float* lse,
+                                     void* stream) {
+  if (!row_ptr || !col_idx || !plan || !order) return SDL_ERR_INVALID_ARG;
+  return attn_common(q, k, v, shape, row_ptr, col_idx, plan, scale, o, lse, stream, 0, order);
 }
 
 sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,

@@ -319,6 +319,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           item = (int)taken;
+          if (a.order != nullptr) {
+            // costliest tiles first (the order is a permutation of the items)
+            const int o = a.order[item];
+            if (o < 0 || o >= n_items) {
+              atomicOr(a.status, kDevBadMask);
+              continue;
+            }
+            item = o;
+          }
           b = item / (a.H * n_qt);
           h = (item / n_qt) % a.H;
           if (a.plan != nullptr) {

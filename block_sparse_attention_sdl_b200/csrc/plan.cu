@@ -14,6 +14,7 @@
 // fp32 summation order.
 #include "internal.cuh"
 #include "plan_impl.cuh"
+#include "select_impl.cuh"
 
 namespace sdl {
 namespace {
@@ -27,6 +28,53 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
                                                             int32_t* __restrict__ plan) {
   extern __shared__ __align__(16) uint8_t psm[];
   plan_body(row_ptr, col_idx, H, nb, n_qt, plan, blockIdx.x, blockIdx.y, psm);
+}
+
+constexpr int kOrderThreads = 1024;
+constexpr int kOrderBins = 2 * 1024 + 1;  // tile costs 0 .. 2 nb, nb <= 1024
+
+// One CTA: the order in which the attention kernel takes its tiles, costliest
+// first, so that the long tiles of heavy heads do not run last and leave the
+// other SMs idle.  A tile's cost is the sum of its two query blocks' list
+// lengths (an upper bound of the union it walks); a counting sort orders them
+// (equal costs in any order).  order[r] = the r-th tile to take.
+__global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __restrict__ row_ptr,
+                                                              const int32_t* __restrict__ plan,
+                                                              int BH, int nb, int n_qt,
+                                                              int32_t* __restrict__ order) {
+  __shared__ int start[kOrderBins];
+  __shared__ int s_warp[32];
+  const int n = BH * n_qt, tid = threadIdx.x;
+  auto cost = [&](int x) -> int {
+    const int64_t r0 = (int64_t)(x / n_qt) * nb;
+    int c = 0;
+    for (int s = 0; s < 2; ++s) {
+      const int qb = plan[2 * (int64_t)x + s];
+      if (qb >= 0 && qb < nb) c += row_ptr[r0 + qb + 1] - row_ptr[r0 + qb];
+    }
+    return c < 0 ? 0 : (c >= kOrderBins ? kOrderBins - 1 : c);
+  };
+  for (int c = tid; c < kOrderBins; c += kOrderThreads) start[c] = 0;
+  __syncthreads();
+  for (int x = tid; x < n; x += kOrderThreads) atomicAdd(&start[cost(x)], 1);
+  __syncthreads();
+  // first position of each cost, costs in descending order: thread t owns bins
+  // kOrderBins - 1 - 3t, -3t-1, -3t-2
+  int cnt[3], local = 0;
+  for (int y = 0; y < 3; ++y) {
+    const int c = kOrderBins - 1 - 3 * tid - y;
+    cnt[y] = c >= 0 ? start[c] : 0;
+    local += cnt[y];
+  }
+  int total = 0;
+  int pos = selimpl::block_excl_scan(local, s_warp, total);
+  for (int y = 0; y < 3; ++y) {
+    const int c = kOrderBins - 1 - 3 * tid - y;
+    if (c >= 0) start[c] = pos;
+    pos += cnt[y];
+  }
+  __syncthreads();
+  for (int x = tid; x < n; x += kOrderThreads) order[atomicAdd(&start[cost(x)], 1)] = x;
 }
 
 // Adjacent pairs (2p, 2p+1), for heads too long for the greedy plan.
@@ -59,6 +107,12 @@ cudaError_t launch_plan(const int32_t* row_ptr, const int32_t* col_idx, int B, i
     attr_set = true;
   }
   plan_kernel<<<dim3(H, B), kPlanThreads, smem, st>>>(row_ptr, col_idx, H, nb, n_qt, plan);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_order(const int32_t* row_ptr, const int32_t* plan, int B, int H, int nb,
+                              int32_t* order, cudaStream_t st) {
+  order_kernel<<<1, kOrderThreads, 0, st>>>(row_ptr, plan, B * H, nb, (nb + 1) / 2, order);
   return cudaGetLastError();
 }
 

@@ -277,6 +277,28 @@ sdl_status sdl_sparse_attn_planned(const void* q, const void* k, const void* v,
                                    const int32_t* col_idx, const int32_t* plan, float scale,
                                    void* o, float* lse, void* stream);
 
+/* Order in which the attention kernel takes the tiles of a plan, costliest
+ * first (a scheduling aid): tiles are taken from a global counter by
+ * persistent CTAs, and when the longest tiles come last (as with heads that
+ * keep many blocks at the end of the head order) the other SMs sit idle while
+ * they finish.  Writes order, int32 [B * H * ceil(nb/2)]: a permutation of the
+ * tile indices (b * H + h) * ceil(nb/2) + p, sorted by the sum of the tile's two
+ * query blocks' list lengths, descending (ties in any order).  Only block ==
+ * 64 (SDL_ERR_UNSUPPORTED otherwise). */
+sdl_status sdl_tile_order(const int32_t* row_ptr, const int32_t* plan, const sdl_shape* shape,
+                          int32_t* order, void* stream);
+
+/* sdl_sparse_attn_planned taking the plan's tiles in `order` (from
+ * sdl_tile_order, or any permutation of the tile indices).  Results are those
+ * of sdl_sparse_attn_planned bit for bit (a tile's result does not depend on
+ * which CTA runs it or when); entries outside the tile range are skipped and
+ * reported as SDL_ERR_BAD_MASK. */
+sdl_status sdl_sparse_attn_scheduled(const void* q, const void* k, const void* v,
+                                     const sdl_shape* shape, const int32_t* row_ptr,
+                                     const int32_t* col_idx, const int32_t* plan,
+                                     const int32_t* order, float scale, void* o, float* lse,
+                                     void* stream);
+
 /* Dense bidirectional attention, the baseline of the same abstract: the
  * sparse call with every block of every row kept. */
 sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,

@@ -314,6 +314,45 @@ def test_sparse_attention_with_tile_plan(L, H, Hkv, density, kind):
     assert np.abs(lse.cpu().numpy() - lw).max() <= TOL["bf16"]["lse"]
 
 
+@pytest.mark.parametrize("L,H,density", [(1024, 4, 0.3), (4096, 8, 0.15), (576, 3, 0.5)])
+def test_tile_order_is_costliest_first_and_exact(L, H, density):
+    """The take order is a permutation of the tiles sorted by the two blocks' list
+    lengths (descending), and attention taken in it equals the plan order bit for bit."""
+    w = synth.small_workload(L=L, H=H, H_kv=H, d=128, bs=64)
+    _, dev = _inputs(w)
+    nb = L // 64
+    rng = np.random.default_rng(L * 7 + H)
+    mask = _random_mask(1, H, nb, density, rng)
+    mask[0, H - 1] = 1  # the last head keeps every block: its tiles are the costliest
+    rp, ci = _mask_to_csr(mask)
+    plan = sdl.tile_plan(rp, ci, 1, H, L, 64)
+    order = sdl.tile_order(rp, plan, 1, H, L, 64)
+    O1 = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, plan=plan)
+    O2 = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, plan=plan, order=order)
+    assert sdl.last_device_status() == sdl.SDL_OK
+    assert torch.equal(O1, O2)
+    o = order.cpu().numpy()
+    n_qt = (nb + 1) // 2
+    assert np.array_equal(np.sort(o), np.arange(H * n_qt))
+    lens = mask.sum(-1).reshape(-1).astype(np.int64)  # list length per (h, query block)
+    pl = plan.cpu().numpy().reshape(-1, 2)
+    cost = np.array([sum(lens[(x // n_qt) * nb + qb] for qb in pl[x] if qb >= 0)
+                     for x in range(H * n_qt)])
+    assert np.all(np.diff(cost[o]) <= 0)
+    assert cost[o[0]] == cost.max()
+
+
+def test_bad_tile_order_entry_is_reported():
+    w = synth.small_workload(L=256, H=1, H_kv=1, d=128)
+    _, dev = _inputs(w)
+    mask = np.ones((1, 1, 4, 4), np.uint8)
+    rp, ci = _mask_to_csr(mask)
+    plan = sdl.tile_plan(rp, ci, 1, 1, 256, 64)
+    order = torch.tensor([1, 5], dtype=torch.int32, device="cuda")  # 5: no such tile
+    sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, plan=plan, order=order)
+    assert sdl.last_device_status() == sdl.SDL_ERR_BAD_MASK
+
+
 def test_bad_tile_plan_entry_is_reported():
     w = synth.small_workload(L=256, H=1, H_kv=1, d=128)
     _, dev = _inputs(w)
