@@ -36,8 +36,9 @@ constexpr int kOrderBins = 2 * 1024 + 1;  // tile costs 0 .. 2 nb, nb <= 1024
 // One CTA: the order in which the attention kernel takes its tiles, costliest
 // first, so that the long tiles of heavy heads do not run last and leave the
 // other SMs idle.  A tile's cost is the sum of its two query blocks' list
-// lengths (an upper bound of the union it walks); a counting sort orders them
-// (equal costs in any order).  order[r] = the r-th tile to take.
+// lengths (an upper bound of the union it walks); a stable counting sort orders
+// them (equal costs keep the tile order, so tiles of one head stay together and
+// share its K and V in L2).  order[r] = the r-th tile to take.
 __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __restrict__ row_ptr,
                                                               const int32_t* __restrict__ plan,
                                                               int BH, int nb, int n_qt,
@@ -74,7 +75,20 @@ __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __r
     pos += cnt[y];
   }
   __syncthreads();
-  for (int x = tid; x < n; x += kOrderThreads) order[atomicAdd(&start[cost(x)], 1)] = x;
+  // stable scatter: one warp walks the tiles in order, 32 at a time; lanes with
+  // equal costs take consecutive places in lane order
+  if (tid < 32) {
+    for (int base = 0; base < n; base += 32) {
+      const int x = base + tid;
+      const int c = x < n ? cost(x) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, c);
+      const int rank = __popc(peers & ((1u << tid) - 1u));
+      if (x < n) order[start[c] + rank] = x;
+      __syncwarp();
+      if (x < n && tid == __ffs(peers) - 1) start[c] += __popc(peers);
+      __syncwarp();
+    }
+  }
 }
 
 // Adjacent pairs (2p, 2p+1), for heads too long for the greedy plan.

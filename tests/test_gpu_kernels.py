@@ -340,6 +340,9 @@ def test_tile_order_is_costliest_first_and_exact(L, H, density):
                      for x in range(H * n_qt)])
     assert np.all(np.diff(cost[o]) <= 0)
     assert cost[o[0]] == cost.max()
+    # stable: equal costs keep the tile order
+    same = np.diff(cost[o]) == 0
+    assert np.all(np.diff(o)[same] > 0)
 
 
 def test_bad_tile_order_entry_is_reported():
