@@ -523,7 +523,7 @@ def main():
                    4 * w.B * runner.H * w.nb * w.nb)
     # dense baseline on distinct inputs per launch (larger than L2 in total)
     de = []
-    for i in range(min(6, len(inputs))):
+    for i in range(min(11, len(inputs))):
         x = inputs[i]
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
