@@ -342,7 +342,8 @@ size_t sdl_col_scores_workspace_bytes(const sdl_shape* shape) {
   if (check_shape(shape) != SDL_OK) return 0;
   const size_t nb = shape->L / shape->block;
   return align256(sdl_scores_workspace_bytes(shape)) +
-         align256(sizeof(float) * 2 * shape->B * shape->H * nb);
+         align256(sizeof(float) * 2 * shape->B * shape->H * nb) +
+         align256(col_partial_bytes(*shape));
 }
 
 sdl_status sdl_col_scores(const void* q, const void* k, const sdl_shape* shape, float scale,
@@ -362,10 +363,12 @@ sdl_status sdl_col_scores(const void* q, const void* k, const sdl_shape* shape, 
   float* qbar = reinterpret_cast<float*>(w);
   float* kbar = reinterpret_cast<float*>(w + align256(sizeof(float) * s.B * s.H * nb * s.d));
   float2* stats = reinterpret_cast<float2*>(w + align256(sdl_scores_workspace_bytes(shape)));
+  float2* part = reinterpret_cast<float2*>(w + align256(sdl_scores_workspace_bytes(shape)) +
+                                           align256(sizeof(float) * 2 * s.B * s.H * nb));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t ce = launch_pool(q, k, s, qbar, kbar, st);
   if (ce != cudaSuccess) return cuda_fail(ce);
-  ce = launch_col_scores(k, s, resolve_scale(scale, s.d), qbar, stats, col_scores, st);
+  ce = launch_col_scores(k, s, resolve_scale(scale, s.d), qbar, part, stats, col_scores, st);
   if (ce != cudaSuccess) return cuda_fail(ce);
   return SDL_OK;
 }

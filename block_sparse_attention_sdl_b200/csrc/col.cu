@@ -12,9 +12,12 @@
 //   attend: softmax over the kept keys only, for every query token of the head
 //
 // Kernels:
-//   col_stats_kernel  per (b, h, 16 query blocks): row max and sum of the
-//                     block-mean queries' logits over every key (fp32 FFMA).
-//   col_sum_kernel    per (b, h, 64 keys): the column sums of the softmax
+//   col_stats_kernel  per (b, h, 128 query blocks, 512 keys): row max and
+//                     sum of exp of the block-mean queries' logits over those
+//                     keys (fp32 FFMA, 128 x 128 tiles, 8 x 8 per thread);
+//   col_combine_kernel per row: its maximum and sum over all keys, merged
+//                     from the partials in key order;
+//   col_sum_kernel    per (b, h, 128 keys): the column sums of the softmax
 //                     weights, over the query blocks in a fixed order (no
 //                     atomics: the same bits on every run).
 //   col_select_kernel per (b, h): radix select of the Lc-th largest score
@@ -54,13 +57,19 @@ void fill_col_args(ColArgs& c, const sdl_shape& s, float scale) {
   }
 }
 
-constexpr int kCR = 16;   // query blocks per tile
-constexpr int kCK = 128;  // keys per tile
-constexpr int kCJ = kCK / 32;  // keys per thread: tx + 32 j
-constexpr int kCThreads = 128;
+// Score tiles: 128 query blocks x 128 keys per CTA of 256 threads, each thread
+// 8 x 8 logits (rows ty + 16 r, keys tx + 16 j), fp32 FFMA over d from shared
+// memory (rows padded by 4 floats: the float4 reads of 16 keys hit every bank
+// once per pair of wavefronts, the 2 rows of a warp are broadcasts).
+constexpr int kGR = 128;       // query blocks per tile
+constexpr int kGK = 128;       // keys per tile
+constexpr int kGT = 256;       // threads
+constexpr int kGKT = 4;        // key tiles per CTA of the statistics pass
 
-// qs [kCR][d+4] (block-mean queries), ks [kCK][d+4] (keys as fp32)
-inline size_t col_smem_bytes(int d) { return sizeof(float) * (size_t)(kCR + kCK) * (d + 4); }
+inline int col_groups(int L) { return ((L + kGK - 1) / kGK + kGKT - 1) / kGKT; }
+// qs [kGR][d+4] (block-mean queries), ks [kGK][d+4] (keys as fp32)
+inline size_t col_smem_bytes(int d) { return sizeof(float) * (size_t)(kGR + kGK) * (d + 4); }
+constexpr size_t kColSumExtra = sizeof(float) * (16 * kGK + 2 * kGR);
 
 template <typename T>
 __device__ __forceinline__ float to_f(T x);
@@ -73,11 +82,11 @@ __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
   return __bfloat162float(x);
 }
 
-// Rows i0 .. i0+kCR of Qbar (head h) into qs; zero rows past nb.
+// Rows i0 .. i0+kGR of Qbar (head h) into qs; zero rows past nb.
 __device__ __forceinline__ void load_q_tile(const float* __restrict__ qsrc, int nb, int d, int i0,
                                             float* qs) {
   const int dp = d + 4, d4 = d / 4;
-  for (int x = threadIdx.x; x < kCR * d4; x += kCThreads) {
+  for (int x = threadIdx.x; x < kGR * d4; x += kGT) {
     const int r = x / d4, c = (x % d4) * 4;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (i0 + r < nb) v = *reinterpret_cast<const float4*>(qsrc + (int64_t)(i0 + r) * d + c);
@@ -85,7 +94,7 @@ __device__ __forceinline__ void load_q_tile(const float* __restrict__ qsrc, int 
   }
 }
 
-// Keys u0 .. u0+kCK of KV head kh into ks (fp32; zero past L), 16 bytes per
+// Keys u0 .. u0+kGK of KV head kh into ks (fp32; zero past L), 16 bytes per
 // load (the (b, t, h) strides are multiples of 16 bytes and d of 8 elements).
 template <typename T>
 __device__ __forceinline__ void load_k_tile(const T* __restrict__ k, const int64_t* ks, int b,
@@ -93,7 +102,7 @@ __device__ __forceinline__ void load_k_tile(const T* __restrict__ k, const int64
   constexpr int V = 16 / sizeof(T);  // elements per load
   const int dp = d + 4, dv = d / V;
 #pragma unroll 4
-  for (int x = threadIdx.x; x < kCK * dv; x += kCThreads) {
+  for (int x = threadIdx.x; x < kGK * dv; x += kGT) {
     const int r = x / dv, c = (x % dv) * V;
     uint4 u = make_uint4(0u, 0u, 0u, 0u);
     if (u0 + r < L)
@@ -107,132 +116,167 @@ __device__ __forceinline__ void load_k_tile(const T* __restrict__ k, const int64
   }
 }
 
-// z[a][j] for the thread's 4 rows (ty*4 + a) and kCJ keys (tx + 32 j).
+// z[r][j] = scale * (qs row ty + 16 r) . (ks row tx + 16 j), summed over d in order.
 __device__ __forceinline__ void tile_logits(const float* qs, const float* kt, int d, float scale,
-                                            float (&z)[4][kCJ]) {
-  const int dp = d + 4, ty = threadIdx.x / 32, tx = threadIdx.x % 32;
+                                            float (&z)[8][8]) {
+  const int dp = d + 4, ty = threadIdx.x / 16, tx = threadIdx.x % 16;
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int j = 0; j < kCJ; ++j) z[a][j] = 0.f;
+    for (int j = 0; j < 8; ++j) z[r][j] = 0.f;
+#pragma unroll 1
   for (int c = 0; c < d; c += 4) {
-    float4 kv[kCJ];
+    float4 a[8], bv[8];
 #pragma unroll
-    for (int j = 0; j < kCJ; ++j) kv[j] = *reinterpret_cast<const float4*>(kt + (tx + 32 * j) * dp + c);
+    for (int r = 0; r < 8; ++r) a[r] = *reinterpret_cast<const float4*>(qs + (ty + 16 * r) * dp + c);
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const float4 q = *reinterpret_cast<const float4*>(qs + (ty * 4 + a) * dp + c);
+    for (int j = 0; j < 8; ++j) bv[j] = *reinterpret_cast<const float4*>(kt + (tx + 16 * j) * dp + c);
 #pragma unroll
-      for (int j = 0; j < kCJ; ++j)
-        z[a][j] += q.x * kv[j].x + q.y * kv[j].y + q.z * kv[j].z + q.w * kv[j].w;
-    }
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float t = fmaf(a[r].x, bv[j].x, z[r][j]);
+        t = fmaf(a[r].y, bv[j].y, t);
+        t = fmaf(a[r].z, bv[j].z, t);
+        z[r][j] = fmaf(a[r].w, bv[j].w, t);
+      }
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int j = 0; j < kCJ; ++j) z[a][j] *= scale;
+    for (int j = 0; j < 8; ++j) z[r][j] *= scale;
 }
 
-// grid (ceil(nb / kCR), H, B): stats[b, h, i] = (max over u of z_iu, sum over u
-// of exp(z_iu - max)).
+// Statistics pass.  grid (col_groups(L), ceil(nb / kGR), B * H): for its
+// query blocks and its kGKT key tiles, part[bh, i, group] = (max over those
+// keys of z_iu, sum of exp(z_iu - max)).
 template <typename T>
-__global__ void __launch_bounds__(kCThreads) col_stats_kernel(const float* __restrict__ qbar,
-                                                              const T* __restrict__ k, ColArgs c,
-                                                              float2* __restrict__ stats) {
+__global__ void __launch_bounds__(kGT) col_stats_kernel(const float* __restrict__ qbar,
+                                                        const T* __restrict__ k, ColArgs c,
+                                                        float2* __restrict__ part) {
   extern __shared__ float sm[];
   float* qs = sm;
-  float* kt = qs + kCR * (c.d + 4);
-  const int b = blockIdx.z, h = blockIdx.y, i0 = blockIdx.x * kCR;
+  float* kt = qs + kGR * (c.d + 4);
+  const int bh = blockIdx.z, b = bh / c.H, h = bh % c.H, i0 = blockIdx.y * kGR;
   const int kh = h / (c.H / c.Hkv);
-  load_q_tile(qbar + ((int64_t)b * c.H + h) * c.nb * c.d, c.nb, c.d, i0, qs);
-  float m[4], l[4];
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  const int ngroups = gridDim.x;
+  load_q_tile(qbar + (int64_t)bh * c.nb * c.d, c.nb, c.d, i0, qs);
+  float m[8], l[8];
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    m[a] = -INFINITY;
-    l[a] = 0.f;
+  for (int r = 0; r < 8; ++r) {
+    m[r] = -INFINITY;
+    l[r] = 0.f;
   }
-  for (int u0 = 0; u0 < c.L; u0 += kCK) {
+  for (int t = 0; t < kGKT; ++t) {
+    const int u0 = (blockIdx.x * kGKT + t) * kGK;
+    if (u0 >= c.L) break;
     __syncthreads();
     load_k_tile<T>(k, c.ks, b, kh, c.d, u0, c.L, kt);
     __syncthreads();
-    float z[4][kCJ];
+    float z[8][8];
     tile_logits(qs, kt, c.d, c.scale, z);
 #pragma unroll
-    for (int j = 0; j < kCJ; ++j)
-      if (u0 + (int)(threadIdx.x % 32) + 32 * j >= c.L)  // no such key
+    for (int j = 0; j < 8; ++j)
+      if (u0 + tx + 16 * j >= c.L)  // no such key
 #pragma unroll
-        for (int a = 0; a < 4; ++a) z[a][j] = -INFINITY;
+        for (int r = 0; r < 8; ++r) z[r][j] = -INFINITY;
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      float mt = m[a];
+    for (int r = 0; r < 8; ++r) {
+      float mt = m[r];
 #pragma unroll
-      for (int j = 0; j < kCJ; ++j) mt = fmaxf(mt, z[a][j]);
-      float t = l[a] * expf(m[a] - mt);
+      for (int j = 0; j < 8; ++j) mt = fmaxf(mt, z[r][j]);
+      float acc = l[r] * expf(m[r] - mt);
 #pragma unroll
-      for (int j = 0; j < kCJ; ++j) t += expf(z[a][j] - mt);
-      l[a] = t;
-      m[a] = mt;
+      for (int j = 0; j < 8; ++j) acc += expf(z[r][j] - mt);
+      l[r] = acc;
+      m[r] = mt;
     }
   }
-  // merge the 32 lanes' partial (max, sum) of each row, in a fixed order
+  // merge the 16 key lanes' partial (max, sum) of each row, in a fixed order
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    for (int o = 16; o > 0; o >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, m[a], o);
-      const float l2 = __shfl_xor_sync(0xffffffffu, l[a], o);
-      const float mt = fmaxf(m[a], m2);
-      l[a] = l[a] * expf(m[a] - mt) + l2 * expf(m2 - mt);
-      m[a] = mt;
+  for (int r = 0; r < 8; ++r) {
+    for (int o = 8; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m[r], o);
+      const float l2 = __shfl_xor_sync(0xffffffffu, l[r], o);
+      const float mt = fmaxf(m[r], m2);
+      l[r] = (mt == -INFINITY) ? 0.f : l[r] * expf(m[r] - mt) + l2 * expf(m2 - mt);
+      m[r] = mt;
     }
-    const int i = i0 + (threadIdx.x / 32) * 4 + a;
-    if (threadIdx.x % 32 == 0 && i < c.nb)
-      stats[((int64_t)b * c.H + h) * c.nb + i] = make_float2(m[a], l[a]);
+    const int i = i0 + ty + 16 * r;
+    if (tx == 0 && i < c.nb)
+      part[((int64_t)bh * c.nb + i) * ngroups + blockIdx.x] = make_float2(m[r], l[r]);
   }
 }
 
-// grid (ceil(L / kCK), H, B): S[b, h, u] = (1/nb) sum over i of exp(z_iu - max_i) / sum_i.
+// stats[bh, i] = (max, 1 / sum) of row i over all keys, from its groups in order.
+__global__ void col_combine_kernel(const float2* __restrict__ part, int rows, int ngroups,
+                                   float2* __restrict__ stats) {
+  const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x >= rows) return;
+  const float2* p = part + x * ngroups;
+  float m = -INFINITY, l = 0.f;
+  for (int g = 0; g < ngroups; ++g) {
+    const float2 v = p[g];
+    const float mt = fmaxf(m, v.x);
+    if (mt == -INFINITY) continue;
+    l = l * expf(m - mt) + v.y * expf(v.x - mt);
+    m = mt;
+  }
+  stats[x] = make_float2(m, 1.0f / l);
+}
+
+// Sum pass.  grid (ceil(L / kGK), B * H): S[bh, u] = (1/nb) sum over i of
+// exp(z_iu - max_i) / sum_i, the query blocks in order (no atomics: the same
+// bits on every run).
 template <typename T>
-__global__ void __launch_bounds__(kCThreads) col_sum_kernel(const float* __restrict__ qbar,
-                                                            const T* __restrict__ k, ColArgs c,
-                                                            const float2* __restrict__ stats,
-                                                            float* __restrict__ S) {
+__global__ void __launch_bounds__(kGT) col_sum_kernel(const float* __restrict__ qbar,
+                                                      const T* __restrict__ k, ColArgs c,
+                                                      const float2* __restrict__ stats,
+                                                      float* __restrict__ S) {
   extern __shared__ float sm[];
   float* qs = sm;
-  float* kt = qs + kCR * (c.d + 4);
-  __shared__ float part[kCThreads / 32][kCK];
-  const int b = blockIdx.z, h = blockIdx.y, u0 = blockIdx.x * kCK;
+  float* kt = qs + kGR * (c.d + 4);
+  float* red = kt + kGK * (c.d + 4);  // [16][kGK]: per row group ty, per key
+  float* rm = red + 16 * kGK;         // [kGR] row maxima of the tile
+  float* rinv = rm + kGR;             // [kGR] inverse row sums
+  const int bh = blockIdx.y, b = bh / c.H, h = bh % c.H, u0 = blockIdx.x * kGK;
   const int kh = h / (c.H / c.Hkv);
-  const int ty = threadIdx.x / 32, tx = threadIdx.x % 32;
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
   load_k_tile<T>(k, c.ks, b, kh, c.d, u0, c.L, kt);
-  const float* qsrc = qbar + ((int64_t)b * c.H + h) * c.nb * c.d;
-  const float2* st = stats + ((int64_t)b * c.H + h) * c.nb;
-  float acc[kCJ];
+  const float* qsrc = qbar + (int64_t)bh * c.nb * c.d;
+  const float2* st = stats + (int64_t)bh * c.nb;
+  float acc[8];
 #pragma unroll
-  for (int j = 0; j < kCJ; ++j) acc[j] = 0.f;
-  for (int i0 = 0; i0 < c.nb; i0 += kCR) {
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  for (int i0 = 0; i0 < c.nb; i0 += kGR) {
     __syncthreads();
     load_q_tile(qsrc, c.nb, c.d, i0, qs);
+    for (int x = threadIdx.x; x < kGR; x += kGT) {
+      const float2 v = i0 + x < c.nb ? st[i0 + x] : make_float2(0.f, 0.f);
+      rm[x] = v.x;
+      rinv[x] = v.y;
+    }
     __syncthreads();
-    float z[4][kCJ];
+    float z[8][8];
     tile_logits(qs, kt, c.d, c.scale, z);
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int i = i0 + ty * 4 + a;
-      if (i < c.nb) {
-        const float2 s2 = st[i];
-        const float inv = 1.0f / s2.y;
+    for (int r = 0; r < 8; ++r) {
+      const int ri = ty + 16 * r;
+      if (i0 + ri < c.nb) {
+        const float mr = rm[ri], ir = rinv[ri];
 #pragma unroll
-        for (int j = 0; j < kCJ; ++j) acc[j] += expf(z[a][j] - s2.x) * inv;
+        for (int j = 0; j < 8; ++j) acc[j] += expf(z[r][j] - mr) * ir;
       }
     }
   }
 #pragma unroll
-  for (int j = 0; j < kCJ; ++j) part[ty][tx + 32 * j] = acc[j];
+  for (int j = 0; j < 8; ++j) red[ty * kGK + tx + 16 * j] = acc[j];
   __syncthreads();
-  for (int x = threadIdx.x; x < kCK && u0 + x < c.L; x += kCThreads) {
+  for (int x = threadIdx.x; x < kGK && u0 + x < c.L; x += kGT) {
     float t = 0.f;
-    for (int w = 0; w < kCThreads / 32; ++w) t += part[w][x];
-    S[((int64_t)b * c.H + h) * c.L + u0 + x] = t / (float)c.nb;
+    for (int w = 0; w < 16; ++w) t += red[w * kGK + x];
+    S[(int64_t)bh * c.L + u0 + x] = t / (float)c.nb;
   }
 }
 
@@ -332,15 +376,20 @@ __global__ void col_gather_kernel(const uint8_t* __restrict__ k, const uint8_t* 
 
 }  // namespace
 
+size_t col_partial_bytes(const sdl_shape& s) {
+  return sizeof(float2) * (size_t)s.B * s.H * (s.L / s.block) * col_groups(s.L);
+}
+
 cudaError_t launch_col_scores(const void* k, const sdl_shape& s, float scale, const float* qbar,
-                              float2* stats, float* S, cudaStream_t st) {
+                              float2* part, float2* stats, float* S, cudaStream_t st) {
   ColArgs c;
   fill_col_args(c, s, scale);
-  const size_t smem = col_smem_bytes(s.d);
-  const dim3 g1((c.nb + kCR - 1) / kCR, s.H, s.B), g2((s.L + kCK - 1) / kCK, s.H, s.B);
+  const size_t smem1 = col_smem_bytes(s.d), smem2 = smem1 + kColSumExtra;
+  const int ngroups = col_groups(s.L);
+  const dim3 g1(ngroups, (c.nb + kGR - 1) / kGR, s.B * s.H), g2((s.L + kGK - 1) / kGK, s.B * s.H);
   static bool attr_set = false;  // per function; the size needed is at most this
   if (!attr_set) {
-    const int most = (int)col_smem_bytes(128);
+    const int most = (int)(col_smem_bytes(128) + kColSumExtra);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(col_stats_kernel<__nv_bfloat16>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, most)) ||
@@ -353,16 +402,20 @@ cudaError_t launch_col_scores(const void* k, const sdl_shape& s, float scale, co
       return e;
     attr_set = true;
   }
+  const int rows = s.B * s.H * c.nb;
   if (s.dtype == SDL_BF16) {
-    col_stats_kernel<__nv_bfloat16><<<g1, kCThreads, smem, st>>>(
-        qbar, static_cast<const __nv_bfloat16*>(k), c, stats);
-    col_sum_kernel<__nv_bfloat16><<<g2, kCThreads, smem, st>>>(
+    col_stats_kernel<__nv_bfloat16><<<g1, kGT, smem1, st>>>(
+        qbar, static_cast<const __nv_bfloat16*>(k), c, part);
+  } else {
+    col_stats_kernel<float><<<g1, kGT, smem1, st>>>(qbar, static_cast<const float*>(k), c, part);
+  }
+  col_combine_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, rows, ngroups, stats);
+  if (s.dtype == SDL_BF16) {
+    col_sum_kernel<__nv_bfloat16><<<g2, kGT, smem2, st>>>(
         qbar, static_cast<const __nv_bfloat16*>(k), c, stats, S);
   } else {
-    col_stats_kernel<float><<<g1, kCThreads, smem, st>>>(qbar, static_cast<const float*>(k), c,
-                                                          stats);
-    col_sum_kernel<float><<<g2, kCThreads, smem, st>>>(qbar, static_cast<const float*>(k), c,
-                                                        stats, S);
+    col_sum_kernel<float><<<g2, kGT, smem2, st>>>(qbar, static_cast<const float*>(k), c, stats,
+                                                   S);
   }
   return cudaGetLastError();
 }

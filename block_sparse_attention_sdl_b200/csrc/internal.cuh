@@ -63,8 +63,9 @@ cudaError_t launch_anchor(const void* q, const void* k, const sdl_shape& s, floa
                           int* status, cudaStream_t st);
 size_t anchor_barrier_bytes();
 // column-sparse attention (col.cu)
+size_t col_partial_bytes(const sdl_shape& s);
 cudaError_t launch_col_scores(const void* k, const sdl_shape& s, float scale, const float* qbar,
-                              float2* stats, float* S, cudaStream_t st);
+                              float2* part, float2* stats, float* S, cudaStream_t st);
 cudaError_t launch_col_select(const float* S, int BH, int L, int Lc, int32_t* cols,
                               cudaStream_t st);
 cudaError_t launch_col_gather(const void* k, const void* v, const sdl_shape& s,

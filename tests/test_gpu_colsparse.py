@@ -119,3 +119,23 @@ def test_col_schedule_refreshes_at_anchors_only():
             Ow, _ = oracle.col_attention(host["q"], host["k"], host["v"], att.cols.cpu().numpy())
             check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, "bf16")
     assert sdl.last_device_status() == sdl.SDL_OK
+
+
+@pytest.mark.parametrize("heads", [(0, 17), (5, 31)])
+def test_col_scores_full_size_sampled_heads(heads):
+    """The 8K / 32-head workload that bench.py times (--variant pulsecol): column
+    scores of two heads against the oracle, and the kept columns of those heads
+    exactly the oracle's rule on the GPU's scores."""
+    w = synth.WORKLOADS["bf16-L8192-H32-s90"]
+    host, dev = _host_dev(w)
+    S = sdl.col_scores(dev["q"], dev["k"], w.bs)
+    cols = sdl.col_select(S, dev["q"], dev["k"], w.bs, w.sparsity)
+    torch.cuda.synchronize()
+    assert sdl.last_device_status() == sdl.SDL_OK
+    hs = list(heads)
+    Sw = oracle.col_scores(np.ascontiguousarray(host["q"][:, :, hs]),
+                           np.ascontiguousarray(host["k"][:, :, hs]), w.bs)
+    got = S.cpu().numpy()[:, hs]
+    assert np.allclose(got, Sw, rtol=2e-5, atol=1e-9)
+    want = oracle.col_select(got.astype(np.float64), w.sparsity)
+    assert np.array_equal(cols.cpu().numpy()[:, hs], want)
