@@ -188,8 +188,9 @@ class Runner:
                    "v": x["v"][:, :, kv0:kv1].contiguous()} for x in xs]
         return xs
 
-    def step(self, x, s, ev=None):
+    def step(self, x, s, ev=None, out=None):
         att, w, rt = self.att, self.w, self.rt
+        out = self.out if out is None else out
         dense = rt.is_dense(s, self.dense_steps)
         if not dense and (rt.is_anchor(s, self.interval, self.dense_steps) or
                           att.mask_step is None):
@@ -205,12 +206,12 @@ class Runner:
             ev["s0"][-1].record()
             self.kinds.append("dense" if dense else "sparse")
         if dense:
-            self.sdl.dense_attn(x["q"], x["k"], x["v"], w.bs, out=self.out)
+            self.sdl.dense_attn(x["q"], x["k"], x["v"], w.bs, out=out)
         elif self.pulsecol:
-            att.attend(x["q"], x["k"], x["v"], out=self.out)
+            att.attend(x["q"], x["k"], x["v"], out=out)
         else:
             self.sdl.sparse_attn(x["q"], x["k"], x["v"], att.row_ptr, att.col_idx, w.bs,
-                                 out=self.out, plan=att.plan, order=att.order)
+                                 out=out, plan=att.plan, order=att.order)
         if ev is not None:
             ev["s1"].append(torch.cuda.Event(enable_timing=True))
             ev["s1"][-1].record()
@@ -280,24 +281,47 @@ def launches_per_anchor(block: int, sharded: bool = False, fused: bool = False):
 
 def e2e_measure(runner, inputs, steps, device):
     """Same step loop with the inputs copied from pinned host memory and the
-    output copied back, every step, inside the timed region."""
+    output copied back, every step, inside the timed region.  Uploads, the step
+    and downloads run on three streams over double-buffered device tensors (the
+    upload of step i+1 and the download of step i-1 overlap step i), ordered by
+    events, as a serving loop would run them."""
     ring = min(len(inputs), 8)
     host_in = []
     for x in inputs[:ring]:
         host_in.append({k: v.cpu().pin_memory() for k, v in x.items()})
     host_out = [torch.empty_like(runner.out, device="cpu").pin_memory() for _ in range(2)]
-    dev_in = {k: torch.empty_like(v) for k, v in inputs[0].items()}
-    bytes_in = sum(v.numel() * v.element_size() for v in dev_in.values())
+    dev_in = [{k: torch.empty_like(v) for k, v in inputs[0].items()} for _ in range(2)]
+    dev_out = [torch.empty_like(runner.out) for _ in range(2)]
+    bytes_in = sum(v.numel() * v.element_size() for v in dev_in[0].values())
     bytes_out = runner.out.numel() * runner.out.element_size()
+    s_c = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
     def loop(n):
         runner.att.mask_step = None
+        s_in.wait_stream(s_c)  # uploads start after whatever the compute stream has queued
+        in_done = [torch.cuda.Event() for _ in range(2)]
+        c_done = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
         for i in range(n):
-            h = host_in[i % ring]
-            for k in dev_in:
-                dev_in[k].copy_(h[k], non_blocking=True)
-            runner.step(dev_in, steps[i])
-            host_out[i % 2].copy_(runner.out, non_blocking=True)
+            b, h = i % 2, host_in[i % ring]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(c_done[b])  # step i-2 has read this input buffer
+                for k in dev_in[b]:
+                    dev_in[b][k].copy_(h[k], non_blocking=True)
+                in_done[b].record(s_in)
+            s_c.wait_event(in_done[b])
+            if i >= 2:
+                s_c.wait_event(out_done[b])  # step i-2's output has been read back
+            runner.step(dev_in[b], steps[i], out=dev_out[b])
+            c_done[b].record(s_c)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(c_done[b])
+                host_out[b].copy_(dev_out[b], non_blocking=True)
+                out_done[b].record(s_out)
+        for e in out_done:
+            s_c.wait_event(e)
 
     loop(min(3, len(steps)))
     torch.cuda.synchronize()
