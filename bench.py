@@ -355,12 +355,16 @@ def traffic_record():
 def cpu_oracle_sample(w, seed, target_s=8.0):
     """Times the fp64 oracle's block-sparse attention on a bounded sample of the
     workload's query rows (all heads, evenly spaced query blocks) of step 0 with
-    its anchor mask; returns (TFLOP/s, cores, description)."""
+    its anchor mask; returns (TFLOP/s, cores, description, sample seconds, extra)
+    with extra = the oracle's anchor work (block scores + selection) in seconds and
+    the sample's time scaled linearly to every query block (an extrapolation)."""
     import oracle
     import synth
     host = synth.host_inputs(w, 0, seed)
+    ta = time.perf_counter()
     P = oracle.block_scores(host["q"], host["k"], w.bs)
     mask, _, _ = oracle.select(P, w.sparsity)
+    anchor_s = time.perf_counter() - ta
     cores = os.cpu_count() or 1
     nb = w.nb
 
@@ -384,7 +388,8 @@ def cpu_oracle_sample(w, seed, target_s=8.0):
     dt = time.perf_counter() - t0
     desc = (f"block-sparse attention of {len(rows)} query rows ({nblk} of {nb} query blocks x "
             f"{w.H} heads, step 0 with its anchor mask), fp64, {cores} threads")
-    return flops(rows) / dt / 1e12, cores, desc, dt
+    extra = {"anchor_s": anchor_s, "full_step_s_extrapolated": dt * nb / nblk}
+    return flops(rows) / dt / 1e12, cores, desc, dt, extra
 
 
 def run_reference(args):
@@ -397,7 +402,7 @@ def run_reference(args):
     per_step_target = max(0.5, 60.0 / max(1, args.steps + args.warmup))
     vals, tot = [], 0.0
     for i in range(args.warmup + args.steps):
-        v, cores, desc, dt = cpu_oracle_sample(w, args.seed, target_s=per_step_target)
+        v, cores, desc, dt, extra = cpu_oracle_sample(w, args.seed, target_s=per_step_target)
         if i >= args.warmup:
             vals.append(v)
             tot += dt
@@ -411,7 +416,7 @@ def run_reference(args):
                    "heads": w.H, "kv_heads": w.H_kv, "head_dim": w.d, "block": w.bs,
                    "sparsity": w.sparsity, "parallelism": "cpu oracle"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, **extra},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -568,8 +573,9 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, desc, _ = cpu_oracle_sample(w, seed)
-        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+        v, cores, desc, _, extra = cpu_oracle_sample(w, seed)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+               **extra}
 
     n_anchor = len(anchor_ms)
     # the ncu record covers the block-sparse kernel's launch only
