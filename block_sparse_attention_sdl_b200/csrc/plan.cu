@@ -32,6 +32,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
 
 constexpr int kOrderThreads = 1024;
 constexpr int kOrderBins = 2 * 1024 + 1;  // tile costs 0 .. 2 nb, nb <= 1024
+// tiles whose costs are kept in shared memory for the serial stable scatter
+// (16 bits each); beyond this the scatter recomputes them from the lists
+constexpr int kOrderCached = 48 * 1024;
 
 // One CTA: the order in which the attention kernel takes its tiles, costliest
 // first, so that the long tiles of heavy heads do not run last and leave the
@@ -45,8 +48,10 @@ __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __r
                                                               int32_t* __restrict__ order) {
   __shared__ int start[kOrderBins];
   __shared__ int s_warp[32];
+  extern __shared__ uint16_t cost_sm[];  // every tile's cost, when n <= kOrderCached
   const int n = BH * n_qt, tid = threadIdx.x;
-  auto cost = [&](int x) -> int {
+  const bool cached = n <= kOrderCached;
+  auto cost_of = [&](int x) -> int {
     const int64_t r0 = (int64_t)(x / n_qt) * nb;
     int c = 0;
     for (int s = 0; s < 2; ++s) {
@@ -55,9 +60,14 @@ __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __r
     }
     return c < 0 ? 0 : (c >= kOrderBins ? kOrderBins - 1 : c);
   };
+  auto cost = [&](int x) -> int { return cached ? (int)cost_sm[x] : cost_of(x); };
   for (int c = tid; c < kOrderBins; c += kOrderThreads) start[c] = 0;
   __syncthreads();
-  for (int x = tid; x < n; x += kOrderThreads) atomicAdd(&start[cost(x)], 1);
+  for (int x = tid; x < n; x += kOrderThreads) {
+    const int c = cost_of(x);
+    if (cached) cost_sm[x] = (uint16_t)c;
+    atomicAdd(&start[c], 1);
+  }
   __syncthreads();
   // first position of each cost, costs in descending order: thread t owns bins
   // kOrderBins - 1 - 3t, -3t-1, -3t-2
@@ -126,7 +136,16 @@ cudaError_t launch_plan(const int32_t* row_ptr, const int32_t* col_idx, int B, i
 
 cudaError_t launch_tile_order(const int32_t* row_ptr, const int32_t* plan, int B, int H, int nb,
                               int32_t* order, cudaStream_t st) {
-  order_kernel<<<1, kOrderThreads, 0, st>>>(row_ptr, plan, B * H, nb, (nb + 1) / 2, order);
+  const int n = B * H * ((nb + 1) / 2);
+  const size_t smem = n <= kOrderCached ? sizeof(uint16_t) * (size_t)n : 0;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(sizeof(uint16_t) * kOrderCached));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  order_kernel<<<1, kOrderThreads, smem, st>>>(row_ptr, plan, B * H, nb, (nb + 1) / 2, order);
   return cudaGetLastError();
 }
 
