@@ -565,10 +565,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
         // P = exp2(S * scale * log2e - m) on a kept half, 0 otherwise (a kept
         // half always has a finite reference here: its own maximum raised it);
-        // bf16 pairs over S's first 64 columns; l sums the rounded weights
-        // (pair arithmetic packed: x = s * scale_log2 - m, row sums)
+        // bf16 pairs over S's first 64 columns; l sums the rounded weights, each
+        // bf16 half added to an fp32 sum by one mixed-precision add (x = s *
+        // scale_log2 - m packed in pairs)
         const uint64_t sl2x2 = pack2(sl2, sl2), nmx2 = pack2(-m, -m);
-        uint64_t rs2 = pack2(0.f, 0.f), rx2 = pack2(0.f, 0.f);
+        float rsa = 0.f, rsb = 0.f;  // row sums of the rounded weights (low, high halves)
+        uint64_t rx2 = pack2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {  // 32 weights -> 16 packed columns at a time
           const bool kp = c < 2 ? keep0 : keep1;
@@ -582,7 +584,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               const float p0 = ex2_approx(xv.x), p1 = ex2_approx(xv.y);
               __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
               const uint32_t u = *reinterpret_cast<uint32_t*>(&pk);
-              rs2 = add2(rs2, pack2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
+              asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+                  "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+                  : "+f"(rsa), "+f"(rsb) : "r"(u));
               if constexpr (kLse) rx2 = add2(rx2, pack2(p0, p1));
               pw[x / 2] = u;
             }
@@ -600,8 +604,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           }
         }
         {
-          const float2 a2 = unpack2(rs2), b2 = unpack2(rx2);
-          l += a2.x + a2.y;
+          const float2 b2 = unpack2(rx2);
+          l += rsa + rsb;
           lx += b2.x + b2.y;
         }
         tmem_wait_st();
