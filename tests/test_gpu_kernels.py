@@ -345,6 +345,27 @@ def test_tile_order_is_costliest_first_and_exact(L, H, density):
     assert np.all(np.diff(o)[same] > 0)
 
 
+def test_scheduled_attention_two_sequences_gqa():
+    """Tile plan and costliest-first take order over two sequences under GQA: the
+    oracle's result, LSE included, with tiles of both sequences interleaved."""
+    B, L, H, Hkv = 2, 1024, 4, 2
+    w = synth.small_workload(B=B, L=L, H=H, H_kv=Hkv, d=128, bs=64)
+    host, dev = _inputs(w)
+    nb = L // 64
+    rng = np.random.default_rng(2024)
+    mask = _random_mask(B, H, nb, 0.3, rng)
+    mask[1, 0] = 1  # one head of the second sequence keeps every block
+    rp, ci = _mask_to_csr(mask)
+    plan = sdl.tile_plan(rp, ci, B, H, L, 64)
+    order = sdl.tile_order(rp, plan, B, H, L, 64)
+    O, lse = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, want_lse=True,
+                             plan=plan, order=order)
+    assert sdl.last_device_status() == sdl.SDL_OK
+    Ow, lw = oracle.attention(host["q"], host["k"], host["v"], 64, mask=mask)
+    check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, "bf16")
+    assert np.abs(lse.cpu().numpy() - lw).max() <= TOL["bf16"]["lse"]
+
+
 def test_bad_tile_order_entry_is_reported():
     w = synth.small_workload(L=256, H=1, H_kv=1, d=128)
     _, dev = _inputs(w)
