@@ -685,15 +685,20 @@ std::atomic<unsigned> g_launches{0};
 
 template <int D, bool kLse>
 cudaError_t launch_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
-                      const CUtensorMap* tv, const CUtensorMap* to, cudaStream_t st, int grid) {
+                      const CUtensorMap* tv, const CUtensorMap* to, cudaStream_t st, int grid,
+                      int dev) {
   using Lay = Layout<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, kLse>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_tc_kernel<D, kLse>,
-                           cudaFuncAttributePreferredSharedMemoryCarveout,
-                           (int)cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) return e;
+  static std::atomic<bool> attrs_set[64];  // once per instantiation and device
+  if (!attrs_set[dev].load()) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, kLse>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_tc_kernel<D, kLse>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    attrs_set[dev].store(true);
+  }
   const int slot = (int)(g_launches.fetch_add(1u) % kSchedRing);
   attn_tc_kernel<D, kLse><<<grid, kThreads, Lay::kSmem, st>>>(*tq, *tk, *tv, *to, a, slot);
   return cudaGetLastError();
@@ -716,10 +721,10 @@ cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUten
   const int64_t cap = (int64_t)kCtasPerSm * g_num_sms[dev];
   const int grid = (int)(n_items < cap ? n_items : cap);
   if (a.d == 128)
-    return a.lse ? launch_tc<128, true>(a, tq, tk, tv, to, st, grid)
-                 : launch_tc<128, false>(a, tq, tk, tv, to, st, grid);
-  return a.lse ? launch_tc<64, true>(a, tq, tk, tv, to, st, grid)
-               : launch_tc<64, false>(a, tq, tk, tv, to, st, grid);
+    return a.lse ? launch_tc<128, true>(a, tq, tk, tv, to, st, grid, dev)
+                 : launch_tc<128, false>(a, tq, tk, tv, to, st, grid, dev);
+  return a.lse ? launch_tc<64, true>(a, tq, tk, tv, to, st, grid, dev)
+               : launch_tc<64, false>(a, tq, tk, tv, to, st, grid, dev);
 }
 
 }  // namespace sdl
