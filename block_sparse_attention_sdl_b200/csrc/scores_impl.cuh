@@ -90,8 +90,8 @@ __device__ __forceinline__ void pool_body(PoolTensor tq, PoolTensor tk, int B, i
   }
 }
 
-constexpr int kTI = 16;  // query blocks per CTA (4 per warp)
-constexpr int kTJ = 64;  // key blocks per shared-memory tile
+constexpr int kTI = 16;   // query blocks per CTA (4 per warp)
+constexpr int kTJ = 128;  // key blocks per shared-memory tile (4 per lane)
 constexpr int kScoreThreads = 128;
 
 inline size_t score_smem_bytes(int nb, int d) {
@@ -136,23 +136,31 @@ __device__ __forceinline__ void score_body(const float* __restrict__ qbar,
     }
     __syncthreads();
     if (!act) continue;
-    float acc[4][2];
+    // 4 query blocks (ty * 4 + a) x 4 key blocks (tx + 32 u) per thread: the
+    // four float4 reads of keys take the 32 banks once per wavefront, the
+    // query reads are broadcasts
+    float acc[4][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = 0.f;
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[a][u] = 0.f;
     for (int c = 0; c < d; c += 4) {
-      float4 kv0 = *reinterpret_cast<const float4*>(ks + tx * dp + c);
-      float4 kv1 = *reinterpret_cast<const float4*>(ks + (tx + 32) * dp + c);
+      float4 kv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        kv[u] = *reinterpret_cast<const float4*>(ks + (tx + 32 * u) * dp + c);
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
         float4 qv = *reinterpret_cast<const float4*>(qs + (ty * 4 + a) * dp + c);
-        acc[a][0] += qv.x * kv0.x + qv.y * kv0.y + qv.z * kv0.z + qv.w * kv0.w;
-        acc[a][1] += qv.x * kv1.x + qv.y * kv1.y + qv.z * kv1.z + qv.w * kv1.w;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          acc[a][u] += qv.x * kv[u].x + qv.y * kv[u].y + qv.z * kv[u].z + qv.w * kv[u].w;
       }
     }
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < 4; ++u) {
         int j = j0 + tx + 32 * u;
         if (j < nb) z[(ty * 4 + a) * nb + j] = acc[a][u] * scale;
       }
