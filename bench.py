@@ -211,7 +211,7 @@ class Runner:
             att.attend(x["q"], x["k"], x["v"], out=out)
         else:
             self.sdl.sparse_attn(x["q"], x["k"], x["v"], att.row_ptr, att.col_idx, w.bs,
-                                 out=out, plan=att.plan, order=att.order)
+                                 out=out, plan=att.plan, order=att.order, lists=att.lists)
         if ev is not None:
             ev["s1"].append(torch.cuda.Event(enable_timing=True))
             ev["s1"][-1].record()
@@ -224,7 +224,7 @@ class Runner:
         else:
             self.sdl.sparse_attn(x["q"], x["k"], x["v"], self.att.row_ptr, self.att.col_idx,
                                  self.w.bs, out=self.out, plan=self.att.plan,
-                                 order=self.att.order)
+                                 order=self.att.order, lists=self.att.lists)
         self.att.mask_step = None
 
 
@@ -269,11 +269,12 @@ def time_steps(runner, inputs, steps, dist_on, device, with_events=True):
     return ms, ev
 
 
-def launches_per_anchor(block: int, sharded: bool = False, fused: bool = False):
+def launches_per_anchor(block: int, sharded: bool = False, fused: bool = False,
+                        lists: bool = False):
     # fused: scores and selection in one launch; else pool, score; select: zero, 3
     # histogram passes, count, scan, write (+ the per-rank totals when the heads are
-    # sharded); tile plan and its order (64-token blocks)
-    plan = 2 if block == 64 else 0  # the plan and its take order
+    # sharded); tile plan and its order (64-token blocks), and the tiles' lists
+    plan = (2 + (1 if lists else 0)) if block == 64 else 0
     if fused:
         return 1 + plan
     return 2 + 7 + (1 if sharded else 0) + plan
@@ -433,7 +434,8 @@ def profile_kernel(runner, args):
     if args.profile == "sparse":
         fn = lambda: sdl.sparse_attn(x["q"], x["k"], x["v"], runner.att.row_ptr,
                                      runner.att.col_idx, w.bs, out=runner.out,
-                                     plan=runner.att.plan, order=runner.att.order)
+                                     plan=runner.att.plan, order=runner.att.order,
+                                     lists=runner.att.lists)
         flop = 4.0 * w.bs * w.bs * w.d * runner.att.budget
     else:
         fn = lambda: sdl.dense_attn(x["q"], x["k"], x["v"], out=runner.out)
@@ -617,11 +619,12 @@ def main():
                      "traffic": traffic},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        # pulsecol: gather + attention per step; pool, two score passes and the
-        # selection per refresh
-        "gpu_launches": (2 * len(steps) + 4 * n_anchor if runner.pulsecol else
-                         len(steps) + n_anchor * launches_per_anchor(w.bs, runner.att.sharded,
-                                                                     runner.att.fused)),
+        # pulsecol: gather + attention per step; pool, the score statistics, their
+        # combination, the score sums and the selection per refresh
+        "gpu_launches": (2 * len(steps) + 5 * n_anchor if runner.pulsecol else
+                         len(steps) + n_anchor * launches_per_anchor(
+                             w.bs, runner.att.sharded, runner.att.fused,
+                             runner.att.lists is not None)),
         "clocks": sampler.summary(),
     }
     if rank == 0:

@@ -29,7 +29,8 @@ EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspac
            "sdl_mask_budget_scoped", "sdl_select_workspace_bytes_scoped", "sdl_select_mask_scoped",
            "sdl_block_scores", "sdl_select_mask", "sdl_select_mask_noalloc", "sdl_sparse_attn",
            "sdl_tile_plan", "sdl_sparse_attn_planned", "sdl_tile_order",
-           "sdl_sparse_attn_scheduled", "sdl_dense_attn",
+           "sdl_sparse_attn_scheduled", "sdl_tile_lists_bytes", "sdl_tile_lists",
+           "sdl_sparse_attn_listed", "sdl_dense_attn",
            "sdl_anchor_workspace_bytes", "sdl_anchor_refresh",
            "sdl_col_budget", "sdl_col_scores_workspace_bytes", "sdl_col_scores",
            "sdl_col_select", "sdl_col_gather", "sdl_col_sparse_attn",
@@ -89,6 +90,10 @@ def _lib():
         L.sdl_sparse_attn_planned.argtypes = [P, P, P, SP, P, P, P, F, P, P, P]
         L.sdl_tile_order.argtypes = [P, P, SP, P, P]
         L.sdl_sparse_attn_scheduled.argtypes = [P, P, P, SP, P, P, P, P, F, P, P, P]
+        L.sdl_tile_lists_bytes.argtypes = [SP]
+        L.sdl_tile_lists_bytes.restype = ctypes.c_size_t
+        L.sdl_tile_lists.argtypes = [P, P, P, P, SP, P, ctypes.c_size_t, P]
+        L.sdl_sparse_attn_listed.argtypes = [P, P, P, SP, P, F, P, P, P]
         L.sdl_dense_attn.argtypes = [P, P, P, SP, F, P, P, P]
         L.sdl_col_budget.argtypes = [SP, D]
         L.sdl_col_budget.restype = I64
@@ -124,6 +129,7 @@ def _lib():
                   "sdl_select_shard_finish",
                   "sdl_sparse_attn", "sdl_tile_plan",
                   "sdl_sparse_attn_planned", "sdl_tile_order", "sdl_sparse_attn_scheduled",
+                  "sdl_tile_lists", "sdl_sparse_attn_listed",
                   "sdl_dense_attn",
                   "sdl_last_device_status", "sdl_last_cuda_error"):
             getattr(L, f).restype = ctypes.c_int
@@ -461,6 +467,34 @@ def tile_order(row_ptr, plan, B: int, H: int, L: int, block: int = 64, order=Non
     return order
 
 
+def tile_lists_bytes(B: int, H: int, L: int, block: int = 64) -> int:
+    """Bytes of the prebuilt tile lists of a shape (see ``sdl_tile_lists_bytes``)."""
+    s = Shape()
+    s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, H, L, 64, block, SDL_BF16
+    nbytes = int(_lib().sdl_tile_lists_bytes(ctypes.byref(s)))
+    if nbytes == 0:
+        raise SdlError(SDL_ERR_INVALID_ARG, "sdl_tile_lists_bytes")
+    return nbytes
+
+
+def tile_lists(row_ptr, col_idx, plan, order, B: int, H: int, L: int, block: int = 64,
+               lists=None, stream=None):
+    """uint8 buffer of the tiles' kept-block lists in take order (see ``sdl_tile_lists``);
+    ``plan`` and ``order`` may be None (adjacent pairs, plan order)."""
+    import torch
+    s = Shape()
+    s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, H, L, 64, block, SDL_BF16
+    if lists is None:
+        lists = torch.empty(tile_lists_bytes(B, H, L, block), dtype=torch.uint8,
+                            device=row_ptr.device)
+    _check(_lib().sdl_tile_lists(row_ptr.data_ptr(), col_idx.data_ptr(),
+                                 None if plan is None else plan.data_ptr(),
+                                 None if order is None else order.data_ptr(), ctypes.byref(s),
+                                 lists.data_ptr(), lists.numel(), _stream(stream)),
+           "sdl_tile_lists")
+    return lists
+
+
 def tile_plan(row_ptr, col_idx, B: int, H: int, L: int, block: int = 64, plan=None,
               stream=None):
     """int32 [B, H, ceil(nb/2), 2] tile plan for 64-token blocks (see ``sdl_tile_plan``)."""
@@ -476,17 +510,25 @@ def tile_plan(row_ptr, col_idx, B: int, H: int, L: int, block: int = 64, plan=No
 
 
 def sparse_attn(q, k, v, row_ptr, col_idx, block: int, scale: float = 0.0, out=None, lse=None,
-                want_lse: bool = False, plan=None, order=None, stream=None):
+                want_lse: bool = False, plan=None, order=None, lists=None, stream=None):
     """O like q (and LSE fp32 [B,H,L] when asked) over the kept blocks; ``plan`` is an
     optional tile plan from :func:`tile_plan` (results equal up to fp32 summation order),
-    ``order`` the order of taking its tiles from :func:`tile_order` (same bits)."""
+    ``order`` the order of taking its tiles from :func:`tile_order` (same bits), ``lists``
+    the tiles' prebuilt lists from :func:`tile_lists` (used instead of the CSR, same bits
+    as the plan and order they were built from)."""
     import torch
     if out is None:
         out = torch.empty_like(q)
     s = make_shape(q, k, block, v, out)
     if lse is None and want_lse:
         lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
-    if plan is not None and order is not None:
+    if lists is not None:
+        _check(_lib().sdl_sparse_attn_listed(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                             ctypes.byref(s), lists.data_ptr(), float(scale),
+                                             out.data_ptr(),
+                                             None if lse is None else lse.data_ptr(),
+                                             _stream(stream)), "sdl_sparse_attn_listed")
+    elif plan is not None and order is not None:
         _check(_lib().sdl_sparse_attn_scheduled(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                                 ctypes.byref(s), row_ptr.data_ptr(),
                                                 col_idx.data_ptr(), plan.data_ptr(),

@@ -101,7 +101,7 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, const sdl_shape& s, int
 sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_shape* shape,
                        const int32_t* row_ptr, const int32_t* col_idx, const int32_t* plan,
                        float scale, void* o, float* lse, void* stream, int Lk = 0,
-                       const int32_t* order = nullptr) {
+                       const int32_t* order = nullptr, const int32_t* lists = nullptr) {
   sdl_status e = check_shape(shape);
   if (e) return e;
   const sdl_shape& s = *shape;
@@ -123,6 +123,7 @@ sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_sh
   a.col_idx = col_idx;
   a.plan = (row_ptr && s.block == 64) ? plan : nullptr;
   a.order = a.plan ? order : nullptr;
+  a.lists = lists;
   a.B = s.B;
   a.H = s.H;
   a.Hkv = s.H_kv;
@@ -568,6 +569,54 @@ sdl_status sdl_sparse_attn_scheduled(const void* q, const void* k, const void* v
                                      void* stream) {
   if (!row_ptr || !col_idx || !plan || !order) return SDL_ERR_INVALID_ARG;
   return attn_common(q, k, v, shape, row_ptr, col_idx, plan, scale, o, lse, stream, 0, order);
+}
+
+size_t sdl_tile_lists_bytes(const sdl_shape* shape) {
+  if (check_shape(shape) != SDL_OK) return 0;
+  const int64_t n_items = (int64_t)shape->B * shape->H * ((shape->L + 127) / 128);
+  return tile_lists_bytes(n_items, shape->L);
+}
+
+sdl_status sdl_tile_lists(const int32_t* row_ptr, const int32_t* col_idx, const int32_t* plan,
+                          const int32_t* order, const sdl_shape* shape, void* lists,
+                          size_t lists_bytes, void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  if (!row_ptr || !col_idx || !lists || !aligned16(lists)) return SDL_ERR_INVALID_ARG;
+  if (shape->block != 64) return SDL_ERR_UNSUPPORTED;
+  if (lists_bytes < sdl_tile_lists_bytes(shape)) return SDL_ERR_WORKSPACE;
+  int* status = device_status_ptr();
+  if (!status) return SDL_ERR_CUDA;
+  AttnArgs a{};
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.plan = plan;
+  a.order = order;
+  a.lists = nullptr;
+  a.B = shape->B;
+  a.H = shape->H;
+  a.Hkv = shape->H_kv;
+  a.L = shape->L;
+  a.d = shape->d;
+  a.block = shape->block;
+  a.nb = shape->L / shape->block;
+  a.Lk = shape->L;
+  a.status = status;
+  const cudaError_t ce =
+      launch_tile_lists(a, static_cast<int32_t*>(lists), static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_sparse_attn_listed(const void* q, const void* k, const void* v,
+                                  const sdl_shape* shape, const void* lists, float scale, void* o,
+                                  float* lse, void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  if (!lists || !aligned16(lists)) return SDL_ERR_INVALID_ARG;
+  if (shape->block != 64 || shape->dtype != SDL_BF16) return SDL_ERR_UNSUPPORTED;
+  return attn_common(q, k, v, shape, nullptr, nullptr, nullptr, scale, o, lse, stream, 0, nullptr,
+                     static_cast<const int32_t*>(lists));
 }
 
 sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,

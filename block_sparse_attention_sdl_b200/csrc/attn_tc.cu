@@ -147,9 +147,99 @@ __device__ __forceinline__ void write_empty_tile(const AttnArgs& a, int b, int h
   }
 }
 
+// The tile of `item`: batch element, head and first tokens of its two 64-row
+// halves (L: half unused), from the plan for 64-token blocks, else adjacent.
+__device__ __forceinline__ void tile_of(const AttnArgs& a, int item, int n_qt, int& b, int& h,
+                                        int& t0, int& t1) {
+  b = item / (a.H * n_qt);
+  h = (item / n_qt) % a.H;
+  if (a.plan != nullptr) {
+    // the tile's two query blocks from the plan (64-token blocks)
+    const int qb0 = a.plan[2 * (int64_t)item], qb1 = a.plan[2 * (int64_t)item + 1];
+    if (qb0 >= a.nb || qb0 < -1 || qb1 >= a.nb || qb1 < -1) atomicOr(a.status, kDevBadMask);
+    t0 = (qb0 >= 0 && qb0 < a.nb) ? qb0 * 64 : a.L;
+    t1 = (qb1 >= 0 && qb1 < a.nb) ? qb1 * 64 : a.L;
+  } else {
+    t0 = (item % n_qt) * kBM;
+    t1 = t0 + 64 < a.L ? t0 + 64 : a.L;
+  }
+}
+
+// The kept 64-token key sub-blocks of a tile's two query halves, as bitmaps
+// in `bmask` (all key sub-blocks without a mask), listed in ascending order
+// with their keep bits into `ent` (shared or global memory); all lanes of one
+// warp.  Returns the list's length.
+__device__ int union_list(const AttnArgs& a, int b, int h, int t0, int t1,
+                          uint32_t (*bmask)[kMaxSub / 32], uint16_t* ent, int lane) {
+  const int nsub = a.Lk / kSubBlock;
+  for (int w = lane; w < kMaxSub / 32; w += 32) bmask[0][w] = bmask[1][w] = 0;
+  __syncwarp();
+  if (a.row_ptr == nullptr) {
+    for (int s = lane; s < nsub; s += 32) {
+      if (t0 < a.L) atomicOr(&bmask[0][s / 32], 1u << (s % 32));
+      if (t1 < a.L) atomicOr(&bmask[1][s / 32], 1u << (s % 32));
+    }
+  } else {
+    const int per = a.block / kSubBlock;  // sub-blocks per block: 1 or 2
+    const int rows_in_tile = a.block == 64 ? 2 : 1;
+    for (int rr = 0; rr < rows_in_tile; ++rr) {
+      const int tr = rr ? t1 : t0;
+      if (tr >= a.L) continue;
+      const int i = tr / a.block;
+      const int64_t r = ((int64_t)b * a.H + h) * a.nb + i;
+      const int beg = a.row_ptr[r], end = a.row_ptr[r + 1];
+      for (int x = beg + lane; x < end; x += 32) {
+        const int jb = a.col_idx[x];
+        const bool bad_range = jb < 0 || jb >= a.nb;
+        if (bad_range || (x > beg && a.col_idx[x - 1] >= jb)) atomicOr(a.status, kDevBadMask);
+        if (bad_range) continue;
+        for (int u = 0; u < per; ++u) {
+          const int s = jb * per + u;
+          if (a.block == 64) {
+            atomicOr(&bmask[rr][s / 32], 1u << (s % 32));
+          } else {
+            atomicOr(&bmask[0][s / 32], 1u << (s % 32));
+            atomicOr(&bmask[1][s / 32], 1u << (s % 32));
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  // ascending union with per-half keep bits: lane w handles bitmap word w
+  const uint32_t w0 = bmask[0][lane], w1 = bmask[1][lane];
+  const uint32_t wu = w0 | w1;
+  const int c = __popc(wu);
+  int incl = c;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int n_ent = __shfl_sync(0xffffffffu, incl, 31);
+  int pos = incl - c;
+  for (uint32_t mb = wu; mb; mb &= mb - 1) {
+    const int bit = __ffs(mb) - 1;
+    const uint32_t keep = ((w0 >> bit) & 1u) | (((w1 >> bit) & 1u) << 1);
+    ent[pos++] = (uint16_t)((uint32_t)(lane * 32 + bit) | (keep << kKeepShift));
+  }
+  __syncwarp();
+  return n_ent;
+}
+
+// Prebuilt tile lists (sdl_tile_lists): per position r of the take order a
+// record of 8 int32 {item, n_ent, t0, t1, 0, 0, 0, 0}, then per position
+// `cap` 16-bit entries (the union list, as in a list slot).
+constexpr int kListRecInts = 8;
+__host__ __device__ inline int lists_cap(int Lk) { return ((Lk / kSubBlock) + 7) / 8 * 8; }
+__host__ __device__ inline size_t lists_bytes(int64_t n_items, int Lk) {
+  return (size_t)n_items * (kListRecInts * 4 + 2 * (size_t)lists_cap(Lk));
+}
+
 // Takes items until a non-empty one and writes its union list into S (all
 // lanes of one warp; lane 0 writes the header).  Returns false once the
-// launch's items are used up (S then holds the end marker).
+// launch's items are used up (S then holds the end marker).  With prebuilt
+// lists the r-th item taken is record r, copied; else the r-th is order[r]
+// (or r) and its list is built here.
 template <int D>
 __device__ bool build_item(const AttnArgs& a, const CUtensorMap* tmq, Slot& S,
                            uint32_t (*bmask)[kMaxSub / 32], int sched_slot, int n_items, int n_qt,
@@ -160,85 +250,52 @@ __device__ bool build_item(const AttnArgs& a, const CUtensorMap* tmq, Slot& S,
     if (lane == 0) taken = atomicAdd(&g_sched[sched_slot].next, 1u);
     taken = __shfl_sync(0xffffffffu, taken, 0);
     if (taken >= (unsigned)n_items) break;
-    int item = (int)taken;
-    if (a.order != nullptr) {
-      // costliest tiles first (the order is a permutation of the items)
-      const int o = a.order[item];
-      if (o < 0 || o >= n_items) {
+    int item = (int)taken, n_ent = 0, b, h, t0, t1;
+    if (a.lists != nullptr) {
+      const int4 rec = *reinterpret_cast<const int4*>(a.lists + (int64_t)taken * kListRecInts);
+      item = rec.x;
+      n_ent = rec.y;
+      if (item < 0 || item >= n_items || n_ent < 0 || n_ent > nsub) {
         if (lane == 0) atomicOr(a.status, kDevBadMask);
         continue;
       }
-      item = o;
-    }
-    const int b = item / (a.H * n_qt);
-    const int h = (item / n_qt) % a.H;
-    int t0, t1;
-    if (a.plan != nullptr) {
-      // the tile's two query blocks from the plan (64-token blocks)
-      const int qb0 = a.plan[2 * (int64_t)item], qb1 = a.plan[2 * (int64_t)item + 1];
-      if (qb0 >= a.nb || qb0 < -1 || qb1 >= a.nb || qb1 < -1) atomicOr(a.status, kDevBadMask);
-      t0 = (qb0 >= 0 && qb0 < a.nb) ? qb0 * 64 : a.L;
-      t1 = (qb1 >= 0 && qb1 < a.nb) ? qb1 * 64 : a.L;
-    } else {
-      t0 = (item % n_qt) * kBM;
-      t1 = t0 + 64 < a.L ? t0 + 64 : a.L;
-    }
-    // kept 64-token key sub-blocks of the two query halves, as bitmaps
-    for (int w = lane; w < kMaxSub / 32; w += 32) bmask[0][w] = bmask[1][w] = 0;
-    __syncwarp();
-    if (a.row_ptr == nullptr) {
-      for (int s = lane; s < nsub; s += 32) {
-        if (t0 < a.L) atomicOr(&bmask[0][s / 32], 1u << (s % 32));
-        if (t1 < a.L) atomicOr(&bmask[1][s / 32], 1u << (s % 32));
+      b = item / (a.H * n_qt);
+      h = (item / n_qt) % a.H;
+      t0 = rec.z;
+      t1 = rec.w;
+      if (t0 < 0 || t0 > a.L || t1 < 0 || t1 > a.L) {
+        if (lane == 0) atomicOr(a.status, kDevBadMask);
+        continue;
       }
-    } else {
-      const int per = a.block / kSubBlock;  // sub-blocks per block: 1 or 2
-      const int rows_in_tile = a.block == 64 ? 2 : 1;
-      for (int rr = 0; rr < rows_in_tile; ++rr) {
-        const int tr = rr ? t1 : t0;
-        if (tr >= a.L) continue;
-        const int i = tr / a.block;
-        const int64_t r = ((int64_t)b * a.H + h) * a.nb + i;
-        const int beg = a.row_ptr[r], end = a.row_ptr[r + 1];
-        for (int x = beg + lane; x < end; x += 32) {
-          const int jb = a.col_idx[x];
-          const bool bad_range = jb < 0 || jb >= a.nb;
-          if (bad_range || (x > beg && a.col_idx[x - 1] >= jb)) atomicOr(a.status, kDevBadMask);
-          if (bad_range) continue;
-          for (int u = 0; u < per; ++u) {
-            const int s = jb * per + u;
-            if (a.block == 64) {
-              atomicOr(&bmask[rr][s / 32], 1u << (s % 32));
-            } else {
-              atomicOr(&bmask[0][s / 32], 1u << (s % 32));
-              atomicOr(&bmask[1][s / 32], 1u << (s % 32));
-            }
-          }
+      const uint16_t* src = reinterpret_cast<const uint16_t*>(a.lists + (int64_t)n_items *
+                                                                            kListRecInts) +
+                            (int64_t)taken * lists_cap(a.Lk);
+      for (int x = lane; x < n_ent; x += 32) {
+        uint16_t e = src[x];
+        if ((int)(e & kSubMask) >= nsub) {
+          atomicOr(a.status, kDevBadMask);
+          e = 0;
         }
+        S.ent[x] = e;
       }
+      __syncwarp();
+    } else {
+      if (a.order != nullptr) {
+        // costliest tiles first (the order is a permutation of the items)
+        const int o = a.order[item];
+        if (o < 0 || o >= n_items) {
+          if (lane == 0) atomicOr(a.status, kDevBadMask);
+          continue;
+        }
+        item = o;
+      }
+      tile_of(a, item, n_qt, b, h, t0, t1);
+      n_ent = union_list(a, b, h, t0, t1, bmask, S.ent, lane);
     }
-    __syncwarp();
-    // ascending union with per-half keep bits: lane w handles bitmap word w
-    const uint32_t w0 = bmask[0][lane], w1 = bmask[1][lane];
-    const uint32_t wu = w0 | w1;
-    const int c = __popc(wu);
-    int incl = c;
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const int n_ent = __shfl_sync(0xffffffffu, incl, 31);
-    __syncwarp();
     if (n_ent == 0) {
       write_empty_tile<D>(a, b, h, t0, t1, lane);
       __syncwarp();
       continue;
-    }
-    int pos = incl - c;
-    for (uint32_t mb = wu; mb; mb &= mb - 1) {
-      const int bit = __ffs(mb) - 1;
-      const uint32_t keep = ((w0 >> bit) & 1u) | (((w1 >> bit) & 1u) << 1);
-      S.ent[pos++] = (uint16_t)((uint32_t)(lane * 32 + bit) | (keep << kKeepShift));
     }
     if (lane == 0) {
       S.item = item;
@@ -261,6 +318,39 @@ __device__ bool build_item(const AttnArgs& a, const CUtensorMap* tmq, Slot& S,
   }
   __syncwarp();
   return false;
+}
+
+// One warp per position r of the take order: record r of the prebuilt lists
+// (the tile order[r], or r, and its union list).
+constexpr int kListWarps = 8;
+__global__ void __launch_bounds__(kListWarps * 32) tile_lists_kernel(AttnArgs a, int32_t* lists) {
+  __shared__ uint32_t bm[kListWarps][2][kMaxSub / 32];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_qt = (a.L + kBM - 1) / kBM;
+  const int n_items = a.B * a.H * n_qt;
+  const int r = blockIdx.x * kListWarps + warp;
+  if (r >= n_items) return;
+  int item = r;
+  if (a.order != nullptr) {
+    item = a.order[r];
+    if (item < 0 || item >= n_items) {
+      if (lane == 0) {
+        atomicOr(a.status, kDevBadMask);
+        *reinterpret_cast<int4*>(lists + (int64_t)r * kListRecInts) = make_int4(-1, 0, 0, 0);
+      }
+      return;
+    }
+  }
+  int b, h, t0, t1;
+  tile_of(a, item, n_qt, b, h, t0, t1);
+  uint16_t* ent = reinterpret_cast<uint16_t*>(lists + (int64_t)n_items * kListRecInts) +
+                  (int64_t)r * lists_cap(a.Lk);
+  const int n_ent = union_list(a, b, h, t0, t1, bm[warp], ent, lane);
+  if (lane == 0) {
+    int4* rec = reinterpret_cast<int4*>(lists + (int64_t)r * kListRecInts);
+    rec[0] = make_int4(item, n_ent, t0, t1);
+    rec[1] = make_int4(0, 0, 0, 0);
+  }
 }
 
 template <int D, bool kLse>
@@ -705,6 +795,15 @@ cudaError_t launch_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMa
 }
 
 }  // namespace
+
+size_t tile_lists_bytes(int64_t n_items, int Lk) { return lists_bytes(n_items, Lk); }
+
+cudaError_t launch_tile_lists(const AttnArgs& a, int32_t* lists, cudaStream_t st) {
+  const int64_t n_items = (int64_t)a.B * a.H * ((a.L + kBM - 1) / kBM);
+  tile_lists_kernel<<<(unsigned)((n_items + kListWarps - 1) / kListWarps), kListWarps * 32, 0,
+                      st>>>(a, lists);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, const CUtensorMap* to, cudaStream_t st) {

@@ -32,6 +32,7 @@ struct AttnArgs {
   const int32_t* col_idx;
   const int32_t* plan;     // tile plan for 64-token blocks (null: adjacent pairs)
   const int32_t* order;    // order of taking the plan's tiles (null: plan order)
+  const int32_t* lists;    // prebuilt tile lists in take order (null: built in the kernel)
   int B, H, Hkv, L, d, block, nb;
   int Lk;  // key (and value) tokens: L, or the gathered columns of column-sparse attention
   int64_t qs[3], ks[3], vs[3], os[3];
@@ -70,6 +71,8 @@ cudaError_t launch_col_select(const float* S, int BH, int L, int Lc, int32_t* co
                               cudaStream_t st);
 cudaError_t launch_col_gather(const void* k, const void* v, const sdl_shape& s,
                               const int32_t* cols, int Lc, void* kc, void* vc, cudaStream_t st);
+size_t tile_lists_bytes(int64_t n_items, int Lk);
+cudaError_t launch_tile_lists(const AttnArgs& a, int32_t* lists, cudaStream_t st);
 cudaError_t launch_tile_order(const int32_t* row_ptr, const int32_t* plan, int B, int H, int nb,
                               int32_t* order, cudaStream_t st);
 // self-check of the bounded waits (selfcheck.cu)

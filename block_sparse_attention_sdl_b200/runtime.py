@@ -30,8 +30,8 @@ import torch
 from . import (anchor_refresh, anchor_workspace_bytes, block_scores, col_budget, col_gather,
                col_scores, col_scores_workspace_bytes, col_select, col_sparse_attn, dense_attn,
                make_shape, mask_budget, scores_workspace_bytes, select_mask,
-               select_shard_capacity, select_workspace_bytes, sparse_attn, tile_order,
-               tile_plan)
+               select_shard_capacity, select_workspace_bytes, sparse_attn, tile_lists,
+               tile_lists_bytes, tile_order, tile_plan)
 from .sharded import CudaStages, select_mask_sharded, torch_collectives
 
 
@@ -106,6 +106,11 @@ class StepSparseAttention:
         # the plan's tiles, costliest first (the attention kernel's take order)
         self.order = (torch.empty(B * H * ((self.nb + 1) // 2), dtype=torch.int32, device=dev)
                       if block == 64 else None)
+        # the tiles' kept-block lists in that order (bf16: the tensor-core kernel reads them
+        # instead of building each tile's list from the CSR when it takes the tile)
+        self.lists = (torch.empty(tile_lists_bytes(B, H, L, block), dtype=torch.uint8,
+                                  device=dev)
+                      if block == 64 and dtype == torch.bfloat16 else None)
         self.mask_step = None  # anchor step whose mask is current
         # the head-adaptive budget on one device: scores and selection in one launch
         self.fused = not self.sharded and not self.per_head
@@ -127,6 +132,9 @@ class StepSparseAttention:
                       plan=self.plan, stream=stream)
             tile_order(self.row_ptr, self.plan, self.B, self.H, self.L, self.block,
                        order=self.order, stream=stream)
+        if self.lists is not None:
+            tile_lists(self.row_ptr, self.col_idx, self.plan, self.order, self.B, self.H, self.L,
+                       self.block, lists=self.lists, stream=stream)
         self.mask_step = step
 
     def select(self, stream=None):
@@ -155,7 +163,7 @@ class StepSparseAttention:
         if is_anchor(step, self.anchor_every, self.dense_steps) or self.mask_step is None:
             self.refresh(q, k, anchor_of(step, self.anchor_every, self.dense_steps), stream)
         return sparse_attn(q, k, v, self.row_ptr, self.col_idx, self.block, out=out, lse=lse,
-                           plan=self.plan, order=self.order, stream=stream)
+                           plan=self.plan, order=self.order, lists=self.lists, stream=stream)
 
 
 class ColSparseAttention:

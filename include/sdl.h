@@ -299,6 +299,32 @@ sdl_status sdl_sparse_attn_scheduled(const void* q, const void* k, const void* v
                                      const int32_t* order, float scale, void* o, float* lse,
                                      void* stream);
 
+/* Tile lists built once per mask (a scheduling aid, like the plan and the
+ * order): for every position r of `order` (NULL: the plan's tile order) the
+ * tile's identity, its two query blocks' first tokens and the ascending union
+ * of their kept 64-token key blocks with a keep bit per query block -- exactly
+ * the list the attention kernel would otherwise build when it takes the tile.
+ * `lists` (16-byte aligned, caller-owned) must hold sdl_tile_lists_bytes
+ * bytes (else SDL_ERR_WORKSPACE): per position a record of 8 int32 {tile,
+ * list length, first token of each half (L: half unused), 0, 0, 0, 0}, then
+ * per position a row of 16-bit entries (key block | keep bits << 14), rows
+ * padded to a multiple of 8 entries.  64-token blocks only
+ * (SDL_ERR_UNSUPPORTED otherwise); plan entries outside the block range are
+ * reported as SDL_ERR_BAD_MASK, as in the attention calls.
+ * sdl_sparse_attn_listed: sdl_sparse_attn_scheduled reading the tiles and
+ * their lists from `lists` (taken in record order) instead of building each
+ * list from the CSR when the tile is taken; results are those of
+ * sdl_sparse_attn_scheduled with the same plan and order, bit for bit.
+ * Records or entries out of range are skipped or zeroed and reported as
+ * SDL_ERR_BAD_MASK.  bf16 only. */
+size_t sdl_tile_lists_bytes(const sdl_shape* shape);
+sdl_status sdl_tile_lists(const int32_t* row_ptr, const int32_t* col_idx, const int32_t* plan,
+                          const int32_t* order, const sdl_shape* shape, void* lists,
+                          size_t lists_bytes, void* stream);
+sdl_status sdl_sparse_attn_listed(const void* q, const void* k, const void* v,
+                                  const sdl_shape* shape, const void* lists, float scale, void* o,
+                                  float* lse, void* stream);
+
 /* Dense bidirectional attention, the baseline of the same abstract: the
  * sparse call with every block of every row kept. */
 sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,

@@ -489,3 +489,74 @@ def test_bounded_wait_times_out_and_the_context_survives():
     assert sdl.last_device_status() == sdl.SDL_OK
     Ow, _ = oracle.attention(host["q"], host["k"], host["v"], 64)
     check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, "bf16")
+
+
+@pytest.mark.parametrize("B,L,H,Hkv,density", [(1, 1024, 4, 2, 0.3), (2, 1024, 4, 2, 0.2),
+                                               (1, 576, 3, 1, 0.5), (1, 4096, 8, 8, 0.12)])
+def test_listed_attention_equals_scheduled(B, L, H, Hkv, density):
+    """Tiles and lists prebuilt once (sdl_tile_lists) give the scheduled path's result
+    bit for bit, LSE included, and the records hold the tiles in take order with the
+    ascending union of their two query blocks' kept blocks."""
+    w = synth.small_workload(B=B, L=L, H=H, H_kv=Hkv, d=128, bs=64)
+    _, dev = _inputs(w)
+    nb = L // 64
+    rng = np.random.default_rng(B * L + H)
+    mask = _random_mask(B, H, nb, density, rng)
+    rp, ci = _mask_to_csr(mask)
+    plan = sdl.tile_plan(rp, ci, B, H, L, 64)
+    order = sdl.tile_order(rp, plan, B, H, L, 64)
+    lists = sdl.tile_lists(rp, ci, plan, order, B, H, L, 64)
+    O1, l1 = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, want_lse=True, plan=plan,
+                             order=order)
+    O2, l2 = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, want_lse=True,
+                             lists=lists)
+    assert sdl.last_device_status() == sdl.SDL_OK
+    assert torch.equal(O1, O2) and torch.equal(l1, l2)
+    # the records, rebuilt on the host
+    n_qt = (nb + 1) // 2
+    n = B * H * n_qt
+    cap = (nb + 7) // 8 * 8
+    raw = lists.cpu().numpy()
+    rec = raw[:n * 32].view(np.int32).reshape(n, 8)
+    ent = raw[n * 32:n * 32 + n * cap * 2].view(np.uint16).reshape(n, cap)
+    o = order.cpu().numpy()
+    pl = plan.cpu().numpy().reshape(-1, 2)
+    assert np.array_equal(rec[:, 0], o)
+    for r in range(n):
+        item = o[r]
+        bh = item // n_qt
+        b, h = bh // H, bh % H
+        rows = [qb for qb in pl[item]]
+        want_t = [qb * 64 if qb >= 0 else L for qb in rows]
+        assert list(rec[r, 2:4]) == want_t
+        keep = np.zeros((2, nb), bool)
+        for s, qb in enumerate(rows):
+            if qb >= 0:
+                keep[s] = mask[b, h, qb].astype(bool)
+        union = np.nonzero(keep[0] | keep[1])[0]
+        assert rec[r, 1] == len(union)
+        e = ent[r, :len(union)]
+        assert np.array_equal(e & 0x3FFF, union)
+        assert np.array_equal((e >> 14) & 1, keep[0][union]) and \
+            np.array_equal((e >> 15) & 1, keep[1][union])
+
+
+def test_listed_attention_adjacent_pairs_and_bad_record():
+    """Lists built without a plan or order pair adjacent query blocks in tile order,
+    which is what the plain call does; a record naming no tile is reported."""
+    B, L, H, Hkv = 1, 1024, 4, 2
+    w = synth.small_workload(B=B, L=L, H=H, H_kv=Hkv, d=128, bs=64)
+    _, dev = _inputs(w)
+    nb = L // 64
+    mask = _random_mask(B, H, nb, 0.3, np.random.default_rng(5))
+    rp, ci = _mask_to_csr(mask)
+    lists = sdl.tile_lists(rp, ci, None, None, B, H, L, 64)
+    O1 = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64)
+    O2 = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, lists=lists)
+    assert sdl.last_device_status() == sdl.SDL_OK
+    assert torch.equal(O1, O2)
+    bad = lists.clone()
+    bad[:4] = torch.tensor(np.array([1 << 20], np.int32).view(np.uint8), device=bad.device)
+    sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, lists=bad)
+    assert sdl.last_device_status() == sdl.SDL_ERR_BAD_MASK
+    assert sdl.last_device_status() == sdl.SDL_OK
