@@ -387,8 +387,8 @@ cudaError_t launch_col_scores(const void* k, const sdl_shape& s, float scale, co
   const size_t smem1 = col_smem_bytes(s.d), smem2 = smem1 + kColSumExtra;
   const int ngroups = col_groups(s.L);
   const dim3 g1(ngroups, (c.nb + kGR - 1) / kGR, s.B * s.H), g2((s.L + kGK - 1) / kGK, s.B * s.H);
-  static bool attr_set = false;  // per function; the size needed is at most this
-  if (!attr_set) {
+  static std::atomic<bool> attr_set[64];  // per device; the size needed is at most this
+  cudaError_t ae = once_per_device(attr_set, [] {
     const int most = (int)(col_smem_bytes(128) + kColSumExtra);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(col_stats_kernel<__nv_bfloat16>,
@@ -400,8 +400,9 @@ cudaError_t launch_col_scores(const void* k, const sdl_shape& s, float scale, co
         (e = cudaFuncSetAttribute(col_sum_kernel<float>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, most)))
       return e;
-    attr_set = true;
-  }
+    return cudaSuccess;
+  });
+  if (ae != cudaSuccess) return ae;
   const int rows = s.B * s.H * c.nb;
   if (s.dtype == SDL_BF16) {
     col_stats_kernel<__nv_bfloat16><<<g1, kGT, smem1, st>>>(

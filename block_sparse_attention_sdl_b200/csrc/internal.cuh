@@ -1,5 +1,6 @@
 // Declarations shared by the translation units of libsdl.
 #pragma once
+#include <atomic>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -21,6 +22,20 @@ int* device_status_ptr();  // address of the library's device status word
 // in the low 16 bits, and in bits 16..17 which halves (query rows 0..63,
 // 64..127) of a 128-row query tile keep it.
 constexpr int kSubBlock = 64;
+
+// Runs `set` (setting a kernel's attributes) once per device for the static
+// flags `done` of one call site; a failure is returned and retried next time.
+template <typename F>
+inline cudaError_t once_per_device(std::atomic<bool> (&done)[64], F&& set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (done[dev].load()) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess) done[dev].store(true);
+  return e;
+}
 
 struct AttnArgs {
   const void* q;

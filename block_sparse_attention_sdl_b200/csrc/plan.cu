@@ -123,13 +123,12 @@ cudaError_t launch_plan(const int32_t* row_ptr, const int32_t* col_idx, int B, i
     return cudaGetLastError();
   }
   const size_t smem = PlanSmem::bytes(nb);
-  static bool attr_set = false;  // the attribute is per function; the maximum is constant
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)PlanSmem::bytes(kPlanMaxNb));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<bool> attr_set[64];  // per device; the maximum is constant
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)PlanSmem::bytes(kPlanMaxNb));
+  });
+  if (e != cudaSuccess) return e;
   plan_kernel<<<dim3(H, B), kPlanThreads, smem, st>>>(row_ptr, col_idx, H, nb, n_qt, plan);
   return cudaGetLastError();
 }
@@ -138,13 +137,12 @@ cudaError_t launch_tile_order(const int32_t* row_ptr, const int32_t* plan, int B
                               int32_t* order, cudaStream_t st) {
   const int n = B * H * ((nb + 1) / 2);
   const size_t smem = n <= kOrderCached ? sizeof(uint16_t) * (size_t)n : 0;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(sizeof(uint16_t) * kOrderCached));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<bool> attr_set[64];  // per device
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(sizeof(uint16_t) * kOrderCached));
+  });
+  if (e != cudaSuccess) return e;
   order_kernel<<<1, kOrderThreads, smem, st>>>(row_ptr, plan, B * H, nb, (nb + 1) / 2, order);
   return cudaGetLastError();
 }

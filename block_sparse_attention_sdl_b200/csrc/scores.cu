@@ -63,13 +63,12 @@ cudaError_t launch_scores(const float* qbar, const float* kbar, const sdl_shape&
                           float* scores, cudaStream_t st) {
   const int nb = s.L / s.block;
   const size_t smem = score_smem_bytes(nb, s.d);
-  static bool attr_set = false;  // the attribute is per function; max size is constant
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<bool> attr_set[64];  // per device; the maximum size is constant
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                227 * 1024);
+  });
+  if (e != cudaSuccess) return e;
   dim3 grid((nb + kTI - 1) / kTI, s.H, s.B);
   score_kernel<<<grid, kScoreThreads, smem, st>>>(qbar, kbar, scores, s.H, s.H_kv, nb, s.d, scale);
   return cudaGetLastError();
