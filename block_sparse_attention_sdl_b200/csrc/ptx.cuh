@@ -135,8 +135,8 @@ __device__ __forceinline__ float exp2_poly(float x) {
 
 // ---------------------------------------------------------------------- TMA
 
-// 4-D tiled bulk tensor load into this CTA's shared memory; completion is
-// signalled on `bar` as transaction bytes.  No multicast.
+// 4-D tiled bulk tensor load into this CTA's own shared memory (no other CTA
+// receives it); completion is signalled on `bar` as transaction bytes.
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2, int c3) {
   asm volatile(
