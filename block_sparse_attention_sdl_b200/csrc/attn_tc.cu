@@ -10,9 +10,10 @@
 // counter, first come first served (tiles differ in cost by the length of
 // their kept lists).
 //
-//   warp 0        loads: takes items and builds the union list of an item's
-//                 two query blocks into a list slot (three slots, the next
-//                 item's list built while the current item runs); per item
+//   warp 0        loads: takes items and copies an item's prebuilt list
+//                 (tile_lists_kernel, run once per mask) or builds the union
+//                 list of its two query blocks into a list slot (three slots,
+//                 the next item's list while the current item runs); per item
 //                 its Q tile, per step its K and V sub-blocks by TMA
 //                 (128-byte-swizzled 64x64 boxes) into one K and one V stage.
 //                 Items whose lists are empty (only a caller's mask can have
