@@ -300,8 +300,9 @@ sdl_status sdl_sparse_attn_scheduled(const void* q, const void* k, const void* v
                                      void* stream);
 
 /* Tile lists built once per mask (a scheduling aid, like the plan and the
- * order): for every position r of `order` (NULL: the plan's tile order) the
- * tile's identity, its two query blocks' first tokens and the ascending union
+ * order): for every position r of `order` (NULL: the plan's tile order;
+ * `plan` NULL: adjacent query blocks paired) the tile's identity, its two
+ * query blocks' first tokens and the ascending union
  * of their kept 64-token key blocks with a keep bit per query block -- exactly
  * the list the attention kernel would otherwise build when it takes the tile.
  * `lists` (16-byte aligned, caller-owned) must hold sdl_tile_lists_bytes
@@ -316,7 +317,8 @@ sdl_status sdl_sparse_attn_scheduled(const void* q, const void* k, const void* v
  * list from the CSR when the tile is taken; results are those of
  * sdl_sparse_attn_scheduled with the same plan and order, bit for bit.
  * Records or entries out of range are skipped or zeroed and reported as
- * SDL_ERR_BAD_MASK.  bf16 only. */
+ * SDL_ERR_BAD_MASK.  bf16 only.  The lists depend on the mask, plan and
+ * order alone (not on Q, K, V): rebuild them whenever one of those changes. */
 size_t sdl_tile_lists_bytes(const sdl_shape* shape);
 sdl_status sdl_tile_lists(const int32_t* row_ptr, const int32_t* col_idx, const int32_t* plan,
                           const int32_t* order, const sdl_shape* shape, void* lists,
