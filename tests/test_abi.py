@@ -96,3 +96,61 @@ def test_status_strings():
     for code in range(8):
         assert lib.sdl_status_string(code)
     assert lib.sdl_last_cuda_error() == 0
+
+
+@pytest.mark.parametrize("B,H,Hkv,L", [(1, 32, 32, 8192), (2, 4, 4, 2112), (1, 28, 4, 16384),
+                                       (3, 2, 1, 64)])
+def test_tile_lists_size_follows_the_documented_layout(B, H, Hkv, L):
+    """Per position of the take order: a record of 8 int32, then a row of 16-bit
+    entries, one per 64-token key block, padded to a multiple of 8 entries."""
+    lib = sdl.lib()
+    shp = _shape(B=B, H=H, Hkv=Hkv, L=L)
+    n_items = B * H * -(-L // 128)          # 128-row tiles
+    row = -(-(L // 64) // 8) * 8
+    want = n_items * 8 * 4 + n_items * row * 2
+    assert lib.sdl_tile_lists_bytes(ctypes.byref(shp)) == want
+    assert sdl.tile_lists_bytes(B, H, L) == want
+    assert want % 16 == 0                   # every row starts 16-byte aligned
+    assert lib.sdl_tile_lists_bytes(ctypes.byref(_shape(block=96))) == 0
+
+
+def test_tile_lists_host_checks():
+    lib = sdl.lib()
+    P = ctypes.c_void_p
+    shp = _shape(H=2, Hkv=2, L=512)
+    need = lib.sdl_tile_lists_bytes(ctypes.byref(shp))
+    # refused before any CUDA call: null or misaligned buffers, 128-token
+    # blocks, too little room
+    rc = lib.sdl_tile_lists(P(16), P(16), None, None, ctypes.byref(shp), None, need, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+    rc = lib.sdl_tile_lists(P(16), P(16), None, None, ctypes.byref(shp), P(24), need, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+    rc = lib.sdl_tile_lists(None, P(16), None, None, ctypes.byref(shp), P(16), need, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+    rc = lib.sdl_tile_lists(P(16), P(16), None, None, ctypes.byref(_shape(H=2, Hkv=2, L=512,
+                                                                          block=128)),
+                            P(16), need, None)
+    assert rc == sdl.SDL_ERR_UNSUPPORTED
+    rc = lib.sdl_tile_lists(P(16), P(16), None, None, ctypes.byref(shp), P(16), need - 16, None)
+    assert rc == sdl.SDL_ERR_WORKSPACE
+    # the listed attention call: lists required, bf16 and 64-token blocks only
+    rc = lib.sdl_sparse_attn_listed(P(16), P(16), P(16), ctypes.byref(shp), None, 0.0, P(16),
+                                    None, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+    rc = lib.sdl_sparse_attn_listed(P(16), P(16), P(16), ctypes.byref(_shape(H=2, Hkv=2, L=512,
+                                                                             dtype=1)),
+                                    P(16), 0.0, P(16), None, None)
+    assert rc == sdl.SDL_ERR_UNSUPPORTED
+
+
+def test_col_scores_workspace_holds_the_block_means_and_row_statistics():
+    """The column scores need the block means of Q and K (as the block scores do)
+    and a (max, sum) pair per query-block row of every head."""
+    lib = sdl.lib()
+    for B, H, Hkv, L in ((1, 32, 32, 8192), (2, 28, 4, 16384), (1, 2, 2, 512)):
+        shp = _shape(B=B, H=H, Hkv=Hkv, L=L)
+        nb = L // 64
+        got = lib.sdl_col_scores_workspace_bytes(ctypes.byref(shp))
+        assert got >= sdl.scores_workspace_bytes(shp) + 8 * B * H * nb
+        assert got % 256 == 0
+    assert lib.sdl_col_scores_workspace_bytes(ctypes.byref(_shape(d=96))) == 0
