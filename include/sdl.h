@@ -317,7 +317,8 @@ sdl_status sdl_sparse_attn_scheduled(const void* q, const void* k, const void* v
  * list from the CSR when the tile is taken; results are those of
  * sdl_sparse_attn_scheduled with the same plan and order, bit for bit.
  * Records or entries out of range are skipped or zeroed and reported as
- * SDL_ERR_BAD_MASK.  bf16 only.  The lists depend on the mask, plan and
+ * SDL_ERR_BAD_MASK.  bf16 and 64-token blocks only (SDL_ERR_UNSUPPORTED
+ * otherwise).  The lists depend on the mask, plan and
  * order alone (not on Q, K, V): rebuild them whenever one of those changes. */
 size_t sdl_tile_lists_bytes(const sdl_shape* shape);
 sdl_status sdl_tile_lists(const int32_t* row_ptr, const int32_t* col_idx, const int32_t* plan,

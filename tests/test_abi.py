@@ -141,6 +141,10 @@ def test_tile_lists_host_checks():
                                                                              dtype=1)),
                                     P(16), 0.0, P(16), None, None)
     assert rc == sdl.SDL_ERR_UNSUPPORTED
+    rc = lib.sdl_sparse_attn_listed(P(16), P(16), P(16), ctypes.byref(_shape(H=2, Hkv=2, L=512,
+                                                                             block=128)),
+                                    P(16), 0.0, P(16), None, None)
+    assert rc == sdl.SDL_ERR_UNSUPPORTED
 
 
 def test_col_scores_workspace_holds_the_block_means_and_row_statistics():
