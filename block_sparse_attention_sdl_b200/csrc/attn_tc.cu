@@ -418,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     bool ended = false;
     int nq = 0;      // Q tiles loaded
     int g = 0;       // steps loaded (K and V stage phases)
+    int gk = 0, gv = 0;  // K and V copies issued (one ahead of g between a step's copies)
     // publishes the next list into its slot once the slot's item is done
     auto publish_next = [&]() -> bool {
       const int slot = built % kSlots;
@@ -465,6 +466,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               tma_load_4d(dst + c * Lay::kChunkRowsKV + s * kBox, &tmk, &bars.kfull, c * 64,
                           (s ? sub1 : sub0) * kSubBlock, kh, b);
         }
+        gk = g + 1;
         // the next item's list, while this one runs
         if (j == 0 && !ended && !(ok = publish_next())) break;
         // V of the step once the previous PV product has completed
@@ -479,14 +481,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               tma_load_4d(dst + c * Lay::kChunkRowsKV + s * kBox, &tmv, &bars.vfull, c * 64,
                           (s ? sub1 : sub0) * kSubBlock, kh, b);
         }
+        gv = g + 1;
       }
     }
     if (leader) {
       if (!ok) raise_timeout(&abort_sh, a.status);
-      // Drain: every copy issued above lands before the CTA exits.
+      // Drain: every copy issued above lands before the CTA exits.  The K and V
+      // copies are counted apart: a step left early has its K copy in flight.
       volatile int no_abort = 0;
-      if (g > 0 && !(mbar_wait(&bars.kfull, (g - 1) & 1, &no_abort, nullptr, kWaitLimitNs) &&
-                     mbar_wait(&bars.vfull, (g - 1) & 1, &no_abort, nullptr, kWaitLimitNs)))
+      if (gk > 0 && !mbar_wait(&bars.kfull, (gk - 1) & 1, &no_abort, nullptr, kWaitLimitNs))
+        atomicOr(a.status, kDevTimeout);
+      if (gv > 0 && !mbar_wait(&bars.vfull, (gv - 1) & 1, &no_abort, nullptr, kWaitLimitNs))
         atomicOr(a.status, kDevTimeout);
       if (nq > 0 && !mbar_wait(&bars.q_full, (nq - 1) & 1, &no_abort, nullptr, kWaitLimitNs))
         atomicOr(a.status, kDevTimeout);
