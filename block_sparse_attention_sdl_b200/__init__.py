@@ -490,7 +490,8 @@ def tile_lists(row_ptr, col_idx, plan, order, B: int, H: int, L: int, block: int
     _check(_lib().sdl_tile_lists(row_ptr.data_ptr(), col_idx.data_ptr(),
                                  None if plan is None else plan.data_ptr(),
                                  None if order is None else order.data_ptr(), ctypes.byref(s),
-                                 lists.data_ptr(), lists.numel(), _stream(stream)),
+                                 lists.data_ptr(), lists.numel() * lists.element_size(),
+                                 _stream(stream)),
            "sdl_tile_lists")
     return lists
 
@@ -523,6 +524,9 @@ def sparse_attn(q, k, v, row_ptr, col_idx, block: int, scale: float = 0.0, out=N
     if lse is None and want_lse:
         lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
     if lists is not None:
+        # the C call takes no size: a buffer built for a smaller shape is refused here
+        if lists.numel() * lists.element_size() < tile_lists_bytes(s.B, s.H, s.L, block):
+            raise SdlError(SDL_ERR_WORKSPACE, "sdl_sparse_attn_listed: lists too small")
         _check(_lib().sdl_sparse_attn_listed(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                              ctypes.byref(s), lists.data_ptr(), float(scale),
                                              out.data_ptr(),

@@ -158,3 +158,19 @@ def test_col_scores_workspace_holds_the_block_means_and_row_statistics():
         assert got >= sdl.scores_workspace_bytes(shp) + 8 * B * H * nb
         assert got % 256 == 0
     assert lib.sdl_col_scores_workspace_bytes(ctypes.byref(_shape(d=96))) == 0
+
+
+def test_binding_refuses_tile_lists_built_for_a_smaller_shape():
+    """The listed attention call takes no buffer size, so the binding checks it on
+    the host before the call (CPU tensors: nothing reaches the GPU)."""
+    torch = pytest.importorskip("torch")
+    B, L, H = 1, 1024, 4
+    q = torch.zeros((B, L, H, 128), dtype=torch.bfloat16)
+    small = torch.zeros(sdl.tile_lists_bytes(B, H, L // 2), dtype=torch.uint8)
+    with pytest.raises(sdl.SdlError) as e:
+        sdl.sparse_attn(q, q, q, None, None, 64, out=torch.empty_like(q), lists=small)
+    assert e.value.status == sdl.SDL_ERR_WORKSPACE
+    # the size counts bytes, whatever the buffer's element type
+    as_int32 = torch.zeros(sdl.tile_lists_bytes(B, H, L) // 4 - 1, dtype=torch.int32)
+    with pytest.raises(sdl.SdlError):
+        sdl.sparse_attn(q, q, q, None, None, 64, out=torch.empty_like(q), lists=as_int32)
