@@ -460,11 +460,22 @@ def tile_order(row_ptr, plan, B: int, H: int, L: int, block: int = 64, order=Non
     nb = L // block
     s = Shape()
     s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, H, L, 64, block, SDL_BF16
+    n_qt = (nb + 1) // 2
+    _need_i32(row_ptr, B * H * nb + 1, "tile_order row_ptr")
+    _need_i32(plan, B * H * n_qt * 2, "tile_order plan")
     if order is None:
-        order = torch.empty(B * H * ((nb + 1) // 2), dtype=torch.int32, device=plan.device)
+        order = torch.empty(B * H * n_qt, dtype=torch.int32, device=plan.device)
+    _need_i32(order, B * H * n_qt, "tile_order order")
     _check(_lib().sdl_tile_order(row_ptr.data_ptr(), plan.data_ptr(), ctypes.byref(s),
                                  order.data_ptr(), _stream(stream)), "sdl_tile_order")
     return order
+
+
+def _need_i32(t, n: int, what: str):
+    """Host check of an int32 index buffer that the C call reads without a size."""
+    import torch
+    if t is None or t.dtype != torch.int32 or t.numel() < n:
+        raise SdlError(SDL_ERR_INVALID_ARG, f"{what}: int32 with at least {n} elements needed")
 
 
 def tile_lists_bytes(B: int, H: int, L: int, block: int = 64) -> int:
@@ -484,6 +495,12 @@ def tile_lists(row_ptr, col_idx, plan, order, B: int, H: int, L: int, block: int
     import torch
     s = Shape()
     s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, H, L, 64, block, SDL_BF16
+    nb, n_qt = L // block, (L // block + 1) // 2
+    _need_i32(row_ptr, B * H * nb + 1, "tile_lists row_ptr")
+    if plan is not None:
+        _need_i32(plan, B * H * n_qt * 2, "tile_lists plan")
+    if order is not None:
+        _need_i32(order, B * H * n_qt, "tile_lists order")
     if lists is None:
         lists = torch.empty(tile_lists_bytes(B, H, L, block), dtype=torch.uint8,
                             device=row_ptr.device)
@@ -503,8 +520,10 @@ def tile_plan(row_ptr, col_idx, B: int, H: int, L: int, block: int = 64, plan=No
     nb = L // block
     s = Shape()
     s.B, s.H, s.H_kv, s.L, s.d, s.block, s.dtype = B, H, H, L, 64, block, SDL_BF16
+    _need_i32(row_ptr, B * H * nb + 1, "tile_plan row_ptr")
     if plan is None:
         plan = torch.empty((B, H, (nb + 1) // 2, 2), dtype=torch.int32, device=row_ptr.device)
+    _need_i32(plan, B * H * ((nb + 1) // 2) * 2, "tile_plan plan")
     _check(_lib().sdl_tile_plan(row_ptr.data_ptr(), col_idx.data_ptr(), ctypes.byref(s),
                                 plan.data_ptr(), _stream(stream)), "sdl_tile_plan")
     return plan
@@ -532,25 +551,34 @@ def sparse_attn(q, k, v, row_ptr, col_idx, block: int, scale: float = 0.0, out=N
                                              out.data_ptr(),
                                              None if lse is None else lse.data_ptr(),
                                              _stream(stream)), "sdl_sparse_attn_listed")
-    elif plan is not None and order is not None:
-        _check(_lib().sdl_sparse_attn_scheduled(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                                ctypes.byref(s), row_ptr.data_ptr(),
-                                                col_idx.data_ptr(), plan.data_ptr(),
-                                                order.data_ptr(), float(scale), out.data_ptr(),
-                                                None if lse is None else lse.data_ptr(),
-                                                _stream(stream)), "sdl_sparse_attn_scheduled")
-    elif plan is None:
-        _check(_lib().sdl_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(s),
-                                      row_ptr.data_ptr(), col_idx.data_ptr(), float(scale),
-                                      out.data_ptr(), None if lse is None else lse.data_ptr(),
-                                      _stream(stream)), "sdl_sparse_attn")
     else:
-        _check(_lib().sdl_sparse_attn_planned(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                              ctypes.byref(s), row_ptr.data_ptr(),
-                                              col_idx.data_ptr(), plan.data_ptr(), float(scale),
-                                              out.data_ptr(),
-                                              None if lse is None else lse.data_ptr(),
-                                              _stream(stream)), "sdl_sparse_attn_planned")
+        nb = s.L // block if block > 0 else 0
+        n_qt = (s.L + 127) // 128
+        _need_i32(row_ptr, s.B * s.H * nb + 1, "sparse_attn row_ptr")
+        _need_i32(col_idx, 0, "sparse_attn col_idx")
+        if plan is not None:
+            _need_i32(plan, s.B * s.H * n_qt * 2, "sparse_attn plan")
+        if order is not None:
+            _need_i32(order, s.B * s.H * n_qt, "sparse_attn order")
+        lse_p = None if lse is None else lse.data_ptr()
+        if plan is not None and order is not None:
+            _check(_lib().sdl_sparse_attn_scheduled(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                    ctypes.byref(s), row_ptr.data_ptr(),
+                                                    col_idx.data_ptr(), plan.data_ptr(),
+                                                    order.data_ptr(), float(scale),
+                                                    out.data_ptr(), lse_p, _stream(stream)),
+                   "sdl_sparse_attn_scheduled")
+        elif plan is None:
+            _check(_lib().sdl_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                          ctypes.byref(s), row_ptr.data_ptr(),
+                                          col_idx.data_ptr(), float(scale), out.data_ptr(),
+                                          lse_p, _stream(stream)), "sdl_sparse_attn")
+        else:
+            _check(_lib().sdl_sparse_attn_planned(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                  ctypes.byref(s), row_ptr.data_ptr(),
+                                                  col_idx.data_ptr(), plan.data_ptr(),
+                                                  float(scale), out.data_ptr(), lse_p,
+                                                  _stream(stream)), "sdl_sparse_attn_planned")
     return (out, lse) if want_lse or lse is not None else out
 
 

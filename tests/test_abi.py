@@ -174,3 +174,43 @@ def test_binding_refuses_tile_lists_built_for_a_smaller_shape():
     as_int32 = torch.zeros(sdl.tile_lists_bytes(B, H, L) // 4 - 1, dtype=torch.int32)
     with pytest.raises(sdl.SdlError):
         sdl.sparse_attn(q, q, q, None, None, 64, out=torch.empty_like(q), lists=as_int32)
+
+
+def test_binding_refuses_short_or_mistyped_index_buffers():
+    """CSR, plan and order buffers are read by the C calls without a size: the
+    binding checks their element counts and int32 type first (every call here
+    is refused before it reaches the library)."""
+    torch = pytest.importorskip("torch")
+    B, L, H = 1, 1024, 4
+    nb, n_qt = L // 64, L // 128
+    q = torch.zeros((B, L, H, 128), dtype=torch.bfloat16)
+    rp = torch.zeros(B * H * nb + 1, dtype=torch.int32)
+    ci = torch.zeros(8, dtype=torch.int32)
+    plan = torch.zeros((B, H, n_qt, 2), dtype=torch.int32)
+    order = torch.zeros(B * H * n_qt, dtype=torch.int32)
+    cases = [
+        dict(row_ptr=rp[:-1], col_idx=ci),
+        dict(row_ptr=rp.to(torch.int64), col_idx=ci),
+        dict(row_ptr=None, col_idx=ci),
+        dict(row_ptr=rp, col_idx=ci.to(torch.int64)),
+        dict(row_ptr=rp, col_idx=ci, plan=plan.reshape(-1)[:-1]),
+        dict(row_ptr=rp, col_idx=ci, plan=plan, order=order[:-1]),
+        dict(row_ptr=rp, col_idx=ci, plan=plan.to(torch.int64), order=order),
+    ]
+    for kw in cases:
+        rpk, cik = kw.pop("row_ptr"), kw.pop("col_idx")
+        with pytest.raises(sdl.SdlError) as e:
+            sdl.sparse_attn(q, q, q, rpk, cik, 64, out=torch.empty_like(q), **kw)
+        assert e.value.status == sdl.SDL_ERR_INVALID_ARG
+    with pytest.raises(sdl.SdlError):
+        sdl.tile_plan(rp[:-1], ci, B, H, L, 64)
+    with pytest.raises(sdl.SdlError):
+        sdl.tile_plan(rp, ci, B, H, L, 64, plan=plan.reshape(-1)[:-1])
+    with pytest.raises(sdl.SdlError):
+        sdl.tile_order(rp, plan.reshape(-1)[:-2], B, H, L, 64)
+    with pytest.raises(sdl.SdlError):
+        sdl.tile_order(rp, plan, B, H, L, 64, order=order[:-1])
+    with pytest.raises(sdl.SdlError):
+        sdl.tile_lists(rp, ci, None, order[:-1], B, H, L, 64)
+    with pytest.raises(sdl.SdlError):
+        sdl.tile_lists(rp[:-1], ci, None, None, B, H, L, 64)
