@@ -163,7 +163,9 @@ def _strides(t):
 
 
 def make_shape(q, k, block: int, v=None, o=None) -> Shape:
-    """sdl_shape for Q [B,L,H,d] and K/V [B,L,H_kv,d] tensors."""
+    """sdl_shape for Q [B,L,H,d] and K/V [B,L,H_kv,d] tensors (CUDA tensors only: the
+    library reads them on the device)."""
+    _on_cuda("inputs", q, k, v, o)
     B, L, H, d = q.shape
     s = Shape()
     s.B, s.H, s.H_kv, s.L, s.d, s.block = B, H, k.shape[2], L, d, block
@@ -466,9 +468,17 @@ def tile_order(row_ptr, plan, B: int, H: int, L: int, block: int = 64, order=Non
     if order is None:
         order = torch.empty(B * H * n_qt, dtype=torch.int32, device=plan.device)
     _need_i32(order, B * H * n_qt, "tile_order order")
+    _on_cuda("tile_order", row_ptr, plan, order)
     _check(_lib().sdl_tile_order(row_ptr.data_ptr(), plan.data_ptr(), ctypes.byref(s),
                                  order.data_ptr(), _stream(stream)), "sdl_tile_order")
     return order
+
+
+def _on_cuda(what: str, *tensors):
+    """Refuses host tensors: the library would hand their addresses to a kernel."""
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise SdlError(SDL_ERR_INVALID_ARG, f"{what}: CUDA tensors required")
 
 
 def _need_i32(t, n: int, what: str):
@@ -501,9 +511,11 @@ def tile_lists(row_ptr, col_idx, plan, order, B: int, H: int, L: int, block: int
         _need_i32(plan, B * H * n_qt * 2, "tile_lists plan")
     if order is not None:
         _need_i32(order, B * H * n_qt, "tile_lists order")
+    _need_i32(col_idx, 0, "tile_lists col_idx")
     if lists is None:
         lists = torch.empty(tile_lists_bytes(B, H, L, block), dtype=torch.uint8,
                             device=row_ptr.device)
+    _on_cuda("tile_lists", row_ptr, col_idx, plan, order, lists)
     _check(_lib().sdl_tile_lists(row_ptr.data_ptr(), col_idx.data_ptr(),
                                  None if plan is None else plan.data_ptr(),
                                  None if order is None else order.data_ptr(), ctypes.byref(s),
@@ -524,6 +536,8 @@ def tile_plan(row_ptr, col_idx, B: int, H: int, L: int, block: int = 64, plan=No
     if plan is None:
         plan = torch.empty((B, H, (nb + 1) // 2, 2), dtype=torch.int32, device=row_ptr.device)
     _need_i32(plan, B * H * ((nb + 1) // 2) * 2, "tile_plan plan")
+    _need_i32(col_idx, 0, "tile_plan col_idx")
+    _on_cuda("tile_plan", row_ptr, col_idx, plan)
     _check(_lib().sdl_tile_plan(row_ptr.data_ptr(), col_idx.data_ptr(), ctypes.byref(s),
                                 plan.data_ptr(), _stream(stream)), "sdl_tile_plan")
     return plan
@@ -537,29 +551,32 @@ def sparse_attn(q, k, v, row_ptr, col_idx, block: int, scale: float = 0.0, out=N
     the tiles' prebuilt lists from :func:`tile_lists` (used instead of the CSR, same bits
     as the plan and order they were built from)."""
     import torch
+    B, L, H = q.shape[0], q.shape[1], q.shape[2]
+    # the C calls read the lists, CSR, plan and order without a size: checked here
+    if lists is not None:
+        if lists.numel() * lists.element_size() < tile_lists_bytes(B, H, L, block):
+            raise SdlError(SDL_ERR_WORKSPACE, "sdl_sparse_attn_listed: lists too small")
+    else:
+        nb, n_qt = (L // block if block > 0 else 0), (L + 127) // 128
+        _need_i32(row_ptr, B * H * nb + 1, "sparse_attn row_ptr")
+        _need_i32(col_idx, 0, "sparse_attn col_idx")
+        if plan is not None:
+            _need_i32(plan, B * H * n_qt * 2, "sparse_attn plan")
+        if order is not None:
+            _need_i32(order, B * H * n_qt, "sparse_attn order")
     if out is None:
         out = torch.empty_like(q)
     s = make_shape(q, k, block, v, out)
     if lse is None and want_lse:
         lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
+    _on_cuda("sparse_attn", lse, lists, row_ptr, col_idx, plan, order)
     if lists is not None:
-        # the C call takes no size: a buffer built for a smaller shape is refused here
-        if lists.numel() * lists.element_size() < tile_lists_bytes(s.B, s.H, s.L, block):
-            raise SdlError(SDL_ERR_WORKSPACE, "sdl_sparse_attn_listed: lists too small")
         _check(_lib().sdl_sparse_attn_listed(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                              ctypes.byref(s), lists.data_ptr(), float(scale),
                                              out.data_ptr(),
                                              None if lse is None else lse.data_ptr(),
                                              _stream(stream)), "sdl_sparse_attn_listed")
     else:
-        nb = s.L // block if block > 0 else 0
-        n_qt = (s.L + 127) // 128
-        _need_i32(row_ptr, s.B * s.H * nb + 1, "sparse_attn row_ptr")
-        _need_i32(col_idx, 0, "sparse_attn col_idx")
-        if plan is not None:
-            _need_i32(plan, s.B * s.H * n_qt * 2, "sparse_attn plan")
-        if order is not None:
-            _need_i32(order, s.B * s.H * n_qt, "sparse_attn order")
         lse_p = None if lse is None else lse.data_ptr()
         if plan is not None and order is not None:
             _check(_lib().sdl_sparse_attn_scheduled(q.data_ptr(), k.data_ptr(), v.data_ptr(),

@@ -214,3 +214,21 @@ def test_binding_refuses_short_or_mistyped_index_buffers():
         sdl.tile_lists(rp, ci, None, order[:-1], B, H, L, 64)
     with pytest.raises(sdl.SdlError):
         sdl.tile_lists(rp[:-1], ci, None, None, B, H, L, 64)
+
+
+def test_binding_refuses_host_tensors():
+    """Every buffer the library reads lives on the device: host tensors of the
+    right sizes are refused before the call."""
+    torch = pytest.importorskip("torch")
+    B, L, H = 1, 512, 2
+    nb = L // 64
+    q = torch.zeros((B, L, H, 128), dtype=torch.bfloat16)
+    rp = torch.zeros(B * H * nb + 1, dtype=torch.int32)
+    ci = torch.zeros(8, dtype=torch.int32)
+    for call in (lambda: sdl.sparse_attn(q, q, q, rp, ci, 64, out=torch.empty_like(q)),
+                 lambda: sdl.dense_attn(q, q, q),
+                 lambda: sdl.tile_plan(rp, ci, B, H, L, 64),
+                 lambda: sdl.tile_lists(rp, ci, None, None, B, H, L, 64)):
+        with pytest.raises(sdl.SdlError) as e:
+            call()
+        assert e.value.status == sdl.SDL_ERR_INVALID_ARG
