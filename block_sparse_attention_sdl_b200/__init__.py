@@ -163,9 +163,8 @@ def _strides(t):
 
 
 def make_shape(q, k, block: int, v=None, o=None) -> Shape:
-    """sdl_shape for Q [B,L,H,d] and K/V [B,L,H_kv,d] tensors (CUDA tensors only: the
-    library reads them on the device)."""
-    _on_cuda("inputs", q, k, v, o)
+    """sdl_shape for Q [B,L,H,d] and K/V [B,L,H_kv,d] tensors (any device: only their
+    shapes, dtype and strides are read)."""
     B, L, H, d = q.shape
     s = Shape()
     s.B, s.H, s.H_kv, s.L, s.d, s.block = B, H, k.shape[2], L, d, block
@@ -223,6 +222,7 @@ def block_scores(q, k, block: int, scale: float = 0.0, scores=None, workspace=No
         scores = torch.empty((s.B, s.H, nb, nb), dtype=torch.float32, device=q.device)
     need = scores_workspace_bytes(s)
     workspace = _workspace(need, q.device, workspace)
+    _on_cuda("sdl_block_scores", q, k, scores, workspace)
     _check(_lib().sdl_block_scores(q.data_ptr(), k.data_ptr(), ctypes.byref(s), float(scale),
                                    scores.data_ptr(), workspace.data_ptr(), workspace.numel(),
                                    _stream(stream)), "sdl_block_scores")
@@ -253,12 +253,14 @@ def select_mask(scores, sparsity: float, block: int, L: int, row_ptr=None, col_i
     workspace = _workspace(select_workspace_bytes(s, per_head), dev, workspace)
     mask_ptr = None if mask is None else mask.data_ptr()
     if per_head:
+        _on_cuda("sdl_select_mask_scoped", scores, row_ptr, col_idx, workspace, mask)
         _check(_lib().sdl_select_mask_scoped(scores.data_ptr(), ctypes.byref(s), float(sparsity),
                                              SDL_BUDGET_HEAD, row_ptr.data_ptr(),
                                              col_idx.data_ptr(), col_idx.numel(), mask_ptr,
                                              workspace.data_ptr(), workspace.numel(),
                                              _stream(stream)), "sdl_select_mask_scoped")
     else:
+        _on_cuda("sdl_select_mask", scores, row_ptr, col_idx, workspace, mask)
         _check(_lib().sdl_select_mask(scores.data_ptr(), ctypes.byref(s), float(sparsity),
                                       row_ptr.data_ptr(), col_idx.data_ptr(), col_idx.numel(),
                                       mask_ptr, workspace.data_ptr(), workspace.numel(),
@@ -291,6 +293,7 @@ def anchor_refresh(q, k, block: int, sparsity: float, scores=None, row_ptr=None,
     if plan is None and want_plan and block == 64:
         plan = torch.empty((s.B, s.H, (nb + 1) // 2, 2), dtype=torch.int32, device=dev)
     workspace = _workspace(anchor_workspace_bytes(q, k, block), dev, workspace)
+    _on_cuda("sdl_anchor_refresh", q, k, scores, row_ptr, col_idx, plan, workspace)
     _check(_lib().sdl_anchor_refresh(q.data_ptr(), k.data_ptr(), ctypes.byref(s), float(scale),
                                      float(sparsity), scores.data_ptr(), row_ptr.data_ptr(),
                                      col_idx.data_ptr(), col_idx.numel(),
@@ -319,6 +322,7 @@ def col_scores(q, k, block: int, scale: float = 0.0, out=None, workspace=None, s
     if out is None:
         out = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
     workspace = _workspace(col_scores_workspace_bytes(q, k, block), q.device, workspace)
+    _on_cuda("sdl_col_scores", q, k, out, workspace)
     _check(_lib().sdl_col_scores(q.data_ptr(), k.data_ptr(), ctypes.byref(s), float(scale),
                                  out.data_ptr(), workspace.data_ptr(), workspace.numel(),
                                  _stream(stream)), "sdl_col_scores")
@@ -332,6 +336,7 @@ def col_select(col_scores_, q, k, block: int, sparsity: float, cols=None, stream
     Lc = col_budget(q, k, block, sparsity)
     if cols is None:
         cols = torch.empty((s.B, s.H, Lc), dtype=torch.int32, device=q.device)
+    _on_cuda("sdl_col_select", col_scores_, cols)
     _check(_lib().sdl_col_select(col_scores_.data_ptr(), ctypes.byref(s), float(sparsity),
                                  cols.data_ptr(), cols.numel(), _stream(stream)),
            "sdl_col_select")
@@ -347,6 +352,7 @@ def col_gather(k, v, cols, q, block: int, k_cols=None, v_cols=None, stream=None)
         k_cols = torch.empty((s.B, Lc, s.H, s.d), dtype=k.dtype, device=k.device)
     if v_cols is None:
         v_cols = torch.empty((s.B, Lc, s.H, s.d), dtype=v.dtype, device=v.device)
+    _on_cuda("sdl_col_gather", k, v, cols, k_cols, v_cols)
     _check(_lib().sdl_col_gather(k.data_ptr(), v.data_ptr(), ctypes.byref(s), cols.data_ptr(),
                                  int(Lc), k_cols.data_ptr(), v_cols.data_ptr(), _stream(stream)),
            "sdl_col_gather")
@@ -365,6 +371,7 @@ def col_sparse_attn(q, k_cols, v_cols, block: int = 64, scale: float = 0.0, out=
         s.o_strides[:] = _strides(out)
     if lse is None and want_lse:
         lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
+    _on_cuda("sdl_col_sparse_attn", q, k_cols, v_cols, out, lse)
     _check(_lib().sdl_col_sparse_attn(q.data_ptr(), k_cols.data_ptr(), v_cols.data_ptr(),
                                       ctypes.byref(s), int(Lc), float(scale), out.data_ptr(),
                                       None if lse is None else lse.data_ptr(), _stream(stream)),
@@ -408,6 +415,7 @@ def select_shard_capacity(scores, sparsity: float, block: int, L: int, heads_tot
 def select_shard_pass(scores, sparsity: float, block: int, L: int, heads_total: int, p: int,
                       workspace, stream=None):
     s = _score_shape(scores, block, L)
+    _on_cuda("sdl_select_shard_pass", scores, workspace)
     _check(_lib().sdl_select_shard_pass(scores.data_ptr(), ctypes.byref(s), int(heads_total),
                                         float(sparsity), int(p), workspace.data_ptr(),
                                         workspace.numel(), _stream(stream)),
@@ -421,6 +429,7 @@ def select_shard_count(scores, sparsity: float, block: int, L: int, heads_total:
     s = _score_shape(scores, block, L)
     if totals is None:
         totals = torch.empty((s.B, 2), dtype=torch.int64, device=scores.device)
+    _on_cuda("sdl_select_shard_count", scores, workspace, totals)
     _check(_lib().sdl_select_shard_count(scores.data_ptr(), ctypes.byref(s), int(heads_total),
                                          float(sparsity), workspace.data_ptr(),
                                          workspace.numel(), totals.data_ptr(), _stream(stream)),
@@ -445,6 +454,7 @@ def select_shard_finish(scores, sparsity: float, block: int, L: int, heads_total
         mask = torch.empty((s.B, s.H, nb, nb), dtype=torch.uint8, device=dev)
     if offsets.dtype != torch.int64 or not offsets.is_contiguous():
         raise ValueError("offsets must be a contiguous int64 [B, 2] tensor")
+    _on_cuda("sdl_select_shard_finish", scores, offsets, row_ptr, col_idx, mask, workspace)
     _check(_lib().sdl_select_shard_finish(scores.data_ptr(), ctypes.byref(s), int(heads_total),
                                           float(sparsity), offsets.data_ptr(),
                                           row_ptr.data_ptr(), col_idx.data_ptr(),
@@ -569,7 +579,7 @@ def sparse_attn(q, k, v, row_ptr, col_idx, block: int, scale: float = 0.0, out=N
     s = make_shape(q, k, block, v, out)
     if lse is None and want_lse:
         lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
-    _on_cuda("sparse_attn", lse, lists, row_ptr, col_idx, plan, order)
+    _on_cuda("sparse_attn", q, k, v, out, lse, lists, row_ptr, col_idx, plan, order)
     if lists is not None:
         _check(_lib().sdl_sparse_attn_listed(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                              ctypes.byref(s), lists.data_ptr(), float(scale),
@@ -608,6 +618,7 @@ def dense_attn(q, k, v, block: int = 64, scale: float = 0.0, out=None, lse=None,
     s = make_shape(q, k, block, v, out)
     if lse is None and want_lse:
         lse = torch.empty((s.B, s.H, s.L), dtype=torch.float32, device=q.device)
+    _on_cuda("sdl_dense_attn", q, k, v, out, lse)
     _check(_lib().sdl_dense_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(s),
                                  float(scale), out.data_ptr(),
                                  None if lse is None else lse.data_ptr(), _stream(stream)),

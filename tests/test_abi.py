@@ -228,7 +228,22 @@ def test_binding_refuses_host_tensors():
     for call in (lambda: sdl.sparse_attn(q, q, q, rp, ci, 64, out=torch.empty_like(q)),
                  lambda: sdl.dense_attn(q, q, q),
                  lambda: sdl.tile_plan(rp, ci, B, H, L, 64),
-                 lambda: sdl.tile_lists(rp, ci, None, None, B, H, L, 64)):
+                 lambda: sdl.tile_lists(rp, ci, None, None, B, H, L, 64),
+                 lambda: sdl.block_scores(q, q, 64),
+                 lambda: sdl.select_mask(torch.zeros((B, H, nb, nb)), 0.5, 64, L),
+                 lambda: sdl.anchor_refresh(q, q, 64, 0.5),
+                 lambda: sdl.col_scores(q, q, 64)):
         with pytest.raises(sdl.SdlError) as e:
             call()
         assert e.value.status == sdl.SDL_ERR_INVALID_ARG
+
+
+def test_sizing_calls_take_shape_only_probes():
+    """Shapes and workspace sizes come from tensors' shapes alone, so the layers
+    size their buffers from meta-device probes before any data exists."""
+    torch = pytest.importorskip("torch")
+    q = torch.empty((1, 8192, 32, 128), dtype=torch.bfloat16, device="meta")
+    assert sdl.make_shape(q, q, 64).L == 8192
+    assert sdl.anchor_workspace_bytes(q, q, 64) > 0
+    assert sdl.col_scores_workspace_bytes(q, q, 64) > 0
+    assert sdl.col_budget(q, q, 64, 0.9) == 832
