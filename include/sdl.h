@@ -248,7 +248,12 @@ sdl_status sdl_select_mask_noalloc(const float* scores, const sdl_shape* shape, 
  * reported as SDL_ERR_BAD_MASK by sdl_last_device_status().
  * lse (nullable): fp32 [B, H, L], natural-log sum of exp of the logits.
  * scale <= 0 means 1/sqrt(d).  bf16 runs on tcgen05 tensor cores (fp32
- * accumulation, output rounded to nearest even); fp32 runs on CUDA cores. */
+ * accumulation, output rounded to nearest even); fp32 runs on CUDA cores.
+ * Tile counter: each bf16 launch of this and the other attention calls takes
+ * its tiles from one of 64 device counters, used in turn across launches,
+ * and the launch's last CTA resets it.  So at most 64 bf16 attention launches
+ * may be in flight at once.  A CUDA graph that captures one keeps the counter
+ * it was captured with, so such a graph must not run concurrently with itself. */
 sdl_status sdl_sparse_attn(const void* q, const void* k, const void* v, const sdl_shape* shape,
                            const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o,
                            float* lse, void* stream);
