@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libsdl.so")
 
 SDL_OK, SDL_ERR_INVALID_ARG, SDL_ERR_UNSUPPORTED, SDL_ERR_CAPACITY = 0, 1, 2, 3
 SDL_ERR_WORKSPACE, SDL_ERR_CUDA, SDL_ERR_TIMEOUT, SDL_ERR_BAD_MASK = 4, 5, 6, 7
+SDL_ERR_OVERLAP = 8
 SDL_BF16, SDL_FP32 = 0, 1
 
 EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspace_bytes",

@@ -44,10 +44,17 @@ sdl_status check_shape(const sdl_shape* s) {
   return SDL_OK;
 }
 
-sdl_status check_strides(const int64_t* st, int dtype) {
+// Strides (b, t, h) in elements of a [B, T, heads, d] tensor: non-negative
+// multiples of 16 bytes, and nonzero on every axis with more than one index.
+// A zero stride there (a broadcast view, e.g. expand along heads) would make
+// distinct rows alias one address, which the TMA tensor maps cannot express.
+sdl_status check_strides(const int64_t* st, int dtype, int B, int T, int heads) {
   const int64_t q = dtype == SDL_BF16 ? 8 : 4;  // elements per 16 bytes
-  for (int i = 0; i < 3; ++i)
+  const int size[3] = {B, T, heads};
+  for (int i = 0; i < 3; ++i) {
     if (st[i] < 0 || st[i] % q) return SDL_ERR_INVALID_ARG;
+    if (st[i] == 0 && size[i] > 1) return SDL_ERR_INVALID_ARG;
+  }
   return SDL_OK;
 }
 
@@ -86,7 +93,8 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, const sdl_shape& s, int
   cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)(tokens > 0 ? tokens : s.L),
                         (cuuint64_t)heads, (cuuint64_t)s.B};
   cuuint64_t strides[3] = {(cuuint64_t)st[1] * 2, (cuuint64_t)st[2] * 2, (cuuint64_t)st[0] * 2};
-  // a zero stride (broadcast) is not expressible: use the dimension's natural size
+  // check_strides admits a zero stride only on an axis of one index, whose
+  // coordinate is always 0; the map still wants a nonzero multiple of 16 there
   for (int i = 0; i < 3; ++i)
     if (strides[i] == 0) strides[i] = 16;
   cuuint32_t box[4] = {box_d, box_t, 1, 1};
@@ -108,8 +116,11 @@ sdl_status attn_common(const void* q, const void* k, const void* v, const sdl_sh
   if (!q || !k || !v || !o) return SDL_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return SDL_ERR_INVALID_ARG;
-  if ((e = check_strides(s.q_strides, s.dtype)) || (e = check_strides(s.k_strides, s.dtype)) ||
-      (e = check_strides(s.v_strides, s.dtype)) || (e = check_strides(s.o_strides, s.dtype)))
+  const int lk = Lk > 0 ? Lk : s.L;
+  if ((e = check_strides(s.q_strides, s.dtype, s.B, s.L, s.H)) ||
+      (e = check_strides(s.k_strides, s.dtype, s.B, lk, s.H_kv)) ||
+      (e = check_strides(s.v_strides, s.dtype, s.B, lk, s.H_kv)) ||
+      (e = check_strides(s.o_strides, s.dtype, s.B, s.L, s.H)))
     return e;
   int* status = device_status_ptr();
   if (!status) return SDL_ERR_CUDA;
@@ -227,7 +238,8 @@ sdl_status sdl_block_scores(const void* q, const void* k, const sdl_shape* shape
   const sdl_shape& s = *shape;
   if (!q || !k || !scores) return SDL_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(scores)) return SDL_ERR_INVALID_ARG;
-  if ((e = check_strides(s.q_strides, s.dtype)) || (e = check_strides(s.k_strides, s.dtype)))
+  if ((e = check_strides(s.q_strides, s.dtype, s.B, s.L, s.H)) ||
+      (e = check_strides(s.k_strides, s.dtype, s.B, s.L, s.H_kv)))
     return e;
   const size_t need = sdl_scores_workspace_bytes(shape);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SDL_ERR_WORKSPACE;
@@ -306,7 +318,8 @@ sdl_status sdl_anchor_refresh(const void* q, const void* k, const sdl_shape* sha
   const sdl_shape& s = *shape;
   if (!q || !k || !scores || !row_ptr || !col_idx) return SDL_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(scores)) return SDL_ERR_INVALID_ARG;
-  if ((e = check_strides(s.q_strides, s.dtype)) || (e = check_strides(s.k_strides, s.dtype)))
+  if ((e = check_strides(s.q_strides, s.dtype, s.B, s.L, s.H)) ||
+      (e = check_strides(s.k_strides, s.dtype, s.B, s.L, s.H_kv)))
     return e;
   if (plan && s.block != 64) return SDL_ERR_INVALID_ARG;
   const int64_t total = sdl_mask_budget(shape, sparsity);
@@ -355,7 +368,8 @@ sdl_status sdl_col_scores(const void* q, const void* k, const sdl_shape* shape, 
   const sdl_shape& s = *shape;
   if (!q || !k || !col_scores) return SDL_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(col_scores)) return SDL_ERR_INVALID_ARG;
-  if ((e = check_strides(s.q_strides, s.dtype)) || (e = check_strides(s.k_strides, s.dtype)))
+  if ((e = check_strides(s.q_strides, s.dtype, s.B, s.L, s.H)) ||
+      (e = check_strides(s.k_strides, s.dtype, s.B, s.L, s.H_kv)))
     return e;
   const size_t need = sdl_col_scores_workspace_bytes(shape);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SDL_ERR_WORKSPACE;
@@ -397,7 +411,8 @@ sdl_status sdl_col_gather(const void* k, const void* v, const sdl_shape* shape,
   if (!k || !v || !cols || !k_cols || !v_cols || Lc <= 0 || Lc > s.L) return SDL_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cols) || !aligned16(v_cols))
     return SDL_ERR_INVALID_ARG;
-  if ((e = check_strides(s.k_strides, s.dtype)) || (e = check_strides(s.v_strides, s.dtype)))
+  if ((e = check_strides(s.k_strides, s.dtype, s.B, s.L, s.H_kv)) ||
+      (e = check_strides(s.v_strides, s.dtype, s.B, s.L, s.H_kv)))
     return e;
   cudaError_t ce = launch_col_gather(k, v, s, cols, Lc, k_cols, v_cols,
                                      static_cast<cudaStream_t>(stream));
@@ -644,6 +659,7 @@ sdl_status sdl_last_device_status(void* stream) {
   if (ce != cudaSuccess) return cuda_fail(ce);
   if (v & kDevTimeout) return SDL_ERR_TIMEOUT;
   if (v & kDevBadMask) return SDL_ERR_BAD_MASK;
+  if (v & kDevOverlap) return SDL_ERR_OVERLAP;
   return SDL_OK;
 }
 
@@ -667,6 +683,8 @@ const char* sdl_status_string(sdl_status status) {
       return "a kernel's bounded wait timed out";
     case SDL_ERR_BAD_MASK:
       return "mask list entry out of range or out of order";
+    case SDL_ERR_OVERLAP:
+      return "attention launches in flight shared a tile counter";
   }
   return "unknown status";
 }

@@ -3,47 +3,58 @@
 // The fused IO-aware block-sparse kernel of the Step-dLLM abstract,
 // re-designed for Blackwell.  A work item is a 128-row query tile of one
 // head; it walks the kept key blocks of its rows, two 64-token sub-blocks
-// (128 keys) per step.  CTAs are persistent and small enough that two run
-// on every SM; each works through one item at a time, so the two CTAs of an
-// SM interleave on its tensor cores (one's softmax overlaps the other's
-// products) without waiting on each other.  Items come from a global
-// counter, first come first served (tiles differ in cost by the length of
-// their kept lists).
+// (128 keys) per step.  CTAs are persistent, one per SM, and take items from
+// a global counter, first come first served (tiles differ in cost by the
+// length of their kept lists).
+//
+// Each step's 128 keys are split between two softmax warpgroups: group 0
+// owns keys 0..63 (the step's first sub-block), group 1 keys 64..127.  Each
+// group runs its own online softmax over its half of every step, with its own
+// running maximum, row sums and O accumulator in TMEM, so the two groups never
+// wait on each other inside a tile; the epilogue merges the two partial
+// results (the same merge as for two key ranges of a split softmax).  S is
+// double-buffered in TMEM, so the product S(n+1) = Q K(n+1)^T runs on the
+// tensor cores while both groups work on S(n).
 //
 //   warp 0        loads: takes items and copies an item's prebuilt list
 //                 (tile_lists_kernel, run once per mask) or builds the union
 //                 list of its two query blocks into a list slot (three slots,
 //                 the next item's list while the current item runs); per item
-//                 its Q tile, per step its K and V sub-blocks by TMA
-//                 (128-byte-swizzled 64x64 boxes) into one K and one V stage.
-//                 Items whose lists are empty (only a caller's mask can have
-//                 empty rows) are written here as zero rows.
-//   warp 1        TMEM allocator and MMA issuer (one thread):
-//                   S = Q K^T    tcgen05.mma kind::f16, A and B from shared
-//                                memory, M=128, N=128, fp32 in TMEM;
-//                   O += P V     A = P (bf16, over S's first 64 TMEM
-//                                columns), B = V from shared memory
-//                                (N-major), M=128, N=d; issued in two
-//                                halves, keys 0..63 as soon as the softmax
-//                                has written their weights.
-//                 The next S is issued after the PV product (the two share
-//                 S's columns), which also leaves O quiescent for the
-//                 softmax once that S product has completed.
-//   warps 2-5     softmax: one thread per query row (its TMEM lane), all 128
-//                 columns of the step.  Online softmax in the log2 domain;
-//                 the running max is raised only when it grows by more than
-//                 8 (a factor 256), and O is rescaled in TMEM only then; P
-//                 written back as bf16, the row sum taken over those rounded
-//                 weights (the LSE's over the fp32 weights).  Epilogue per
-//                 item: O / l rounded to bf16 and written by TMA tensor
-//                 stores from a per-warp shared-memory box, LSE.
+//                 its Q tile into one of two Q stages, per step its K and V
+//                 sub-blocks by TMA (128-byte-swizzled 64x64 boxes) into
+//                 two-stage K and V rings, K one step ahead of V.  Items whose
+//                 lists are empty (only a caller's mask can have empty rows)
+//                 are written here as zero rows.
+//   warp 1        TMEM allocator and MMA issuer (one elected thread):
+//                   S(n) = Q K(n)^T  tcgen05.mma kind::f16, A and B from shared
+//                                    memory, M=128, N=128, fp32 into TMEM
+//                                    buffer n % 2;
+//                   O_g += P_g V_g   for each group g once it has written its
+//                                    weights: A = P_g (bf16 in TMEM, over the
+//                                    group's own S columns), B = the group's 64
+//                                    V rows (N-major), M=128, N=d.
+//                 Issue order S(n), O(n-1): the next S is on the tensor pipe
+//                 before the groups finish the current step.
+//   warps 2-5     softmax group 0, warps 6-9 group 1: one thread per query row
+//                 (its TMEM lane quadrant), 64 columns of each step.  Online
+//                 softmax in the log2 domain; the running maximum is raised only
+//                 when it grows by more than 8 (a factor 256), and the group's O
+//                 is rescaled in TMEM only then; P written back as bf16, the row
+//                 sum taken over those rounded weights (the LSE's over the fp32
+//                 weights).  Epilogue per item: the groups exchange their row
+//                 maxima and sums through shared memory, each merges and scales
+//                 half of O's columns, rounds to bf16 and writes them by TMA
+//                 tensor stores from per-warp shared-memory boxes; group 0
+//                 writes the LSE.
 //
 // With 64-token blocks a 128-row tile covers two query blocks; the item walks
 // the union of their kept lists and masks, per 64x64 quadrant, the key
 // sub-blocks a query block did not keep.  With 128-token blocks both halves
 // share one list.  Dense attention is the same walk over every sub-block.
 //
-// TMEM (256 columns per CTA): S at column 0, O at 128.
+// TMEM (512 columns, the whole SM's): S buffers at columns 0 and 128 (group g
+// reads columns 64 g .. 64 g + 63 of a buffer and writes its P over the first 32
+// of them), O of group g at 256 + 128 g.
 // Every mbarrier wait is bounded; on timeout the CTA raises the device status
 // word, drains its own copies and MMAs, frees TMEM and exits.
 #include <cuda_bf16.h>
@@ -61,15 +72,16 @@ constexpr int kBM = 128;         // query rows per item
 constexpr int kBN = 128;         // key rows per step
 constexpr int kSlots = 3;        // list slots
 constexpr int kMaxSub = 1024;    // 64-token sub-blocks per sequence (L <= 65536)
-constexpr int kThreads = 192;    // 6 warps
-constexpr int kCtasPerSm = 2;
+constexpr int kGroups = 2;       // softmax warpgroups (one per 64-key half of a step)
+constexpr int kSoftWarps = 4 * kGroups;
+constexpr int kThreads = 32 * (2 + kSoftWarps);  // load, MMA, softmax
 constexpr int kLoadWarp = 0, kMmaWarp = 1, kSoftWarp0 = 2;
+constexpr int kQStages = 2, kKStages = 2, kVStages = 2;
 constexpr int kBox = 64 * 128;   // bytes of one 64-row x 64-column bf16 box
 constexpr int kOBoxBytes = 32 * 64;  // one 32-row x 32-column bf16 output box
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColO = 128;
-// PV issued in two halves, the first once the softmax has written keys 0..63
-constexpr bool kSplitPV = true;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;    // S buffer b at kColS + 128 b
+constexpr uint32_t kColO = 256;  // O of group g at kColO + 128 g
 
 template <int D>
 struct Layout {
@@ -79,30 +91,33 @@ struct Layout {
   static constexpr int kChunkRowsQ = kBM * 128;    // bytes per Q column chunk
   static constexpr int kChunkRowsKV = kBN * 128;   // bytes per K/V column chunk
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kQBytes;
-  static constexpr int kOffV = kOffK + kKVBytes;
+  static constexpr int kOffK = kOffQ + kQStages * kQBytes;
+  static constexpr int kOffV = kOffK + kKStages * kKVBytes;
   // output staging: per softmax warp one 32-row x 32-column bf16 box
   // (64-byte rows, 64-byte swizzle) for the tensor stores of O
-  static constexpr int kOffO = kOffV + kKVBytes;
-  static constexpr int kBytes = kOffO + 4 * kOBoxBytes;
+  static constexpr int kOffO = kOffV + kVStages * kKVBytes;
+  static constexpr int kBytes = kOffO + kSoftWarps * kOBoxBytes;
   static constexpr int kSmem = kBytes + 1024;      // + alignment slack
 };
-// two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per
-// CTA, and up to 8 KB of static shared memory per CTA
-static_assert(kCtasPerSm * (Layout<128>::kSmem + 8192 + 1024) <= 228 * 1024, "shared memory");
+// one CTA per SM: 228 KB of shared memory per SM, 1 KB of it reserved per
+// CTA, and up to 12 KB of static shared memory
+static_assert(Layout<128>::kSmem + 12 * 1024 + 1024 <= 228 * 1024, "shared memory");
 
-// Consumers of a list slot: the MMA warp and the 4 softmax warps.
-constexpr int kListConsumers = 1 + 4;
+// Consumers of a list slot: the MMA warp and the softmax warps.
+constexpr int kListConsumers = 1 + kSoftWarps;
 
 struct Bars {
   uint64_t list_full[kSlots];   // slot published by the load warp
   uint64_t list_empty[kSlots];  // slot released by every consumer
-  uint64_t q_full, q_empty;     // Q landed / the item's S products completed
-  uint64_t kfull, kempty, vfull, vempty;
-  uint64_t s_full;              // S written
-  uint64_t p_half;              // P of keys 0..63 written (one arrival per softmax warp)
-  uint64_t p_full;              // all of P written (one arrival per softmax warp)
+  uint64_t q_full[kQStages], q_empty[kQStages];  // Q landed / the item's S products completed
+  uint64_t kfull[kKStages], kempty[kKStages];
+  uint64_t vfull[kVStages], vempty[kVStages];
+  uint64_t s_full[2];           // S buffer b written
+  uint64_t p_ready[kGroups][2]; // group g's P in buffer b written (one arrival per warp)
+  uint64_t pv_done[kGroups][2]; // group g's product of a step of parity b completed
   uint64_t o_full;              // every product of the item completed
+  uint64_t o_empty;             // the epilogue has read O (one arrival per softmax warp)
+  uint64_t xch;                 // the groups' row maxima and sums exchanged
   uint64_t done;
 };
 
@@ -119,8 +134,10 @@ constexpr uint32_t kKeepShift = 14;
 constexpr uint32_t kSubMask = (1u << kKeepShift) - 1u;
 
 // Item counters of in-flight launches.  Launch n uses entry n % kSchedRing;
-// its CTAs take items with atomicAdd on `next`, and the last CTA to finish
-// puts the entry back to zero for a later launch.
+// its CTAs take items with atomicAdd on `next` (each CTA's last add is the
+// one past the end), and the last CTA to finish checks that the counter saw
+// exactly the launch's items and one add per CTA past them -- more means
+// another launch in flight shared the entry -- then puts it back to zero.
 constexpr int kSchedRing = 64;
 struct Sched {
   unsigned next;
@@ -354,8 +371,9 @@ __global__ void __launch_bounds__(kListWarps * 32) tile_lists_kernel(AttnArgs a,
   }
 }
 
+
 template <int D, bool kLse>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                    const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
                    AttnArgs a, int sched_slot) {
@@ -366,6 +384,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __shared__ Bars bars;
   __shared__ Slot slots[kSlots];
   __shared__ uint32_t bmask[2][kMaxSub / 32];
+  // the groups' final row maxima (log2 units), sums of the rounded weights and
+  // sums of the unrounded weights, exchanged at the epilogue
+  __shared__ float xm[kGroups][kBM], xl[kGroups][kBM], xlx[kGroups][kBM];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
 
@@ -379,16 +400,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         mbar_init(&bars.list_full[s], 1);
         mbar_init(&bars.list_empty[s], kListConsumers);
       }
-      mbar_init(&bars.q_full, 1);
-      mbar_init(&bars.q_empty, 1);
-      mbar_init(&bars.kfull, 1);
-      mbar_init(&bars.kempty, 1);
-      mbar_init(&bars.vfull, 1);
-      mbar_init(&bars.vempty, 1);
-      mbar_init(&bars.s_full, 1);
-      mbar_init(&bars.p_half, 4);
-      mbar_init(&bars.p_full, 4);
+      for (int s = 0; s < kQStages; ++s) {
+        mbar_init(&bars.q_full[s], 1);
+        mbar_init(&bars.q_empty[s], 1);
+      }
+      for (int s = 0; s < kKStages; ++s) {
+        mbar_init(&bars.kfull[s], 1);
+        mbar_init(&bars.kempty[s], 1);
+      }
+      for (int s = 0; s < kVStages; ++s) {
+        mbar_init(&bars.vfull[s], 1);
+        mbar_init(&bars.vempty[s], 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&bars.s_full[b], 1);
+        for (int g = 0; g < kGroups; ++g) {
+          mbar_init(&bars.p_ready[g][b], 4);
+          mbar_init(&bars.pv_done[g][b], 1);
+        }
+      }
       mbar_init(&bars.o_full, 1);
+      mbar_init(&bars.o_empty, kSoftWarps);
+      mbar_init(&bars.xch, kSoftWarps);
       mbar_init(&bars.done, 1);
       abort_sh = 0;
       fence_barrier_init();
@@ -417,8 +450,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     int built = 0;   // lists published (the end marker included)
     bool ended = false;
     int nq = 0;      // Q tiles loaded
-    int g = 0;       // steps loaded (K and V stage phases)
-    int gk = 0, gv = 0;  // K and V copies issued (one ahead of g between a step's copies)
+    int nk = 0;      // K copies issued (one per step)
+    int nv = 0;      // V copies issued (one per step, one step behind K)
+    // the step whose V is still to be loaded: its two sub-blocks, KV head, batch
+    bool v_pend = false;
+    int pv_sub0 = 0, pv_sub1 = 0, pv_kh = 0, pv_b = 0;
     // publishes the next list into its slot once the slot's item is done
     auto publish_next = [&]() -> bool {
       const int slot = built % kSlots;
@@ -431,70 +467,101 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       ++built;
       return true;
     };
+    // V of the pending step, once the product that last read its stage has completed
+    auto load_v = [&]() -> bool {
+      if (!v_pend) return true;
+      const int vs = nv % kVStages;
+      if (nv >= kVStages &&
+          !__all_sync(0xffffffffu, mbar_wait(&bars.vempty[vs], ((nv / kVStages) - 1) & 1,
+                                             &abort_sh, a.status, kWaitLimitNs)))
+        return false;
+      if (leader) {
+        uint8_t* dst = dsm + Lay::kOffV + vs * Lay::kKVBytes;
+        mbar_arrive_expect_tx(&bars.vfull[vs], Lay::kKVBytes);
+        for (int c = 0; c < Lay::kChunks; ++c)
+          for (int s = 0; s < 2; ++s)
+            tma_load_4d(dst + c * Lay::kChunkRowsKV + s * kBox, &tmv, &bars.vfull[vs], c * 64,
+                        (s ? pv_sub1 : pv_sub0) * kSubBlock, pv_kh, pv_b);
+      }
+      ++nv;
+      v_pend = false;
+      return true;
+    };
     ok = publish_next();
     for (int k = 0; ok; ++k) {
       const Slot& S = slots[k % kSlots];
       if (S.item < 0) break;
       const int n_ent = S.n_ent, kh = S.h / group, b = S.b;
-      // Q of the item, once the previous item's S products have completed
-      if (nq > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&bars.q_empty, (nq - 1) & 1,
-                                                             &abort_sh, a.status, kWaitLimitNs))))
+      // Q of the item, once the S products of the item that last used its stage have completed
+      const int qs = nq % kQStages;
+      if (nq >= kQStages &&
+          !(ok = __all_sync(0xffffffffu, mbar_wait(&bars.q_empty[qs], ((nq / kQStages) - 1) & 1,
+                                                   &abort_sh, a.status, kWaitLimitNs))))
         break;
       if (leader) {
-        uint8_t* sq = dsm + Lay::kOffQ;
-        mbar_arrive_expect_tx(&bars.q_full, Lay::kQBytes);
+        uint8_t* sq = dsm + Lay::kOffQ + qs * Lay::kQBytes;
+        mbar_arrive_expect_tx(&bars.q_full[qs], Lay::kQBytes);
         for (int cc = 0; cc < Lay::kChunks; ++cc)
           for (int s = 0; s < 2; ++s)
-            tma_load_4d(sq + cc * Lay::kChunkRowsQ + s * kBox, &tmq, &bars.q_full, cc * 64,
+            tma_load_4d(sq + cc * Lay::kChunkRowsQ + s * kBox, &tmq, &bars.q_full[qs], cc * 64,
                         s ? S.t1 : S.t0, S.h, b);
       }
       ++nq;
       const int n_steps = (n_ent + 1) / 2;
-      for (int j = 0; j < n_steps; ++j, ++g) {
+      for (int j = 0; j < n_steps; ++j) {
         const uint32_t e0 = S.ent[2 * j];
         const uint32_t e1 = (2 * j + 1 < n_ent) ? S.ent[2 * j + 1] : e0;
         const int sub0 = (int)(e0 & kSubMask), sub1 = (int)(e1 & kSubMask);
-        // K of the step once the previous S product has completed
-        if (g > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&bars.kempty, (g - 1) & 1,
-                                                              &abort_sh, a.status, kWaitLimitNs))))
+        // K of the step once the S product that last read its stage has completed
+        const int ks = nk % kKStages;
+        if (nk >= kKStages &&
+            !(ok = __all_sync(0xffffffffu, mbar_wait(&bars.kempty[ks], ((nk / kKStages) - 1) & 1,
+                                                     &abort_sh, a.status, kWaitLimitNs))))
           break;
         if (leader) {
-          uint8_t* dst = dsm + Lay::kOffK;
-          mbar_arrive_expect_tx(&bars.kfull, Lay::kKVBytes);
+          uint8_t* dst = dsm + Lay::kOffK + ks * Lay::kKVBytes;
+          mbar_arrive_expect_tx(&bars.kfull[ks], Lay::kKVBytes);
           for (int c = 0; c < Lay::kChunks; ++c)
             for (int s = 0; s < 2; ++s)
-              tma_load_4d(dst + c * Lay::kChunkRowsKV + s * kBox, &tmk, &bars.kfull, c * 64,
+              tma_load_4d(dst + c * Lay::kChunkRowsKV + s * kBox, &tmk, &bars.kfull[ks], c * 64,
                           (s ? sub1 : sub0) * kSubBlock, kh, b);
         }
-        gk = g + 1;
+        ++nk;
+        // V of the previous step (its product is issued after this step's S)
+        if (!(ok = load_v())) break;
+        v_pend = true;
+        pv_sub0 = sub0;
+        pv_sub1 = sub1;
+        pv_kh = kh;
+        pv_b = b;
         // the next item's list, while this one runs
         if (j == 0 && !ended && !(ok = publish_next())) break;
-        // V of the step once the previous PV product has completed
-        if (g > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&bars.vempty, (g - 1) & 1,
-                                                              &abort_sh, a.status, kWaitLimitNs))))
-          break;
-        if (leader) {
-          uint8_t* dst = dsm + Lay::kOffV;
-          mbar_arrive_expect_tx(&bars.vfull, Lay::kKVBytes);
-          for (int c = 0; c < Lay::kChunks; ++c)
-            for (int s = 0; s < 2; ++s)
-              tma_load_4d(dst + c * Lay::kChunkRowsKV + s * kBox, &tmv, &bars.vfull, c * 64,
-                          (s ? sub1 : sub0) * kSubBlock, kh, b);
-        }
-        gv = g + 1;
       }
     }
+    if (ok) ok = load_v();
     if (leader) {
       if (!ok) raise_timeout(&abort_sh, a.status);
-      // Drain: every copy issued above lands before the CTA exits.  The K and V
-      // copies are counted apart: a step left early has its K copy in flight.
+      // Drain: every copy issued above lands before the CTA exits (the last
+      // copy into each stage; earlier ones completed before it was reused).
       volatile int no_abort = 0;
-      if (gk > 0 && !mbar_wait(&bars.kfull, (gk - 1) & 1, &no_abort, nullptr, kWaitLimitNs))
-        atomicOr(a.status, kDevTimeout);
-      if (gv > 0 && !mbar_wait(&bars.vfull, (gv - 1) & 1, &no_abort, nullptr, kWaitLimitNs))
-        atomicOr(a.status, kDevTimeout);
-      if (nq > 0 && !mbar_wait(&bars.q_full, (nq - 1) & 1, &no_abort, nullptr, kWaitLimitNs))
-        atomicOr(a.status, kDevTimeout);
+      for (int s = 0; s < kKStages; ++s) {
+        const int c = nk - 1 - ((nk - 1 - s) % kKStages + kKStages) % kKStages;  // last copy into s
+        if (c >= 0 && c % kKStages == s &&
+            !mbar_wait(&bars.kfull[s], (c / kKStages) & 1, &no_abort, nullptr, kWaitLimitNs))
+          atomicOr(a.status, kDevTimeout);
+      }
+      for (int s = 0; s < kVStages; ++s) {
+        const int c = nv - 1 - ((nv - 1 - s) % kVStages + kVStages) % kVStages;
+        if (c >= 0 && c % kVStages == s &&
+            !mbar_wait(&bars.vfull[s], (c / kVStages) & 1, &no_abort, nullptr, kWaitLimitNs))
+          atomicOr(a.status, kDevTimeout);
+      }
+      for (int s = 0; s < kQStages; ++s) {
+        const int c = nq - 1 - ((nq - 1 - s) % kQStages + kQStages) % kQStages;
+        if (c >= 0 && c % kQStages == s &&
+            !mbar_wait(&bars.q_full[s], (c / kQStages) & 1, &no_abort, nullptr, kWaitLimitNs))
+          atomicOr(a.status, kDevTimeout);
+      }
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -508,73 +575,102 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const uint64_t dq = smem_desc_sw128(smem_u32(dsm + Lay::kOffQ), 16, 1024);
     const uint64_t dk = smem_desc_sw128(smem_u32(dsm + Lay::kOffK), 16, 1024);
     const uint64_t dv = smem_desc_sw128(smem_u32(dsm + Lay::kOffV), Lay::kChunkRowsKV, 1024);
-    const uint32_t scol = tmem + kColS, ocol = tmem + kColO;
     bool ok = true;
-    int n = 0;  // steps issued
+    int n = 0;  // steps whose S product was issued
+    int t = 0;  // items
+    // the step whose PV products are still to be issued
+    bool pend = false, pend_first = false, pend_last = false;
+    int pend_step = 0, pend_item = 0;
+    // O_g += P_g V_g of the pending step m for both groups (keys 64 g .. 64 g + 63)
+    auto issue_pv = [&]() -> bool {
+      const int m = pend_step;
+      const int vs = m % kVStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.vfull[vs], (m / kVStages) & 1, &abort_sh,
+                                             a.status, kWaitLimitNs)))
+        return false;
+      // the first product of an item overwrites O: the previous epilogue must have read it
+      if (pend_first && pend_item > 0 &&
+          !__all_sync(0xffffffffu, mbar_wait(&bars.o_empty, (pend_item - 1) & 1, &abort_sh,
+                                             a.status, kWaitLimitNs)))
+        return false;
+      const uint64_t dvs = dv + (uint64_t)((vs * Lay::kKVBytes) >> 4);
+#pragma unroll
+      for (int g = 0; g < kGroups; ++g) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.p_ready[g][m & 1], (m >> 1) & 1, &abort_sh,
+                                               a.status, kWaitLimitNs)))
+          return false;
+        tc_fence_after();
+        const uint32_t pcol = tmem + kColS + 128u * (uint32_t)(m & 1) + 64u * g;
+        const uint32_t ocol = tmem + kColO + 128u * g;
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          // keys [64 g + 16 kq, +16): V rows of the stage (128 bytes each); P
+          // elements packed in the group's columns [8 kq, 8 kq + 8)
+          const int kk = 4 * g + kq;
+          if (leader)
+            mma_bf16_ts(ocol, pcol + 8 * kq, dvs + (uint64_t)((kk * 16 * 128) >> 4), idPV,
+                        (pend_first && kq == 0) ? 0u : 1u);
+        }
+        if (leader) tc_commit(&bars.pv_done[g][m & 1]);
+      }
+      if (leader) {
+        tc_commit(&bars.vempty[vs]);
+        if (pend_last) tc_commit(&bars.o_full);
+      }
+      pend = false;
+      return true;
+    };
     for (int k = 0; ok; ++k) {
       const int slot = k % kSlots;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.list_full[slot], (k / kSlots) & 1,
                                                    &abort_sh, a.status, kWaitLimitNs))))
         break;
       const Slot& S = slots[slot];
-      if (S.item < 0) break;
+      const int item_valid = S.item >= 0;
       const int n_steps = (S.n_ent + 1) / 2;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.q_full, k & 1, &abort_sh, a.status,
-                                                   kWaitLimitNs))))
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.list_empty[slot]);  // the slot's header was all it needed
+      if (!item_valid) break;
+      const int qs = t % kQStages;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.q_full[qs], (t / kQStages) & 1,
+                                                   &abort_sh, a.status, kWaitLimitNs))))
         break;
-      for (int j = 0; j < n_steps; ++j, ++n) {
-        const bool last = j == n_steps - 1;
-        // S = Q K^T (the previous PV product, which reads S's columns, was issued before)
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.kfull, n & 1, &abort_sh, a.status,
-                                                     kWaitLimitNs))))
+      const uint64_t dqs = dq + (uint64_t)((qs * Lay::kQBytes) >> 4);
+      for (int j = 0; j < n_steps; ++j) {
+        // S(n) into buffer n % 2: its previous content S(n - 2) has been read
+        // by both groups (their weights for step n - 2 were awaited before the
+        // PV products of n - 2, issued ahead of this product)
+        const int ks = n % kKStages;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.kfull[ks], (n / kKStages) & 1,
+                                                     &abort_sh, a.status, kWaitLimitNs))))
           break;
         tc_fence_after();
+        const uint64_t dks = dk + (uint64_t)((ks * Lay::kKVBytes) >> 4);
+        const uint32_t scol = tmem + kColS + 128u * (uint32_t)(n & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           // 16 d-columns: chunk kk / 4, 32 bytes (kk % 4) inside the swizzle atom
           const uint64_t offq = (uint64_t)(((kk / 4) * Lay::kChunkRowsQ + (kk % 4) * 32) >> 4);
           const uint64_t offk = (uint64_t)(((kk / 4) * Lay::kChunkRowsKV + (kk % 4) * 32) >> 4);
-          if (leader) mma_bf16_ss(scol, dq + offq, dk + offk, idS, kk > 0 ? 1u : 0u);
+          if (leader) mma_bf16_ss(scol, dqs + offq, dks + offk, idS, kk > 0 ? 1u : 0u);
         }
         if (leader) {
-          tc_commit(&bars.kempty);
-          tc_commit(&bars.s_full);
-          if (last) tc_commit(&bars.q_empty);
+          tc_commit(&bars.kempty[ks]);
+          tc_commit(&bars.s_full[n & 1]);
+          if (j == n_steps - 1) tc_commit(&bars.q_empty[qs]);
         }
-        // O += P V in two halves: keys 0..63 once the softmax has written their
-        // weights (the product runs while it computes the rest), then keys 64..127
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(kSplitPV ? &bars.p_half : &bars.p_full, n & 1,
-                                                     &abort_sh, a.status, kWaitLimitNs))))
-          break;
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars.vfull, n & 1, &abort_sh, a.status,
-                                                     kWaitLimitNs))))
-          break;
-#pragma unroll
-        for (int hk = 0; hk < 2; ++hk) {
-          if (kSplitPV && hk == 1 &&
-              !(ok = __all_sync(0xffffffffu, mbar_wait(&bars.p_full, n & 1, &abort_sh, a.status,
-                                                       kWaitLimitNs))))
-            break;
-          tc_fence_after();
-#pragma unroll
-          for (int kq = 0; kq < kBN / 32; ++kq) {
-            // keys [16 kk, 16 kk + 16): V rows 16 kk.. (128 bytes each); P elements
-            // packed in columns [8 kk, 8 kk + 8)
-            const int kk = hk * (kBN / 32) + kq;
-            if (leader)
-              mma_bf16_ts(ocol, scol + 8 * kk, dv + (uint64_t)((kk * 16 * 128) >> 4), idPV,
-                          (j > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        if (!ok) break;
-        if (leader) {
-          tc_commit(&bars.vempty);
-          if (last) tc_commit(&bars.o_full);
-        }
+        // then the PV products of the previous step
+        if (pend && !(ok = issue_pv())) break;
+        pend = true;
+        pend_step = n;
+        pend_first = j == 0;
+        pend_last = j == n_steps - 1;
+        pend_item = t;
+        ++n;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
+      ++t;
     }
+    if (ok && pend) ok = issue_pv();
     if (leader) {
       if (!ok) raise_timeout(&abort_sh, a.status);
       // Every MMA issued above completes before TMEM is released.
@@ -586,15 +682,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     __syncwarp();
   } else {
     // ============================================================ softmax
-    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int sw = warp - kSoftWarp0;  // 0..7
+    const int grp = sw / 4;            // 0: keys 0..63 of every step, 1: keys 64..127
+    const int quad = warp & 3;         // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;
     const int half = row >> 6;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t scol = trow + kColS;
-    const uint32_t ocol = trow + kColO;
-    uint8_t* ostage = dsm + Lay::kOffO + (warp - kSoftWarp0) * kOBoxBytes;
+    const uint32_t ocol_own = trow + kColO + 128u * grp;
+    const uint32_t ocol_oth = trow + kColO + 128u * (1 - grp);
+    uint8_t* ostage = dsm + Lay::kOffO + sw * kOBoxBytes;
     const float sl2 = a.scale_log2;
     int n = 0;  // steps so far
+    uint32_t xuses = 0;
     bool ok = true;
     for (int k = 0;; ++k) {
       const int slot = k % kSlots;
@@ -609,128 +708,131 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       float l = 0.f;        // row sum of the bf16-rounded weights
       float lx = 0.f;       // row sum of the unrounded weights (LSE only)
       for (int j = 0; j < n_steps; ++j, ++n) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(&bars.s_full, n & 1, &abort_sh, a.status, kWaitLimitNs));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full[n & 1], (n >> 1) & 1, &abort_sh,
+                                               a.status, kWaitLimitNs));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t e0 = S.ent[2 * j];
-        const uint32_t e1 = (2 * j + 1 < n_ent) ? S.ent[2 * j + 1] : (e0 & kSubMask);
+        // this group's sub-block of the step (the padding of an odd list keeps nothing)
+        const uint32_t e = grp == 0 ? (uint32_t)S.ent[2 * j]
+                                    : ((2 * j + 1 < n_ent) ? (uint32_t)S.ent[2 * j + 1] : 0u);
         // (keep is uniform over a warp: its 32 rows lie in one query block)
-        const bool keep0 = (e0 >> (kKeepShift + half)) & 1u;
-        const bool keep1 = (e1 >> (kKeepShift + half)) & 1u;
-        uint32_t r[128];
-        tmem_ld32(scol + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_ld32(scol + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-        tmem_ld32(scol + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
-        tmem_wait_ld();
-        // tile maxima of the two 64-column halves (three-input max)
-        float mh[2];
+        const bool keep = (e >> (kKeepShift + half)) & 1u;
+        const uint32_t scol = trow + kColS + 128u * (uint32_t)(n & 1) + 64u * grp;
+        uint32_t pw[32];
+        if (keep) {
+          uint32_t r[64];
+          tmem_ld32(scol + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          tmem_wait_ld();
+          // tile maximum (three-input max)
+          float m0 = __uint_as_float(r[0]), m1 = __uint_as_float(r[1]);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int x0 = 64 * hf;
-          float m0 = __uint_as_float(r[x0]), m1 = __uint_as_float(r[x0 + 1]);
-#pragma unroll
-          for (int x = x0 + 2; x < x0 + 62; x += 4) {
+          for (int x = 2; x < 62; x += 4) {
             m0 = max3f(m0, __uint_as_float(r[x]), __uint_as_float(r[x + 1]));
             m1 = max3f(m1, __uint_as_float(r[x + 2]), __uint_as_float(r[x + 3]));
           }
-          mh[hf] = max3f(m0, m1, fmaxf(__uint_as_float(r[x0 + 62]), __uint_as_float(r[x0 + 63])));
-        }
-        const float mt = fmaxf(keep0 ? mh[0] : -INFINITY, keep1 ? mh[1] : -INFINITY) * sl2;
-        const bool raise = mt > m + 8.0f;
-        if (__any_sync(0xffffffffu, raise)) {
-          if (j > 0) {
-            // O is quiescent: this step's S product was issued after the
-            // previous PV product and has completed.
-            const float alpha = raise ? ex2_approx(m - mt) : 1.0f;
-            l *= alpha;
-            lx *= alpha;
+          const float mt =
+              max3f(m0, m1, fmaxf(__uint_as_float(r[62]), __uint_as_float(r[63]))) * sl2;
+          const bool raise = mt > m + 8.0f;
+          if (__any_sync(0xffffffffu, raise)) {
+            // O holds this group's products of the item's earlier steps; rows
+            // that kept nothing yet (m = -inf) hold zeros and need no rescale
+            if (j > 0 && __any_sync(0xffffffffu, raise && m != -INFINITY)) {
+              // the product of step n - 1 completes before O is touched (the
+              // barrier of steps of that parity: its phase n - 3 arrived before
+              // S(n - 1)'s, which this group has seen, so the parity is exact)
+              const int pm = n - 1;
+              ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_done[grp][pm & 1], (pm >> 1) & 1,
+                                                     &abort_sh, a.status, kWaitLimitNs));
+              if (!ok) break;
+              tc_fence_after();
+              const float alpha = (raise && m != -INFINITY) ? ex2_approx(m - mt) : 1.0f;
 #pragma unroll 1
-            for (int c = 0; c < D / 16; ++c) {
-              uint32_t ov[16];
-              tmem_ld16(ocol + c * 16, ov);
-              tmem_wait_ld();
+              for (int c = 0; c < D / 16; ++c) {
+                uint32_t ov[16];
+                tmem_ld16(ocol_own + c * 16, ov);
+                tmem_wait_ld();
 #pragma unroll
-              for (int x = 0; x < 16; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
-              tmem_st16(ocol + c * 16, ov);
+                for (int x = 0; x < 16; ++x)
+                  ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
+                tmem_st16(ocol_own + c * 16, ov);
+              }
+              tmem_wait_st();
+              l *= alpha;
+              lx *= alpha;
             }
-            tmem_wait_st();
+            if (raise) m = mt;
           }
-          if (raise) m = mt;
-        }
-        // P = exp2(S * scale * log2e - m) on a kept half, 0 otherwise (a kept
-        // half always has a finite reference here: its own maximum raised it);
-        // bf16 pairs over S's first 64 columns; l sums the rounded weights, each
-        // bf16 half added to an fp32 sum by one mixed-precision add (x = s *
-        // scale_log2 - m packed in pairs)
-        const uint64_t sl2x2 = pack2(sl2, sl2), nmx2 = pack2(-m, -m);
-        float rsa = 0.f, rsb = 0.f;  // row sums of the rounded weights (low, high halves)
-        uint64_t rx2 = pack2(0.f, 0.f);
+          // P = exp2(S * scale * log2e - m) in bf16 pairs; l sums the rounded
+          // weights, each bf16 half added to an fp32 sum by one mixed-precision
+          // add (x = s * scale_log2 - m packed in pairs)
+          const uint64_t sl2x2 = pack2(sl2, sl2), nmx2 = pack2(-m, -m);
+          float rsa = 0.f, rsb = 0.f;  // row sums of the rounded weights (low, high halves)
+          uint64_t rx2 = pack2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {  // 32 weights -> 16 packed columns at a time
-          const bool kp = c < 2 ? keep0 : keep1;
-          uint32_t pw[16];
-          if (kp) {
-#pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const float2 xv = unpack2(fma2(
-                  pack2(__uint_as_float(r[32 * c + x]), __uint_as_float(r[32 * c + x + 1])), sl2x2,
-                  nmx2));
-              const float p0 = ex2_approx(xv.x), p1 = ex2_approx(xv.y);
-              __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
-              const uint32_t u = *reinterpret_cast<uint32_t*>(&pk);
-              asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-                  "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
-                  : "+f"(rsa), "+f"(rsb) : "r"(u));
-              if constexpr (kLse) rx2 = add2(rx2, pack2(p0, p1));
-              pw[x / 2] = u;
-            }
-          } else {
-#pragma unroll
-            for (int x = 0; x < 16; ++x) pw[x] = 0u;
+          for (int x = 0; x < 64; x += 2) {
+            const float2 xv = unpack2(
+                fma2(pack2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])), sl2x2, nmx2));
+            const float p0 = ex2_approx(xv.x), p1 = ex2_approx(xv.y);
+            __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+            const uint32_t u = *reinterpret_cast<uint32_t*>(&pk);
+            asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+                "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+                : "+f"(rsa), "+f"(rsb) : "r"(u));
+            if constexpr (kLse) rx2 = add2(rx2, pack2(p0, p1));
+            pw[x / 2] = u;
           }
-          tmem_st16(scol + 16 * c, pw);
-          if (kSplitPV && c == 1) {
-            // keys 0..63 are ready for their half of the PV product
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.p_half);
-          }
-        }
-        {
           const float2 b2 = unpack2(rx2);
           l += rsa + rsb;
           lx += b2.x + b2.y;
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) pw[x] = 0u;
         }
+        tmem_st16(scol, *reinterpret_cast<uint32_t(*)[16]>(&pw[0]));
+        tmem_st16(scol + 16, *reinterpret_cast<uint32_t(*)[16]>(&pw[16]));
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full);
+        if (lane == 0) mbar_arrive(&bars.p_ready[grp][n & 1]);
       }
       if (!ok) break;
       // --------------------------------------------------------- epilogue
+      // every product of the item has completed; the groups swap their row
+      // maxima and sums, then each merges and writes half of O's columns
       ok = __all_sync(0xffffffffu,
                       mbar_wait(&bars.o_full, k & 1, &abort_sh, a.status, kWaitLimitNs));
       if (!ok) break;
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      xm[grp][row] = m;
+      xl[grp][row] = l;
+      xlx[grp][row] = lx;
+      ok = __all_sync(0xffffffffu, group_sync(&bars.xch, xuses, &abort_sh, a.status, kWaitLimitNs));
+      if (!ok) break;
+      const float m2 = xm[1 - grp][row], l2 = xl[1 - grp][row], lx2 = xlx[1 - grp][row];
+      const float mf = fmaxf(m, m2);
+      const float a_own = m != -INFINITY ? ex2_approx(m - mf) : 0.f;
+      const float a_oth = m2 != -INFINITY ? ex2_approx(m2 - mf) : 0.f;
+      const float lt = l * a_own + l2 * a_oth;
+      const float inv = lt > 0.f ? 1.0f / lt : 0.f;
+      const float s_own = a_own * inv, s_oth = a_oth * inv;
       // O / l as bf16, 32 columns at a time through this warp's staging box
       // (row `lane` holds its 64 bytes as four 16-byte chunks, chunk x at
       // x ^ ((lane / 2) % 4): the 64-byte swizzle), then one tensor store per
       // box; rows past L are clipped by the store
       const int tok0 = tok - lane;  // first token of this warp's 32 rows
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld32(ocol + c * 32, ov);
+      for (int c = grp * (D / 64); c < (grp + 1) * (D / 64); ++c) {
+        uint32_t ov[32], ow[32];
+        tmem_ld32(ocol_own + c * 32, ov);
+        tmem_ld32(ocol_oth + c * 32, ow);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(ov[2 * x]) * inv,
-                                                   __uint_as_float(ov[2 * x + 1]) * inv);
+          const float o0 = __uint_as_float(ov[2 * x]) * s_own + __uint_as_float(ow[2 * x]) * s_oth;
+          const float o1 =
+              __uint_as_float(ov[2 * x + 1]) * s_own + __uint_as_float(ow[2 * x + 1]) * s_oth;
+          __nv_bfloat162 v = __floats2bfloat162_rn(o0, o1);
           pk[x] = *reinterpret_cast<uint32_t*>(&v);
         }
         if (lane == 0) bulk_wait_read_all();  // the previous box has been read out
@@ -749,10 +851,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
-      if (a.lse && tok < a.L)
+      if (lane == 0) {
+        mbar_arrive(&bars.o_empty);
+        mbar_arrive(&bars.list_empty[slot]);
+      }
+      if (kLse && grp == 0 && a.lse && tok < a.L) {
+        const float lxt = lx * a_own + lx2 * a_oth;
         a.lse[((int64_t)b * a.H + h) * a.L + tok] =
-            lx > 0.f ? (m + log2f(lx)) * 0.69314718055994531f : -INFINITY;
+            lxt > 0.f ? (mf + log2f(lxt)) * 0.69314718055994531f : -INFINITY;
+      }
     }
     if (lane == 0) bulk_wait_all();  // this warp's output stores have completed
     __syncwarp();
@@ -767,10 +874,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     tmem_dealloc(tmem, kTmemCols);
   }
   if (threadIdx.x == 0) {
-    // this CTA takes no more items; the last one out resets the counter
+    // this CTA takes no more items; the last one out checks the counter and
+    // resets it for a later launch
     __threadfence();
     if (atomicAdd(&g_sched[sched_slot].finished, 1u) == gridDim.x - 1) {
-      atomicExch(&g_sched[sched_slot].next, 0u);
+      const unsigned taken = atomicExch(&g_sched[sched_slot].next, 0u);
+      if (!(*(volatile int*)a.status & kDevTimeout) && taken != (unsigned)n_items + gridDim.x)
+        atomicOr(a.status, kDevOverlap);
       atomicExch(&g_sched[sched_slot].finished, 0u);
     }
   }
@@ -821,9 +931,9 @@ cudaError_t launch_attn_tc(const AttnArgs& a, const CUtensorMap* tq, const CUten
     e = cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
   }
-  // persistent CTAs, two per SM, each running one tile at a time
+  // persistent CTAs, one per SM
   const int64_t n_items = (int64_t)a.B * a.H * ((a.L + kBM - 1) / kBM);
-  const int64_t cap = (int64_t)kCtasPerSm * g_num_sms[dev];
+  const int64_t cap = (int64_t)g_num_sms[dev];
   const int grid = (int)(n_items < cap ? n_items : cap);
   if (a.d == 128)
     return a.lse ? launch_tc<128, true>(a, tq, tk, tv, to, st, grid, dev)

@@ -11,7 +11,8 @@
 namespace sdl {
 
 // Device status word bits (set by kernels, read by sdl_last_device_status).
-enum : int { kDevTimeout = 1, kDevBadMask = 2 };
+// kDevOverlap: two attention launches in flight shared one tile counter.
+enum : int { kDevTimeout = 1, kDevBadMask = 2, kDevOverlap = 4 };
 
 // Wall-time bound for every spin wait inside a kernel.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

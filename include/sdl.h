@@ -18,7 +18,9 @@
  *     one status word, the fixed scratch array of sdl_select_mask_noalloc,
  *     and a ring of 64 tile counters for the attention kernels (each launch
  *     takes the next one and its last CTA resets it, so at most 64 attention
- *     launches may be in flight on one device at a time).
+ *     launches may be in flight on one device at a time; a launch that found
+ *     its counter shared is reported as SDL_ERR_OVERLAP by
+ *     sdl_last_device_status).
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL is the legacy default stream).  Argument errors are returned
  *     before anything is launched; a launch failure returns SDL_ERR_CUDA and
@@ -26,7 +28,9 @@
  *   - Q is [B, L, H, d], K and V are [B, L, H_kv, d] and O is [B, L, H, d],
  *     each addressed through element strides (b, t, h) with d contiguous.
  *   - bf16 tensors must start on 16-byte boundaries and have strides that are
- *     multiples of 8 elements (the tensor-memory-access unit's rule).
+ *     multiples of 8 elements (the tensor-memory-access unit's rule); a zero
+ *     stride (a broadcast view) is refused on any axis with more than one
+ *     index (SDL_ERR_INVALID_ARG).
  *   - No exception or abort crosses the ABI.
  */
 #ifndef SDL_H
@@ -47,7 +51,9 @@ typedef enum {
   SDL_ERR_WORKSPACE = 4,   /* workspace null or smaller than required */
   SDL_ERR_CUDA = 5,        /* a CUDA call failed; see sdl_last_cuda_error() */
   SDL_ERR_TIMEOUT = 6,     /* a kernel's bounded wait ran out (device status) */
-  SDL_ERR_BAD_MASK = 7     /* a col_idx entry out of range or out of order */
+  SDL_ERR_BAD_MASK = 7,    /* a col_idx entry out of range or out of order */
+  SDL_ERR_OVERLAP = 8      /* two attention launches in flight shared a tile counter
+                              (device status; their outputs are not trustworthy) */
 } sdl_status;
 
 typedef enum { SDL_BF16 = 0, SDL_FP32 = 1 } sdl_dtype;
@@ -340,7 +346,10 @@ sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl
 
 /* Synchronizes `stream`, then reports and clears the device status word set by
  * kernels: SDL_ERR_TIMEOUT if a bounded wait ran out, SDL_ERR_BAD_MASK if a
- * list entry was rejected, SDL_OK otherwise. */
+ * list entry was rejected, SDL_ERR_OVERLAP if more bf16 attention launches
+ * were in flight at once than there are tile counters (the last CTA of each
+ * launch checks its counter's final count), SDL_OK otherwise; the first of
+ * these in that order when several bits are set. */
 sdl_status sdl_last_device_status(void* stream);
 
 /* Self-check of the failure path: launches one warp that waits, through the

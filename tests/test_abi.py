@@ -91,9 +91,42 @@ def test_shape_validation():
     assert rc == sdl.SDL_ERR_INVALID_ARG
 
 
+def test_zero_strides_refused_on_axes_with_more_than_one_index():
+    """A broadcast view (stride 0 along tokens, heads or batch) would make distinct
+    rows alias one address; every call taking Q/K/V/O refuses it before any launch."""
+    import torch
+    lib = sdl.lib()
+    P = ctypes.c_void_p
+    q = torch.zeros(2, 512, 4, 64, dtype=torch.bfloat16)
+    k1 = torch.zeros(2, 512, 1, 64, dtype=torch.bfloat16)
+    k = k1.expand(2, 512, 4, 64)          # stride 0 along the 4 KV heads
+    assert k.stride(2) == 0
+    shp = sdl.make_shape(q, k, 64)
+    assert shp.k_strides[2] == 0
+    rc = lib.sdl_dense_attn(P(16), P(16), P(16), ctypes.byref(shp), 0.0, P(16), None, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+    rc = lib.sdl_sparse_attn(P(16), P(16), P(16), ctypes.byref(shp), P(16), P(16), 0.0, P(16),
+                             None, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+    # stride 0 along tokens of V, and along the batch of O
+    for field, axis in (("v_strides", 1), ("o_strides", 0)):
+        bad = sdl.make_shape(q, k1.expand(2, 512, 4, 64).contiguous(), 64)
+        getattr(bad, field)[axis] = 0
+        rc = lib.sdl_dense_attn(P(16), P(16), P(16), ctypes.byref(bad), 0.0, P(16), None, None)
+        assert rc == sdl.SDL_ERR_INVALID_ARG, field
+    # an axis of one index may carry any stride: the stride check passes and the
+    # call stops at the next host check (no workspace), never reaching a launch
+    one = sdl.make_shape(q[:1], k1[:1].expand(1, 512, 4, 64).contiguous(), 64)
+    one.q_strides[0] = 0
+    rc = lib.sdl_block_scores(P(16), P(16), ctypes.byref(one), 0.0, P(16), None, 0, None)
+    assert rc == sdl.SDL_ERR_WORKSPACE
+    rc = lib.sdl_block_scores(P(16), P(16), ctypes.byref(shp), 0.0, P(16), None, 0, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+
+
 def test_status_strings():
     lib = sdl.lib()
-    for code in range(8):
+    for code in range(9):
         assert lib.sdl_status_string(code)
     assert lib.sdl_last_cuda_error() == 0
 
