@@ -353,7 +353,81 @@ def traffic_record():
 # ------------------------------------------------------------- cpu oracle
 
 
-def cpu_oracle_sample(w, seed, target_s=8.0):
+def csr_mask(row_ptr: np.ndarray, col_idx: np.ndarray, B: int, H: int, nb: int) -> np.ndarray:
+    """uint8 [B, H, nb, nb] block mask of a CSR list."""
+    rows = np.repeat(np.arange(B * H * nb), np.diff(row_ptr))
+    mask = np.zeros((B * H * nb, nb), dtype=np.uint8)
+    mask[rows, col_idx[:row_ptr[-1]]] = 1
+    return mask.reshape(B, H, nb, nb)
+
+
+def parity_check(runner, w, seed, step, out, n_random=2, rows_per_block=4):
+    """Outside the timed region: the output of timed step `step` (`out`, on the
+    device) on sampled query rows against the fp64 oracle with the GPU's own mask
+    (all heads; per head the first and last query block, the block with the
+    longest kept list and `n_random` others), and the GPU's mask of that step's
+    anchor against the oracle's selection (differences allowed only within 1e-5
+    relative of the oracle's threshold, and counted).  Attention under the
+    oracle's own mask on the same rows is reported beside it, not checked."""
+    import oracle
+    import synth
+    rt = runner.rt
+    if runner.pulsecol or runner.shard is not None:
+        return None
+    nb, H = w.nb, w.H
+    host = synth.host_inputs(w, step, seed)
+    a_step = rt.anchor_of(step, runner.interval, runner.dense_steps)
+    rng = np.random.default_rng(seed + 1)
+    res = {"step": step, "anchor_step": a_step}
+    if a_step is None:  # a dense step of the sparsed schedule
+        gpu_mask = None
+        lens = np.full((w.B, H, nb), nb)
+    else:
+        rp = runner.att.row_ptr.cpu().numpy()
+        ci = runner.att.col_idx.cpu().numpy()
+        gpu_mask = csr_mask(rp, ci, w.B, H, nb)
+        lens = np.diff(rp).reshape(w.B, H, nb)
+        ha = host if a_step == step else synth.host_inputs(w, a_step, seed)
+        P = oracle.block_scores(ha["q"], ha["k"], w.bs)
+        want, tau, kept = oracle.select(P, w.sparsity, per_head=runner.att.per_head)
+        diff = np.argwhere(gpu_mask != want)
+        taus = tau.reshape(w.B, -1)
+        near = 0
+        for b, h, i, j in diff:
+            t_b = taus[b, h if runner.att.per_head else 0]
+            if i != j and abs(P[b, h, i, j] - t_b) <= 1e-5 * t_b:
+                near += 1
+        res.update({"mask_blocks": int(gpu_mask.sum()), "oracle_blocks": kept,
+                    "mask_entries_near_threshold": near,
+                    "mask_entries_other": int(len(diff) - near)})
+    rows = []
+    for b in range(w.B):
+        for h in range(H):
+            blocks = {0, nb - 1, int(np.argmax(lens[b, h]))}
+            blocks |= set(int(x) for x in rng.integers(nb, size=n_random))
+            for i in sorted(blocks):
+                ts = {i * w.bs, i * w.bs + w.bs - 1}
+                ts |= set(int(i * w.bs + x) for x in rng.integers(w.bs, size=rows_per_block))
+                rows.extend((b, h, t) for t in sorted(ts))
+    rows = np.array(rows, dtype=np.int64)
+    idx = torch.as_tensor(rows, device=out.device)
+    got = out[idx[:, 0], idx[:, 2], idx[:, 1]].float().cpu().numpy().astype(np.float64)
+    want_o, _ = oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=gpu_mask, rows=rows)
+    err = np.abs(got - want_o)
+    tol_max, tol_mean = (1e-2, 1e-3) if w.dtype == "bf16" else (1e-4, 1e-4)
+    res.update({"rows": int(len(rows)), "max_abs": float(err.max()),
+                "mean_abs": float(err.mean()), "tol_max_abs": tol_max,
+                "tol_mean_abs": tol_mean, "finite": bool(np.isfinite(got).all())})
+    res["ok"] = bool(res["finite"] and res["max_abs"] <= tol_max and res["mean_abs"] <= tol_mean
+                     and res.get("mask_entries_other", 0) == 0)
+    if gpu_mask is not None:
+        own, _ = oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=want, rows=rows)
+        res["oracle_mask_max_abs"] = float(np.abs(got - own).max())
+    return res
+
+
+
+def cpu_oracle_sample(w, seed, target_s=20.0):
     """Times the fp64 oracle's block-sparse attention on a bounded sample of the
     workload's query rows (all heads, evenly spaced query blocks) of step 0 with
     its anchor mask; returns (TFLOP/s, cores, description, sample seconds, extra)
@@ -387,9 +461,14 @@ def cpu_oracle_sample(w, seed, target_s=8.0):
     t0 = time.perf_counter()
     oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=mask, rows=rows, nthreads=cores)
     dt = time.perf_counter() - t0
-    desc = (f"block-sparse attention of {len(rows)} query rows ({nblk} of {nb} query blocks x "
-            f"{w.H} heads, step 0 with its anchor mask), fp64, {cores} threads")
-    extra = {"anchor_s": anchor_s, "full_step_s_extrapolated": dt * nb / nblk}
+    what = "one full step" if nblk == nb else f"{nblk} of {nb} query blocks x {w.H} heads"
+    desc = (f"block-sparse attention of {len(rows)} query rows ({what}, step 0 with its "
+            f"anchor mask), fp64, {cores} threads")
+    extra = {"anchor_s": anchor_s}
+    if nblk == nb:
+        extra["full_step_s"] = dt
+    else:
+        extra["full_step_s_extrapolated"] = dt * nb / nblk
     return flops(rows) / dt / 1e12, cores, desc, dt, extra
 
 
@@ -504,6 +583,11 @@ def main():
             break
         sampler = ClockSampler(local)
     ms_max = max_over_ranks(ms, dist_on, device)
+    # outside the timed region: the device status word, and the last timed
+    # step's output kept for the parity check (later launches reuse the buffer)
+    sdl = runner.sdl
+    status_timed = sdl.last_device_status()
+    last_out = runner.out.clone()
 
     pk, pk_kind = peaks()
     budget = runner.att.budget  # kept blocks of the whole sequence
@@ -528,7 +612,6 @@ def main():
     peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
 
     # anchor-step kernels, timed apart: scoring bandwidth and selection latency
-    sdl = runner.sdl
     x0 = inputs[0]
 
     def ev_time(fn, n=10):
@@ -572,6 +655,11 @@ def main():
         e_ms = max_over_ranks(e_ms, dist_on, device)
         e2e = {"value": job_rate(flop_step, len(steps), seqs, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e_ms / len(steps)}
+    status_after = sdl.last_device_status()  # the e2e loop and the separate timings
+
+    parity = None
+    if rank == 0 and not heads:
+        parity = parity_check(runner, w, seed, steps[-1], last_out)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -626,12 +714,20 @@ def main():
                              w.bs, runner.att.sharded, runner.att.fused,
                              runner.att.lists is not None)),
         "clocks": sampler.summary(),
+        "device_status": {"timed": status_timed, "after": status_after},
+        "parity": parity,
     }
     if rank == 0:
         print(json.dumps(line))
     if dist_on:
         import torch.distributed as dist
         dist.destroy_process_group()
+    # a kernel that reported a timeout or a rejected list entry, or an output
+    # off the oracle, voids the line's numbers
+    if status_timed != sdl.SDL_OK or status_after != sdl.SDL_OK:
+        sys.exit(3)
+    if parity is not None and not parity["ok"]:
+        sys.exit(4)
 
 
 if __name__ == "__main__":

@@ -82,6 +82,9 @@ constexpr int kOBoxBytes = 32 * 64;  // one 32-row x 32-column bf16 output box
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;    // S buffer b at kColS + 128 b
 constexpr uint32_t kColO = 256;  // O of group g at kColO + 128 g
+// The reference maximum of a row is raised (and O rescaled) only when the
+// tile maximum exceeds it by more than this many log2 units.
+constexpr float kRaiseLog2 = 16.0f;
 
 template <int D>
 struct Layout {
@@ -371,6 +374,39 @@ __global__ void __launch_bounds__(kListWarps * 32) tile_lists_kernel(AttnArgs a,
   }
 }
 
+
+// Maximum of 32 fp32 logits (three-input max).
+__device__ __forceinline__ float max32(const uint32_t* r) {
+  float m0 = __uint_as_float(r[0]), m1 = __uint_as_float(r[1]);
+#pragma unroll
+  for (int x = 2; x < 30; x += 4) {
+    m0 = max3f(m0, __uint_as_float(r[x]), __uint_as_float(r[x + 1]));
+    m1 = max3f(m1, __uint_as_float(r[x + 2]), __uint_as_float(r[x + 3]));
+  }
+  return max3f(m0, m1, fmaxf(__uint_as_float(r[30]), __uint_as_float(r[31])));
+}
+
+// Softmax weights of 32 logits: p = exp2(s * scale_log2 - m) (x packed in
+// pairs), rounded to bf16 pairs into pw[0..15]; rsa / rsb sum the rounded
+// weights, each bf16 half added to an fp32 sum by one mixed-precision add;
+// rx2 sums the unrounded ones (the LSE's).
+template <bool kLse>
+__device__ __forceinline__ void weights32(const uint32_t* r, uint64_t sl2x2, uint64_t nmx2,
+                                          uint32_t* pw, float& rsa, float& rsb, uint64_t& rx2) {
+#pragma unroll
+  for (int x = 0; x < 32; x += 2) {
+    const float2 xv =
+        unpack2(fma2(pack2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])), sl2x2, nmx2));
+    const float p0 = ex2_approx(xv.x), p1 = ex2_approx(xv.y);
+    __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+    const uint32_t u = *reinterpret_cast<uint32_t*>(&pk);
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(rsa), "+f"(rsb) : "r"(u));
+    if constexpr (kLse) rx2 = add2(rx2, pack2(p0, p1));
+    pw[x / 2] = u;
+  }
+}
 
 template <int D, bool kLse>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -720,21 +756,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t scol = trow + kColS + 128u * (uint32_t)(n & 1) + 64u * grp;
         uint32_t pw[32];
         if (keep) {
+          // S in two 32-column chunks: the second loads while the first is
+          // turned into weights
           uint32_t r[64];
           tmem_ld32(scol + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
-          // tile maximum (three-input max)
-          float m0 = __uint_as_float(r[0]), m1 = __uint_as_float(r[1]);
-#pragma unroll
-          for (int x = 2; x < 62; x += 4) {
-            m0 = max3f(m0, __uint_as_float(r[x]), __uint_as_float(r[x + 1]));
-            m1 = max3f(m1, __uint_as_float(r[x + 2]), __uint_as_float(r[x + 3]));
+          tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          const uint64_t sl2x2 = pack2(sl2, sl2);
+          float rsa = 0.f, rsb = 0.f;  // row sums of the rounded weights (low, high halves)
+          uint64_t rx2 = pack2(0.f, 0.f);
+          // (warp-uniform: a warp's rows share their keep bits, so either all
+          // or none of them have kept a block of this item yet)
+          const bool first = __any_sync(0xffffffffu, m == -INFINITY);
+          float mt;
+          if (first) {
+            tmem_wait_ld();
+            mt = fmaxf(max32(r), max32(r + 32)) * sl2;
+          } else {
+            // weights against the current reference while the tile maximum is
+            // found alongside; they stand unless the maximum grew by more than 8
+            const uint64_t nmx2 = pack2(-m, -m);
+            weights32<kLse>(r, sl2x2, nmx2, pw, rsa, rsb, rx2);
+            const float m0 = max32(r);
+            tmem_st16(scol, *reinterpret_cast<uint32_t(*)[16]>(&pw[0]));
+            tmem_wait_ld();
+            weights32<kLse>(r + 32, sl2x2, nmx2, pw + 16, rsa, rsb, rx2);
+            mt = fmaxf(m0, max32(r + 32)) * sl2;
           }
-          const float mt =
-              max3f(m0, m1, fmaxf(__uint_as_float(r[62]), __uint_as_float(r[63]))) * sl2;
-          const bool raise = mt > m + 8.0f;
-          if (__any_sync(0xffffffffu, raise)) {
+          const bool raise = mt > m + kRaiseLog2;
+          if (first || __any_sync(0xffffffffu, raise)) {
             // O holds this group's products of the item's earlier steps; rows
             // that kept nothing yet (m = -inf) hold zeros and need no rescale
             if (j > 0 && __any_sync(0xffffffffu, raise && m != -INFINITY)) {
@@ -757,30 +807,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                   ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
                 tmem_st16(ocol_own + c * 16, ov);
               }
-              tmem_wait_st();
               l *= alpha;
               lx *= alpha;
             }
             if (raise) m = mt;
-          }
-          // P = exp2(S * scale * log2e - m) in bf16 pairs; l sums the rounded
-          // weights, each bf16 half added to an fp32 sum by one mixed-precision
-          // add (x = s * scale_log2 - m packed in pairs)
-          const uint64_t sl2x2 = pack2(sl2, sl2), nmx2 = pack2(-m, -m);
-          float rsa = 0.f, rsb = 0.f;  // row sums of the rounded weights (low, high halves)
-          uint64_t rx2 = pack2(0.f, 0.f);
-#pragma unroll
-          for (int x = 0; x < 64; x += 2) {
-            const float2 xv = unpack2(
-                fma2(pack2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])), sl2x2, nmx2));
-            const float p0 = ex2_approx(xv.x), p1 = ex2_approx(xv.y);
-            __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
-            const uint32_t u = *reinterpret_cast<uint32_t*>(&pk);
-            asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-                "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
-                : "+f"(rsa), "+f"(rsb) : "r"(u));
-            if constexpr (kLse) rx2 = add2(rx2, pack2(p0, p1));
-            pw[x / 2] = u;
+            // the weights against the (new) reference
+            const uint64_t nmx2 = pack2(-m, -m);
+            rsa = rsb = 0.f;
+            rx2 = pack2(0.f, 0.f);
+            weights32<kLse>(r, sl2x2, nmx2, pw, rsa, rsb, rx2);
+            weights32<kLse>(r + 32, sl2x2, nmx2, pw + 16, rsa, rsb, rx2);
+            tmem_wait_st();  // an earlier store of the first chunk lands before this one
+            tmem_st16(scol, *reinterpret_cast<uint32_t(*)[16]>(&pw[0]));
           }
           const float2 b2 = unpack2(rx2);
           l += rsa + rsb;
@@ -788,8 +826,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int x = 0; x < 32; ++x) pw[x] = 0u;
+          tmem_st16(scol, *reinterpret_cast<uint32_t(*)[16]>(&pw[0]));
         }
-        tmem_st16(scol, *reinterpret_cast<uint32_t(*)[16]>(&pw[0]));
         tmem_st16(scol + 16, *reinterpret_cast<uint32_t(*)[16]>(&pw[16]));
         tmem_wait_st();
         tc_fence_before();

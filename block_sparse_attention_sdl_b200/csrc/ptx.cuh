@@ -115,24 +115,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x >= -125 after clamping (smaller inputs give
-// 2^-125, which is 0 for every use here).  x = n + f with n = round(x) taken
-// from the low mantissa bits of x + 1.5 * 2^23, f in [-1/2, 1/2]; 2^f is a
-// cubic fitted in relative error at Chebyshev nodes (csrc/exp2_poly.py, max
-// relative error 7.7e-5); 2^n is added to the exponent field.  Valid for
-// x < 128; larger x are only ever produced for results that get discarded.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  float p = fmaf(f, 0x1.c34958p-5f, 0x1.f0da64p-3f);
-  p = fmaf(p, f, 0x1.62f51ap-1f);
-  p = fmaf(p, f, 0x1.fff6b0p-1f);
-  const int j = __float_as_int(t) - 0x4B400000;
-  return __int_as_float(__float_as_int(p) + (j << 23));
-}
-
 // ---------------------------------------------------------------------- TMA
 
 // 4-D tiled bulk tensor load into this CTA's own shared memory (no other CTA
@@ -363,32 +345,12 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// exp2_poly on a pair, with the pair arithmetic packed (see exp2_poly).
-__device__ __forceinline__ float2 exp2_poly2(float x0, float x1) {
-  const uint64_t x = pack2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t C = pack2(12582912.0f, 12582912.0f);
-  const uint64_t t = add2(x, C);
-  const uint64_t f = sub2(x, sub2(t, C));
-  uint64_t p = fma2(f, pack2(0x1.c34958p-5f, 0x1.c34958p-5f), pack2(0x1.f0da64p-3f, 0x1.f0da64p-3f));
-  p = fma2(p, f, pack2(0x1.62f51ap-1f, 0x1.62f51ap-1f));
-  p = fma2(p, f, pack2(0x1.fff6b0p-1f, 0x1.fff6b0p-1f));
-  const float2 tp = unpack2(t), pp = unpack2(p);
-  const int j0 = __float_as_int(tp.x) - 0x4B400000, j1 = __float_as_int(tp.y) - 0x4B400000;
-  return make_float2(__int_as_float(__float_as_int(pp.x) + (j0 << 23)),
-                     __int_as_float(__float_as_int(pp.y) + (j1 << 23)));
 }
 
 }  // namespace sdl

@@ -41,3 +41,58 @@ def test_traffic_record_follows_the_kernel_source(tmp_path, monkeypatch):
     assert bench.traffic_record() is None
     os.remove(tmp_path / "profiles" / "sparse_attn_traffic.json")
     assert bench.traffic_record() is None
+
+
+def test_csr_mask_matches_a_dense_mask():
+    import numpy as np
+    rng = np.random.default_rng(3)
+    B, H, nb = 2, 3, 5
+    want = (rng.random((B, H, nb, nb)) < 0.4).astype(np.uint8)
+    rows = want.reshape(-1, nb)
+    row_ptr = np.concatenate([[0], np.cumsum(rows.sum(1))]).astype(np.int32)
+    col_idx = np.concatenate([np.flatnonzero(r) for r in rows]).astype(np.int32)
+    assert np.array_equal(bench.csr_mask(row_ptr, col_idx, B, H, nb), want)
+
+
+class _FakeAtt:
+    def __init__(self, row_ptr, col_idx):
+        import torch
+        self.row_ptr, self.col_idx = torch.as_tensor(row_ptr), torch.as_tensor(col_idx)
+        self.per_head = False
+
+
+class _FakeRunner:
+    """What parity_check reads from the bench's runner, on the CPU."""
+
+    def __init__(self, att, interval):
+        from block_sparse_attention_sdl_b200 import runtime
+        self.rt, self.att, self.interval, self.dense_steps = runtime, att, interval, 0
+        self.pulsecol, self.shard = False, None
+
+
+def test_parity_check_passes_the_oracle_output_and_catches_a_wrong_one():
+    """The bench's self-check: an output equal to the oracle's (rounded to bf16) with
+    the oracle's own mask passes; the same output with one row perturbed fails."""
+    import numpy as np
+    import torch
+    import oracle
+    import synth
+    w = synth.small_workload(L=512, H=2, H_kv=1, d=64, sparsity=0.5, planted=1, steps=3,
+                             anchor_every=2)
+    step = 2  # an anchor step: its own mask
+    host = synth.host_inputs(w, step)
+    P = oracle.block_scores(host["q"], host["k"], w.bs)
+    mask, _, kept = oracle.select(P, w.sparsity)
+    rows = mask.reshape(-1, w.nb)
+    row_ptr = np.concatenate([[0], np.cumsum(rows.sum(1))]).astype(np.int32)
+    col_idx = np.concatenate([np.flatnonzero(r) for r in rows]).astype(np.int32)
+    O, _ = oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=mask)
+    out = torch.as_tensor(O.transpose(0, 2, 1, 3).copy()).to(torch.bfloat16)  # [B, L, H, d]
+    runner = _FakeRunner(_FakeAtt(row_ptr, col_idx), w.anchor_every)
+    res = bench.parity_check(runner, w, 0, step, out)
+    assert res["ok"], res
+    assert res["mask_entries_other"] == 0 and res["mask_blocks"] == kept
+    assert res["max_abs"] < 1e-2 and res["oracle_mask_max_abs"] == res["max_abs"]
+    bad = out.clone()
+    bad[0, w.L - 1, 1] += 0.05   # the last row of the last query block is always sampled
+    assert not bench.parity_check(runner, w, 0, step, bad)["ok"]
