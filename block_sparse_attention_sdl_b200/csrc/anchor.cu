@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kAnchorThreads, 1) anchor_kernel(AnchorArgs a)
     a.ws.hist[x] = 0;
 
   // ---- block means of Q and K
-  pool_body<T>(a.tq, a.tk, a.B, a.L, a.d, a.bs, blockIdx.x, nblk);
+  pool_body<T, 16, true>(a.tq, a.tk, a.B, a.L, a.d, a.bs, blockIdx.x, nblk);
   if (!grid_barrier(a, 0, &give_up)) return;
 
   // ---- pooled products and row softmax: items (query-block tile, head, batch)
