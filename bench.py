@@ -696,6 +696,10 @@ def main():
         "speedup_vs_dense": dense_ms / sp_avg,
         "speedup_vs_dense_amortized": dense_ms / (ms_max / len(steps)),
         "anchor_ms": statistics.mean(anchor_ms) if anchor_ms else None,
+        # the first anchor is issued into an idle queue right after the timing
+        # barrier; the later ones behind the previous steps' attention launches
+        "anchor_ms_first": anchor_ms[0] if anchor_ms else None,
+        "anchor_ms_steady": statistics.mean(anchor_ms[1:]) if len(anchor_ms) > 1 else None,
         "block_scores_ms": sc_ms,
         "block_scores_gbs": None if runner.pulsecol else score_bytes / (sc_ms * 1e-3) / 1e9,
         "select_mask_ms": se_ms, "mask_blocks": budget,

@@ -238,9 +238,13 @@ sdl_status sdl_select_shard_finish(const float* scores, const sdl_shape* local,
  * library until exit).  Problems needing more scratch than that
  * (sdl_select_workspace_bytes > 2 MiB) return SDL_ERR_WORKSPACE without launching.
  * The first call on each device looks up the array's device address; make it
- * before any stream capture.  Nothing is allocated by any call.  All calls share
- * the array: calls that may overlap on the GPU (other streams, other threads)
- * race and must be serialized by the caller. */
+ * before any stream capture.  The array used is the one of the current device:
+ * `stream` must belong to the device that is current when the call is made.
+ * The looked-up address is kept for the life of the process, so it is not
+ * valid after a cudaDeviceReset (the same holds for the device status word
+ * behind sdl_last_device_status).  Nothing is allocated by any call.  All calls
+ * share the array: calls that may overlap on the GPU (other streams, other
+ * threads) race and must be serialized by the caller. */
 sdl_status sdl_select_mask_noalloc(const float* scores, const sdl_shape* shape, double sparsity,
                                    int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
                                    uint8_t* mask_u8, void* stream);

@@ -179,6 +179,46 @@ def test_sparse_attention(dtype, B, L, H, Hkv, d, bs, density):
     assert np.abs(lse.cpu().numpy() - lw).max() <= TOL[dtype]["lse"]
 
 
+@pytest.mark.parametrize("kind", ["dense", "sparse"])
+def test_sharp_logits_raise_the_reference_within_and_across_tiles(kind):
+    """Sharpness 16 to 48 per head: along an item's key blocks the maximum logit
+    grows past the running reference by more than the lazy-rescale threshold
+    (16 in log2 units), so the raise path runs (the step's weights redone against
+    the new reference, O and the row sums rescaled in TMEM), and weights come
+    close to 2^16 where the reference lags; O and LSE still match the oracle."""
+    B, H, Hkv, L, d, bs = 1, 4, 2, 2048, 128, 64
+    w = synth.Workload("sharp", "bf16", B, H, Hkv, L, d, bs, 0.5, 1, 1, 0.02,
+                       ("fixed", [16.0, 24.0, 32.0, 48.0]), 1)
+    host, dev = _inputs(w)
+    nb = L // bs
+    if kind == "dense":
+        mask = np.ones((B, H, nb, nb), np.uint8)
+    else:
+        mask = _random_mask(B, H, nb, 0.5, np.random.default_rng(11))
+    # the inputs reach the raise path: for rows of query block 0, the logits of
+    # the first kept 64-key block against those of the later kept blocks
+    q = host["q"][0].astype(np.float64)
+    k = host["k"][0].astype(np.float64)
+    growth = 0.0
+    for h in range(H):
+        kept = np.flatnonzero(mask[0, h, 0])
+        x = q[:bs, h] @ k[:, h // (H // Hkv)].T / np.sqrt(d) * np.log2(np.e)
+        first = x[:, kept[0] * bs:(kept[0] + 1) * bs].max(1)
+        later = np.max([x[:, j * bs:(j + 1) * bs].max(1) for j in kept], axis=0)
+        growth = max(growth, float((later - first).max()))
+    assert growth > 2 * 16.0, growth
+    if kind == "dense":
+        O, lse = sdl.dense_attn(dev["q"], dev["k"], dev["v"], want_lse=True)
+        Ow, lw = oracle.attention(host["q"], host["k"], host["v"], bs)
+    else:
+        rp, ci = _mask_to_csr(mask)
+        O, lse = sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, bs, want_lse=True)
+        Ow, lw = oracle.attention(host["q"], host["k"], host["v"], bs, mask=mask)
+    assert sdl.last_device_status() == sdl.SDL_OK
+    check_close(bf16_to_f64(O).transpose(0, 2, 1, 3), Ow, "bf16")
+    assert np.abs(lse.cpu().numpy() - lw).max() <= TOL["bf16"]["lse"]
+
+
 @pytest.mark.parametrize("kind", ["diag", "ones", "single_far"])
 @pytest.mark.parametrize("bs", [64, 128])
 def test_sparse_attention_edge_masks(kind, bs):

@@ -38,7 +38,7 @@ def _check_anchor(att, w, host):
     check_csr(rp, ci, w.B, w.H, w.nb, kept)
     got = csr_to_mask(rp, ci, w.B, w.H, w.nb)
     excused = compare_masks(got, want, P_or, tau)
-    return got, excused
+    return got, excused, want
 
 
 @pytest.mark.parametrize("name,steps", [("fp32-L512-H2-s50", [0, 1, 2, 3]),
@@ -60,7 +60,7 @@ def test_schedule_full_parity(name, steps):
             continue
         host = synth.host_inputs(w, step)
         if w.is_anchor(step):
-            mask, _ = _check_anchor(att, w, host)
+            mask, _, _ = _check_anchor(att, w, host)
         else:
             mask = csr_to_mask(att.row_ptr.cpu().numpy(), att.col_idx.cpu().numpy(), w.B, w.H,
                                w.nb)
@@ -115,12 +115,19 @@ def test_full_size_anchor_and_sampled_rows(name, step):
                    lse=torch.empty((w.B, w.H, w.L), dtype=torch.float32, device="cuda"))
     torch.cuda.synchronize()
     host = synth.host_inputs(w, step)
-    mask, excused = _check_anchor(att, w, host)
+    mask, excused, want = _check_anchor(att, w, host)
     print(f"{name} step {step}: {excused} near-threshold mask differences excused")
     rows = sample_rows(w.B, w.H, w.L, w.bs, mask.sum(-1), n_blocks=4, rows_per_block=8)
     Ow, lw = oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=mask, rows=rows)
     got = bf16_to_f64(out)[rows[:, 0], rows[:, 2], rows[:, 1]]
     check_close(got, Ow, "bf16")
+    # attention under the oracle's own mask on the same rows: reported; where the
+    # two masks agree entirely it must pass the same tolerance
+    Oo, _ = oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=want, rows=rows)
+    err_own = float(np.abs(got - Oo).max())
+    print(f"{name} step {step}: max abs error against the oracle's own mask {err_own:.3e}")
+    if excused == 0:
+        check_close(got, Oo, "bf16", "O under the oracle's mask")
     lse_got = lse.cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
     assert np.abs(lse_got - lw).max() <= TOL["bf16"]["lse"]
     assert sdl.last_device_status() == sdl.SDL_OK
