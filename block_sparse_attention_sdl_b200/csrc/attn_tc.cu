@@ -705,6 +705,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++n;
       }
       ++t;
+      // the item's last products go out now, not behind the next item's first
+      // S product (which waits for that item's Q and K): the epilogue starts as
+      // soon as the softmax has written the last weights
+      if (ok && pend && !(ok = issue_pv())) break;
     }
     if (ok && pend) ok = issue_pv();
     if (leader) {

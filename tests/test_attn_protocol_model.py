@@ -12,9 +12,10 @@ and is kept in step with it by hand:
 * the MMA issuer computes S(n) = Q K(n)^T into TMEM buffer n % 2, then, for the
   previous step, O_g += P_g V for each of the two softmax groups once that
   group has written its weights, with commits to kempty, s_full, q_empty,
-  pv_done, vempty and o_full; the first product of an item waits until the
-  epilogue of the item before has read O (o_empty); on its way out it commits
-  once more and waits for that commit, so every product has completed;
+  pv_done, vempty and o_full; an item's last PV products are issued before
+  the next item's first S product; the first product of an item waits until
+  the epilogue of the item before has read O (o_empty); on its way out it
+  commits once more and waits for that commit, so every product has completed;
 * eight softmax warps, two groups of four (one warp per TMEM lane quadrant in
   each group): each reads its group's columns of S(n), sometimes rescales its
   group's O (a raised maximum; it first waits for its group's product of the
@@ -366,6 +367,10 @@ class Cta:
                 yield ("yield",)
             t += 1
             k += 1
+            # the item's last products go out before the next item's first S
+            if ok and pend is not None and "last_pv_deferred" not in self.faults:
+                ok = yield from issue_pv(*pend)
+                pend = None
         if ok and pend is not None:
             ok = yield from issue_pv(*pend)
         # every product issued completes before TMEM is released
