@@ -187,9 +187,9 @@ __device__ __forceinline__ void tile_of(const AttnArgs& a, int item, int n_qt, i
 }
 
 // The kept 64-token key sub-blocks of a tile's two query halves, as bitmaps
-// in `bmask` (all key sub-blocks without a mask), listed in ascending order
-// with their keep bits into `ent` (shared or global memory); all lanes of one
-// warp.  Returns the list's length.
+// in `bmask` (all key sub-blocks without a mask), listed with their keep
+// bits into `ent` (shared or global memory) in the order below; all lanes of
+// one warp.  Returns the list's length.
 __device__ int union_list(const AttnArgs& a, int b, int h, int t0, int t1,
                           uint32_t (*bmask)[kMaxSub / 32], uint16_t* ent, int lane) {
   const int nsub = a.Lk / kSubBlock;
@@ -227,24 +227,50 @@ __device__ int union_list(const AttnArgs& a, int b, int h, int t0, int t1,
     }
   }
   __syncwarp();
-  // ascending union with per-half keep bits: lane w handles bitmap word w
+  // The union with per-half keep bits, ordered for the two softmax groups: a
+  // step's first entry goes to group 0, its second to group 1, and a query
+  // block's rows sit in two of the four lane quadrants (two SMSPs).  A step
+  // pairing an entry only the first query block keeps (A) with one only the
+  // second keeps (B) gives every SMSP one busy warp; any other pair loads two
+  // SMSPs with two.  So the first min(|A|, |B|) steps pair A with B; the
+  // unpaired rest of A or B follows, then the entries both keep (C), each class
+  // in ascending sub-block order.  Lane w handles bitmap word w.
   const uint32_t w0 = bmask[0][lane], w1 = bmask[1][lane];
-  const uint32_t wu = w0 | w1;
-  const int c = __popc(wu);
-  int incl = c;
+  const uint32_t wa = w0 & ~w1, wb = w1 & ~w0, wc = w0 & w1;
+  int ia = __popc(wa), ib = __popc(wb), ic = __popc(wc);  // inclusive prefix sums
   for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
+    const int va = __shfl_up_sync(0xffffffffu, ia, o);
+    const int vb = __shfl_up_sync(0xffffffffu, ib, o);
+    const int vc = __shfl_up_sync(0xffffffffu, ic, o);
+    if (lane >= o) {
+      ia += va;
+      ib += vb;
+      ic += vc;
+    }
   }
-  const int n_ent = __shfl_sync(0xffffffffu, incl, 31);
-  int pos = incl - c;
-  for (uint32_t mb = wu; mb; mb &= mb - 1) {
+  const int na = __shfl_sync(0xffffffffu, ia, 31), nb_ = __shfl_sync(0xffffffffu, ib, 31);
+  const int nc = __shfl_sync(0xffffffffu, ic, 31);
+  const int np = na < nb_ ? na : nb_;           // A-B pairs
+  const int rest = 2 * np + (na - np) + (nb_ - np);  // where C starts
+  int ra = ia - __popc(wa), rb = ib - __popc(wb), rc = ic - __popc(wc);  // exclusive ranks
+  for (uint32_t mb = w0 | w1; mb; mb &= mb - 1) {
     const int bit = __ffs(mb) - 1;
     const uint32_t keep = ((w0 >> bit) & 1u) | (((w1 >> bit) & 1u) << 1);
-    ent[pos++] = (uint16_t)((uint32_t)(lane * 32 + bit) | (keep << kKeepShift));
+    int pos;
+    if (keep == 1u) {
+      pos = ra < np ? 2 * ra : 2 * np + (ra - np);
+      ++ra;
+    } else if (keep == 2u) {
+      pos = rb < np ? 2 * rb + 1 : 2 * np + (na - np) + (rb - np);
+      ++rb;
+    } else {
+      pos = rest + rc;
+      ++rc;
+    }
+    ent[pos] = (uint16_t)((uint32_t)(lane * 32 + bit) | (keep << kKeepShift));
   }
   __syncwarp();
-  return n_ent;
+  return na + nb_ + nc;
 }
 
 // Prebuilt tile lists (sdl_tile_lists): per position r of the take order a

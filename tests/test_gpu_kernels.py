@@ -536,7 +536,9 @@ def test_bounded_wait_times_out_and_the_context_survives():
 def test_listed_attention_equals_scheduled(B, L, H, Hkv, density):
     """Tiles and lists prebuilt once (sdl_tile_lists) give the scheduled path's result
     bit for bit, LSE included, and the records hold the tiles in take order with the
-    ascending union of their two query blocks' kept blocks."""
+    union of their two query blocks' kept blocks in step order: blocks only the first
+    keeps paired with blocks only the second keeps, then the unpaired rest of either,
+    then the blocks both keep, each class ascending."""
     w = synth.small_workload(B=B, L=L, H=H, H_kv=Hkv, d=128, bs=64)
     _, dev = _inputs(w)
     nb = L // 64
@@ -573,7 +575,12 @@ def test_listed_attention_equals_scheduled(B, L, H, Hkv, density):
         for s, qb in enumerate(rows):
             if qb >= 0:
                 keep[s] = mask[b, h, qb].astype(bool)
-        union = np.nonzero(keep[0] | keep[1])[0]
+        a_only = np.nonzero(keep[0] & ~keep[1])[0]
+        b_only = np.nonzero(keep[1] & ~keep[0])[0]
+        both = np.nonzero(keep[0] & keep[1])[0]
+        npair = min(len(a_only), len(b_only))
+        union = np.concatenate([np.stack([a_only[:npair], b_only[:npair]], 1).reshape(-1),
+                                a_only[npair:], b_only[npair:], both]).astype(np.int64)
         assert rec[r, 1] == len(union)
         e = ent[r, :len(union)]
         assert np.array_equal(e & 0x3FFF, union)
