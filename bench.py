@@ -633,6 +633,9 @@ def main():
         sc_ms = ev_time(lambda: sdl.block_scores(x0["q"], x0["k"], w.bs, scores=att.scores,
                                                  workspace=att.ws_scores))
     se_ms = ev_time(att.select)
+    # the whole anchor step, launches queued back to back (the GPU's own time for
+    # it, with no idle queue in front)
+    an_ms = None if runner.pulsecol else ev_time(lambda: att.refresh(x0["q"], x0["k"], 0))
     score_bytes = (2 * w.B * w.L * (runner.H + runner.H_kv) * w.d +
                    4 * w.B * runner.H * w.nb * w.nb)
     # dense baseline on distinct inputs per launch (larger than L2 in total)
@@ -700,6 +703,7 @@ def main():
         # barrier; the later ones behind the previous steps' attention launches
         "anchor_ms_first": anchor_ms[0] if anchor_ms else None,
         "anchor_ms_steady": statistics.mean(anchor_ms[1:]) if len(anchor_ms) > 1 else None,
+        "anchor_ms_back_to_back": an_ms,
         "block_scores_ms": sc_ms,
         "block_scores_gbs": None if runner.pulsecol else score_bytes / (sc_ms * 1e-3) / 1e9,
         "select_mask_ms": se_ms, "mask_blocks": budget,

@@ -16,6 +16,7 @@ strides on the other axes).  The calls mirror ``include/sdl.h``:
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -32,7 +33,7 @@ EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspac
            "sdl_tile_plan", "sdl_sparse_attn_planned", "sdl_tile_order",
            "sdl_sparse_attn_scheduled", "sdl_tile_lists_bytes", "sdl_tile_lists",
            "sdl_sparse_attn_listed", "sdl_dense_attn",
-           "sdl_anchor_workspace_bytes", "sdl_anchor_refresh",
+           "sdl_anchor_workspace_bytes", "sdl_anchor_refresh", "sdl_anchor_step",
            "sdl_col_budget", "sdl_col_scores_workspace_bytes", "sdl_col_scores",
            "sdl_col_select", "sdl_col_gather", "sdl_col_sparse_attn",
            "sdl_select_shard_workspace_bytes", "sdl_select_shard_hist",
@@ -107,6 +108,7 @@ def _lib():
         L.sdl_anchor_workspace_bytes.argtypes = [SP]
         L.sdl_anchor_workspace_bytes.restype = SZ
         L.sdl_anchor_refresh.argtypes = [P, P, SP, F, D, P, P, P, I64, P, P, SZ, P]
+        L.sdl_anchor_step.argtypes = [P, P, SP, F, D, P, P, P, I64, P, P, P, SZ, P, SZ, P]
         L.sdl_select_shard_workspace_bytes.argtypes = [SP]
         L.sdl_select_shard_workspace_bytes.restype = SZ
         L.sdl_select_shard_hist.argtypes = [SP, ctypes.c_int, ctypes.POINTER(SZ),
@@ -123,7 +125,7 @@ def _lib():
         L.sdl_status_string.argtypes = [ctypes.c_int]
         L.sdl_status_string.restype = ctypes.c_char_p
         for f in ("sdl_block_scores", "sdl_select_mask", "sdl_select_mask_scoped",
-                  "sdl_anchor_refresh", "sdl_col_scores", "sdl_col_select",
+                  "sdl_anchor_refresh", "sdl_anchor_step", "sdl_col_scores", "sdl_col_select",
                   "sdl_wait_selfcheck",
                   "sdl_col_gather", "sdl_col_sparse_attn",
                   "sdl_select_shard_hist", "sdl_select_shard_pass", "sdl_select_shard_count",
@@ -163,18 +165,29 @@ def _strides(t):
     return (t.stride(0), t.stride(1), t.stride(2))
 
 
+_SHAPES = {}  # built shapes by the tensors' geometry (a step loop repeats a few)
+
+
 def make_shape(q, k, block: int, v=None, o=None) -> Shape:
     """sdl_shape for Q [B,L,H,d] and K/V [B,L,H_kv,d] tensors (any device: only their
-    shapes, dtype and strides are read)."""
-    B, L, H, d = q.shape
-    s = Shape()
-    s.B, s.H, s.H_kv, s.L, s.d, s.block = B, H, k.shape[2], L, d, block
-    s.dtype = _dtype_code(q)
-    s.q_strides[:] = _strides(q)
-    s.k_strides[:] = _strides(k)
-    s.v_strides[:] = _strides(v if v is not None else k)
-    s.o_strides[:] = _strides(o if o is not None else q)
-    return s
+    shapes, dtype and strides are read).  Returns a fresh struct the caller may modify."""
+    key = (q.shape, q.stride(), q.dtype, k.shape, k.stride(), k.dtype,
+           None if v is None else (v.shape, v.stride()),
+           None if o is None else (o.shape, o.stride()), block)
+    s = _SHAPES.get(key)
+    if s is None:
+        B, L, H, d = q.shape
+        s = Shape()
+        s.B, s.H, s.H_kv, s.L, s.d, s.block = B, H, k.shape[2], L, d, block
+        s.dtype = _dtype_code(q)
+        s.q_strides[:] = _strides(q)
+        s.k_strides[:] = _strides(k)
+        s.v_strides[:] = _strides(v if v is not None else k)
+        s.o_strides[:] = _strides(o if o is not None else q)
+        if len(_SHAPES) >= 64:
+            _SHAPES.clear()
+        _SHAPES[key] = s
+    return Shape.from_buffer_copy(s)
 
 
 def _stream(stream):
@@ -302,6 +315,48 @@ def anchor_refresh(q, k, block: int, sparsity: float, scores=None, row_ptr=None,
                                      workspace.data_ptr(), workspace.numel(), _stream(stream)),
            "sdl_anchor_refresh")
     return scores, row_ptr, col_idx, plan
+
+
+def anchor_step(q, k, block: int, sparsity: float, scores=None, row_ptr=None, col_idx=None,
+                plan=None, order=None, lists=None, want_lists: bool = True, workspace=None,
+                scale: float = 0.0, stream=None):
+    """The whole anchor step in one call (see ``sdl_anchor_step``): block scores, mask,
+    tile plan, take order and (``want_lists``) the tile lists; 64-token blocks.
+    Returns (scores, row_ptr, col_idx, plan, order, lists or None)."""
+    import torch
+    s = make_shape(q, k, block)
+    nb = s.L // block
+    dev = q.device
+    n_qt = (nb + 1) // 2
+    # buffers the caller did not pass (a layer passes all of them: no host work here)
+    if scores is None:
+        scores = torch.empty((s.B, s.H, nb, nb), dtype=torch.float32, device=dev)
+    if row_ptr is None:
+        row_ptr = torch.empty(s.B * s.H * nb + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        total = mask_budget(s, sparsity)
+        if total < 0:
+            raise SdlError(SDL_ERR_INVALID_ARG, "sdl_mask_budget")
+        col_idx = torch.empty(total, dtype=torch.int32, device=dev)
+    if plan is None:
+        plan = torch.empty((s.B, s.H, n_qt, 2), dtype=torch.int32, device=dev)
+    if order is None:
+        order = torch.empty(s.B * s.H * n_qt, dtype=torch.int32, device=dev)
+    if lists is None and want_lists:
+        lists = torch.empty(int(_lib().sdl_tile_lists_bytes(ctypes.byref(s))), dtype=torch.uint8,
+                            device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(int(_lib().sdl_anchor_workspace_bytes(ctypes.byref(s))), 16),
+                                dtype=torch.uint8, device=dev)
+    _on_cuda("sdl_anchor_step", q, k, scores, row_ptr, col_idx, plan, order, lists, workspace)
+    _check(_lib().sdl_anchor_step(q.data_ptr(), k.data_ptr(), ctypes.byref(s), float(scale),
+                                  float(sparsity), scores.data_ptr(), row_ptr.data_ptr(),
+                                  col_idx.data_ptr(), col_idx.numel(), plan.data_ptr(),
+                                  order.data_ptr(), None if lists is None else lists.data_ptr(),
+                                  0 if lists is None else lists.numel(), workspace.data_ptr(),
+                                  workspace.numel(), _stream(stream)),
+           "sdl_anchor_step")
+    return scores, row_ptr, col_idx, plan, order, lists
 
 
 def col_budget(q, k, block: int, sparsity: float) -> int:
@@ -499,6 +554,7 @@ def _need_i32(t, n: int, what: str):
         raise SdlError(SDL_ERR_INVALID_ARG, f"{what}: int32 with at least {n} elements needed")
 
 
+@functools.lru_cache(maxsize=256)
 def tile_lists_bytes(B: int, H: int, L: int, block: int = 64) -> int:
     """Bytes of the prebuilt tile lists of a shape (see ``sdl_tile_lists_bytes``)."""
     s = Shape()

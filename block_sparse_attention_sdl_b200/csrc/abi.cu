@@ -189,6 +189,27 @@ int* device_status_ptr() {
 
 using namespace sdl;
 
+// Arguments of the tile-list kernel for a 64-token-block mask.
+static AttnArgs lists_args(const sdl_shape& s, const int32_t* row_ptr, const int32_t* col_idx,
+                    const int32_t* plan, const int32_t* order, int* status) {
+  AttnArgs a{};
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.plan = plan;
+  a.order = order;
+  a.lists = nullptr;
+  a.B = s.B;
+  a.H = s.H;
+  a.Hkv = s.H_kv;
+  a.L = s.L;
+  a.d = s.d;
+  a.block = s.block;
+  a.nb = s.L / s.block;
+  a.Lk = s.L;
+  a.status = status;
+  return a;
+}
+
 extern "C" {
 
 int64_t sdl_mask_budget(const sdl_shape* shape, double sparsity) {
@@ -309,10 +330,25 @@ size_t sdl_anchor_workspace_bytes(const sdl_shape* shape) {
          align256(sdl_select_workspace_bytes(shape)) + anchor_barrier_bytes();
 }
 
-sdl_status sdl_anchor_refresh(const void* q, const void* k, const sdl_shape* shape, float scale,
-                              double sparsity, float* scores, int32_t* row_ptr,
-                              int32_t* col_idx, int64_t col_capacity, int32_t* plan,
-                              void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Validation and workspace carving shared by the fused anchor entry points;
+// `plan` is checked by the callers.
+struct AnchorCall {
+  float* qbar;
+  float* kbar;
+  char* sel;
+  unsigned* bar;
+  int* status;
+  int64_t total;
+};
+
+sdl_status anchor_prepare(const void* q, const void* k, const sdl_shape* shape, double sparsity,
+                          const float* scores, const int32_t* row_ptr, const int32_t* col_idx,
+                          int64_t col_capacity, void* workspace, size_t workspace_bytes,
+                          AnchorCall& c) {
   sdl_status e = check_shape(shape);
   if (e) return e;
   const sdl_shape& s = *shape;
@@ -321,23 +357,69 @@ sdl_status sdl_anchor_refresh(const void* q, const void* k, const sdl_shape* sha
   if ((e = check_strides(s.q_strides, s.dtype, s.B, s.L, s.H)) ||
       (e = check_strides(s.k_strides, s.dtype, s.B, s.L, s.H_kv)))
     return e;
-  if (plan && s.block != 64) return SDL_ERR_INVALID_ARG;
-  const int64_t total = sdl_mask_budget(shape, sparsity);
-  if (total < 0) return SDL_ERR_INVALID_ARG;
-  if (col_capacity < total) return SDL_ERR_CAPACITY;
+  c.total = sdl_mask_budget(shape, sparsity);
+  if (c.total < 0) return SDL_ERR_INVALID_ARG;
+  if (col_capacity < c.total) return SDL_ERR_CAPACITY;
   const size_t need = sdl_anchor_workspace_bytes(shape);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return SDL_ERR_WORKSPACE;
-  int* status = device_status_ptr();
-  if (!status) return SDL_ERR_CUDA;
+  c.status = device_status_ptr();
+  if (!c.status) return SDL_ERR_CUDA;
   const size_t nb = s.L / s.block;
   char* w = static_cast<char*>(workspace);
-  float* qbar = reinterpret_cast<float*>(w);
-  float* kbar = reinterpret_cast<float*>(w + align256(sizeof(float) * s.B * s.H * nb * s.d));
-  char* sel = w + align256(sdl_scores_workspace_bytes(shape));
-  unsigned* bar = reinterpret_cast<unsigned*>(sel + align256(sdl_select_workspace_bytes(shape)));
-  cudaError_t ce = launch_anchor(q, k, s, resolve_scale(scale, s.d), total / s.B, qbar, kbar,
-                                 scores, sel, row_ptr, col_idx, plan, bar, status,
+  c.qbar = reinterpret_cast<float*>(w);
+  c.kbar = reinterpret_cast<float*>(w + align256(sizeof(float) * s.B * s.H * nb * s.d));
+  c.sel = w + align256(sdl_scores_workspace_bytes(shape));
+  c.bar = reinterpret_cast<unsigned*>(c.sel + align256(sdl_select_workspace_bytes(shape)));
+  return SDL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sdl_status sdl_anchor_refresh(const void* q, const void* k, const sdl_shape* shape, float scale,
+                              double sparsity, float* scores, int32_t* row_ptr,
+                              int32_t* col_idx, int64_t col_capacity, int32_t* plan,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  AnchorCall c;
+  const sdl_status e = anchor_prepare(q, k, shape, sparsity, scores, row_ptr, col_idx,
+                                      col_capacity, workspace, workspace_bytes, c);
+  if (e) return e;
+  const sdl_shape& s = *shape;
+  if (plan && s.block != 64) return SDL_ERR_INVALID_ARG;
+  cudaError_t ce = launch_anchor(q, k, s, resolve_scale(scale, s.d), c.total / s.B, c.qbar,
+                                 c.kbar, scores, c.sel, row_ptr, col_idx, plan, c.bar, c.status,
                                  static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce);
+  return SDL_OK;
+}
+
+sdl_status sdl_anchor_step(const void* q, const void* k, const sdl_shape* shape, float scale,
+                           double sparsity, float* scores, int32_t* row_ptr, int32_t* col_idx,
+                           int64_t col_capacity, int32_t* plan, int32_t* order, void* lists,
+                           size_t lists_bytes, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  sdl_status e = check_shape(shape);
+  if (e) return e;
+  const sdl_shape& s = *shape;
+  if (s.block != 64) return SDL_ERR_UNSUPPORTED;
+  if (!plan || !order) return SDL_ERR_INVALID_ARG;
+  if (lists && !aligned16(lists)) return SDL_ERR_INVALID_ARG;
+  if (lists && lists_bytes < sdl_tile_lists_bytes(shape)) return SDL_ERR_WORKSPACE;
+  AnchorCall c;
+  e = anchor_prepare(q, k, shape, sparsity, scores, row_ptr, col_idx, col_capacity, workspace,
+                     workspace_bytes, c);
+  if (e) return e;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nb = s.L / s.block;
+  cudaError_t ce = launch_anchor(q, k, s, resolve_scale(scale, s.d), c.total / s.B, c.qbar,
+                                 c.kbar, scores, c.sel, row_ptr, col_idx, nullptr, c.bar,
+                                 c.status, st);
+  if (ce == cudaSuccess) ce = launch_plan(row_ptr, col_idx, s.B, s.H, nb, plan, st);
+  if (ce == cudaSuccess) ce = launch_tile_order(row_ptr, plan, s.B, s.H, nb, order, st);
+  if (ce == cudaSuccess && lists)
+    ce = launch_tile_lists(lists_args(s, row_ptr, col_idx, plan, order, c.status),
+                           static_cast<int32_t*>(lists), st);
   if (ce != cudaSuccess) return cuda_fail(ce);
   return SDL_OK;
 }
@@ -602,21 +684,7 @@ sdl_status sdl_tile_lists(const int32_t* row_ptr, const int32_t* col_idx, const 
   if (lists_bytes < sdl_tile_lists_bytes(shape)) return SDL_ERR_WORKSPACE;
   int* status = device_status_ptr();
   if (!status) return SDL_ERR_CUDA;
-  AttnArgs a{};
-  a.row_ptr = row_ptr;
-  a.col_idx = col_idx;
-  a.plan = plan;
-  a.order = order;
-  a.lists = nullptr;
-  a.B = shape->B;
-  a.H = shape->H;
-  a.Hkv = shape->H_kv;
-  a.L = shape->L;
-  a.d = shape->d;
-  a.block = shape->block;
-  a.nb = shape->L / shape->block;
-  a.Lk = shape->L;
-  a.status = status;
+  const AttnArgs a = lists_args(*shape, row_ptr, col_idx, plan, order, status);
   const cudaError_t ce =
       launch_tile_lists(a, static_cast<int32_t*>(lists), static_cast<cudaStream_t>(stream));
   if (ce != cudaSuccess) return cuda_fail(ce);

@@ -150,19 +150,27 @@ cudaError_t launch_anchor_t(AnchorArgs& a, size_t smem, cudaStream_t st) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  e = cudaFuncSetAttribute(anchor_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
-  if (e != cudaSuccess) return e;
-  int sms = 0, per_sm = 0;
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, anchor_kernel<T>, kAnchorThreads,
-                                                    smem);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  // every block resident (the barriers need it); two per SM keep HBM busy
-  // while pooling
-  const int grid = sms * (per_sm < 2 ? per_sm : 2);
+  // per device: the shared-memory size last configured and the grid it gives
+  // ((smem << 24) | grid; 0: none yet), so that steady calls make no queries
+  static std::atomic<uint64_t> config[64];
+  const uint64_t c = config[dev].load();
+  int grid = (int)(c & 0xFFFFFFu);
+  if (c == 0 || (c >> 24) != (uint64_t)smem) {
+    e = cudaFuncSetAttribute(anchor_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, anchor_kernel<T>, kAnchorThreads,
+                                                      smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    // every block resident (the barriers need it); two per SM keep HBM busy
+    // while pooling
+    grid = sms * (per_sm < 2 ? per_sm : 2);
+    config[dev].store(((uint64_t)smem << 24) | (uint64_t)grid);
+  }
   e = cudaMemsetAsync(a.bar, 0, sizeof(unsigned) * kBarriers, st);
   if (e != cudaSuccess) return e;
   void* args[] = {&a};

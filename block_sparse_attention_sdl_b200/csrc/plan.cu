@@ -32,9 +32,17 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
 
 constexpr int kOrderThreads = 1024;
 constexpr int kOrderBins = 2 * 1024 + 1;  // tile costs 0 .. 2 nb, nb <= 1024
-// tiles whose costs are kept in shared memory for the serial stable scatter
-// (16 bits each); beyond this the scatter recomputes them from the lists
+// tiles whose costs are kept in shared memory between the two walks (16 bits
+// each); beyond this the second walk recomputes them from the lists
 constexpr int kOrderCached = 48 * 1024;
+constexpr size_t kOrderCountBytes = 112 * 1024;  // per-warp bin counters, at most
+
+// Warps that count their own chunk of the tiles: as many as the per-warp
+// counters of nbins bins allow (at least one).
+inline int order_warps(int nbins) {
+  const int w = (int)(kOrderCountBytes / (sizeof(int) * (size_t)nbins));
+  return w < 1 ? 1 : (w > kOrderThreads / 32 ? kOrderThreads / 32 : w);
+}
 
 // One CTA: the order in which the attention kernel takes its tiles, costliest
 // first, so that the long tiles of heavy heads do not run last and leave the
@@ -42,15 +50,22 @@ constexpr int kOrderCached = 48 * 1024;
 // lengths (an upper bound of the union it walks); a stable counting sort orders
 // them (equal costs keep the tile order, so tiles of one head stay together and
 // share its K and V in L2).  order[r] = the r-th tile to take.
+//
+// Warp w < W counts the costs of its contiguous chunk of tiles into its own
+// row of counters; a scan over (cost descending, warp ascending) gives every
+// (warp, cost) its first place; each warp then walks its chunk again in order,
+// lanes of equal cost taking consecutive places in lane order.
 __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __restrict__ row_ptr,
                                                               const int32_t* __restrict__ plan,
-                                                              int BH, int nb, int n_qt,
+                                                              int BH, int nb, int n_qt, int W,
                                                               int32_t* __restrict__ order) {
   __shared__ int start[kOrderBins];
   __shared__ int s_warp[32];
-  extern __shared__ uint16_t cost_sm[];  // every tile's cost, when n <= kOrderCached
-  const int n = BH * n_qt, tid = threadIdx.x;
+  extern __shared__ __align__(16) int cnt_sm[];  // [W][nbins], then the costs (16 bits)
+  const int n = BH * n_qt, tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  const int nbins = 2 * nb + 1;
   const bool cached = n <= kOrderCached;
+  uint16_t* cost_sm = reinterpret_cast<uint16_t*>(cnt_sm + (size_t)W * nbins);
   auto cost_of = [&](int x) -> int {
     const int64_t r0 = (int64_t)(x / n_qt) * nb;
     int c = 0;
@@ -58,44 +73,56 @@ __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int32_t* __r
       const int qb = plan[2 * (int64_t)x + s];
       if (qb >= 0 && qb < nb) c += row_ptr[r0 + qb + 1] - row_ptr[r0 + qb];
     }
-    return c < 0 ? 0 : (c >= kOrderBins ? kOrderBins - 1 : c);
+    return c < 0 ? 0 : (c >= nbins ? nbins - 1 : c);
   };
-  auto cost = [&](int x) -> int { return cached ? (int)cost_sm[x] : cost_of(x); };
-  for (int c = tid; c < kOrderBins; c += kOrderThreads) start[c] = 0;
+  const int chunk = (n + W - 1) / W;
+  const int x0 = warp * chunk, x1 = x0 + chunk < n ? x0 + chunk : n;
+  for (int c = tid; c < W * nbins; c += kOrderThreads) cnt_sm[c] = 0;
   __syncthreads();
-  for (int x = tid; x < n; x += kOrderThreads) {
-    const int c = cost_of(x);
-    if (cached) cost_sm[x] = (uint16_t)c;
-    atomicAdd(&start[c], 1);
+  if (warp < W)
+    for (int x = x0 + lane; x < x1; x += 32) {
+      const int c = cost_of(x);
+      if (cached) cost_sm[x] = (uint16_t)c;
+      atomicAdd(&cnt_sm[warp * nbins + c], 1);
+    }
+  __syncthreads();
+  // per cost: the warps' counts into exclusive offsets, the total into start[]
+  for (int c = tid; c < nbins; c += kOrderThreads) {
+    int s = 0;
+    for (int w = 0; w < W; ++w) {
+      const int v = cnt_sm[w * nbins + c];
+      cnt_sm[w * nbins + c] = s;
+      s += v;
+    }
+    start[c] = s;
   }
   __syncthreads();
-  // first position of each cost, costs in descending order: thread t owns bins
-  // kOrderBins - 1 - 3t, -3t-1, -3t-2
+  // first place of each cost, costs in descending order: thread t owns bins
+  // nbins - 1 - 3t, -3t-1, -3t-2
   int cnt[3], local = 0;
   for (int y = 0; y < 3; ++y) {
-    const int c = kOrderBins - 1 - 3 * tid - y;
+    const int c = nbins - 1 - 3 * tid - y;
     cnt[y] = c >= 0 ? start[c] : 0;
     local += cnt[y];
   }
   int total = 0;
   int pos = selimpl::block_excl_scan(local, s_warp, total);
   for (int y = 0; y < 3; ++y) {
-    const int c = kOrderBins - 1 - 3 * tid - y;
+    const int c = nbins - 1 - 3 * tid - y;
     if (c >= 0) start[c] = pos;
     pos += cnt[y];
   }
   __syncthreads();
-  // stable scatter: one warp walks the tiles in order, 32 at a time; lanes with
-  // equal costs take consecutive places in lane order
-  if (tid < 32) {
-    for (int base = 0; base < n; base += 32) {
-      const int x = base + tid;
-      const int c = x < n ? cost(x) : -1;
+  if (warp < W) {
+    int* run = cnt_sm + warp * nbins;  // this warp's next place per cost, less start[]
+    for (int base = x0; base < x1; base += 32) {
+      const int x = base + lane;
+      const int c = x < x1 ? (cached ? (int)cost_sm[x] : cost_of(x)) : -1;
       const unsigned peers = __match_any_sync(0xffffffffu, c);
-      const int rank = __popc(peers & ((1u << tid) - 1u));
-      if (x < n) order[start[c] + rank] = x;
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      if (x < x1) order[start[c] + run[c] + rank] = x;
       __syncwarp();
-      if (x < n && tid == __ffs(peers) - 1) start[c] += __popc(peers);
+      if (x < x1 && lane == __ffs(peers) - 1) run[c] += __popc(peers);
       __syncwarp();
     }
   }
@@ -135,15 +162,19 @@ cudaError_t launch_plan(const int32_t* row_ptr, const int32_t* col_idx, int B, i
 
 cudaError_t launch_tile_order(const int32_t* row_ptr, const int32_t* plan, int B, int H, int nb,
                               int32_t* order, cudaStream_t st) {
+  if (nb < 1 || nb > (kOrderBins - 1) / 2) return cudaErrorInvalidValue;
   const int n = B * H * ((nb + 1) / 2);
-  const size_t smem = n <= kOrderCached ? sizeof(uint16_t) * (size_t)n : 0;
+  const int nbins = 2 * nb + 1, W = order_warps(nbins);
+  const size_t smem = sizeof(int) * (size_t)W * nbins +
+                      (n <= kOrderCached ? sizeof(uint16_t) * (size_t)n : 0);
   static std::atomic<bool> attr_set[64];  // per device
   cudaError_t e = once_per_device(attr_set, [] {
     return cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)(sizeof(uint16_t) * kOrderCached));
+                                (int)(kOrderCountBytes + sizeof(uint16_t) * kOrderCached));
   });
   if (e != cudaSuccess) return e;
-  order_kernel<<<1, kOrderThreads, smem, st>>>(row_ptr, plan, B * H, nb, (nb + 1) / 2, order);
+  order_kernel<<<1, kOrderThreads, smem, st>>>(row_ptr, plan, B * H, nb, (nb + 1) / 2, W,
+                                               order);
   return cudaGetLastError();
 }
 

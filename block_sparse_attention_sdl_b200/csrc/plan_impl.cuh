@@ -65,20 +65,33 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ row_ptr,
     for (int w = 0; w < nw; ++w) c += __popc(bits[w * nb + i]);
     len[i] = c;
   }
-  // intersections of every unordered pair once: (i, i + d mod nb), 1 <= d <= nb / 2
-  const int half = nb / 2;
-  for (int x = tid; x < nb * half; x += nthr) {
-    const int i = x / half, dd = x % half + 1, j = (i + dd) % nb;
-    if (2 * dd == nb && i > j) continue;  // that pair comes from its other end
-    int c = 0;
-    for (int w = 0; w < nw; ++w) c += __popc(bits[w * nb + i] & bits[w * nb + j]);
-    ov[i * nb + j] = ov[j * nb + i] = (uint16_t)c;
-  }
   __syncthreads();
-  for (int i = tid; i < nb; i += nthr) {
+  const int nwarps = nthr / 32;
+  // intersections, one warp per row i: lanes read consecutive words of the
+  // word-major bitmaps and write consecutive entries (no bank conflicts)
+  for (int i = warp; i < nb; i += nwarps) {
+    uint32_t bi[kPlanMaxNb / 32];
+#pragma unroll
+    for (int w = 0; w < kPlanMaxNb / 32; ++w) bi[w] = w < nw ? bits[w * nb + i] : 0u;
+    for (int j = lane; j < nb; j += 32) {
+      int c = 0;
+#pragma unroll
+      for (int w = 0; w < kPlanMaxNb / 32; ++w)
+        if (w < nw) c += __popc(bi[w] & bits[w * nb + j]);
+      ov[i * nb + j] = (uint16_t)c;
+    }
+  }
+  // visiting order: by descending list length, ties by lower index; the rank of
+  // block i counts the blocks before it, 32 at a time by ballot
+  for (int i = warp; i < nb; i += nwarps) {
+    const int li = len[i];
     int rank = 0;
-    for (int j = 0; j < nb; ++j) rank += (len[j] > len[i]) || (len[j] == len[i] && j < i);
-    order[rank] = i;
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      const bool before = j < nb && (len[j] > li || (len[j] == li && j < i));
+      rank += __popc(__ballot_sync(0xffffffffu, before));
+    }
+    if (lane == 0) order[rank] = i;
   }
   __syncthreads();
   if (warp == 0) {
@@ -89,20 +102,28 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ row_ptr,
     for (int c = 0; c < nc; ++c)
       if (lane + 32 * c < nb) unpaired |= 1u << c;
     int p = 0;
+    int i_next = order[0];
     for (int k = 0; k < nb; ++k) {
-      const int i = order[k];
+      const int i = i_next;
+      if (k + 1 < nb) i_next = order[k + 1];
+      // candidate keys of row i, (intersection + 1) << 16 | (0xFFFF - j): the
+      // largest is the largest intersection, lowest index on ties.  They do not
+      // depend on the pairing so far, so their loads leave the serial chain.
+      uint32_t kj[kPlanMaxNb / 32];
+#pragma unroll
+      for (int c = 0; c < kPlanMaxNb / 32; ++c) {
+        const int j = lane + 32 * c;
+        kj[c] = (c < nc && j < nb)
+                    ? ((uint32_t)ov[i * nb + j] + 1u) << 16 | (0xFFFFu - (uint32_t)j)
+                    : 0u;
+      }
       if (!((__shfl_sync(0xffffffffu, unpaired, i & 31) >> (i >> 5)) & 1u)) continue;
       if (lane == (i & 31)) unpaired &= ~(1u << (i >> 5));
-      // unpaired partner of largest intersection, lowest index on ties: the
-      // largest key (intersection + 1) << 16 | (0xFFFF - j); 0 when none is left
+      // the unpaired partner with the largest key; 0 when none is left
       uint32_t key = 0;
 #pragma unroll
       for (int c = 0; c < kPlanMaxNb / 32; ++c)
-        if (c < nc && ((unpaired >> c) & 1u)) {
-          const int j = lane + 32 * c;
-          const uint32_t kj = ((uint32_t)ov[i * nb + j] + 1u) << 16 | (0xFFFFu - (uint32_t)j);
-          key = kj > key ? kj : key;
-        }
+        if ((unpaired >> c) & 1u) key = kj[c] > key ? kj[c] : key;
       key = __reduce_max_sync(0xffffffffu, key);
       const int best = key ? (int)(0xFFFFu - (key & 0xFFFFu)) : -1;
       if (best >= 0 && lane == (best & 31)) unpaired &= ~(1u << (best >> 5));

@@ -74,8 +74,9 @@ __device__ void resolve(const int* hist, int B, int b, int npass, uint32_t kfree
     const int hi = nbin - per * threadIdx.x;
     int cnt[8];
     int local = 0;
-    for (int x = 0; x < per; ++x) {
-      cnt[x] = hb[hi - 1 - x];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      cnt[x] = x < per ? hb[hi - 1 - x] : 0;
       local += cnt[x];
     }
     // exclusive scan of `local` over threads in order
@@ -91,7 +92,9 @@ __device__ void resolve(const int* hist, int B, int b, int npass, uint32_t kfree
     for (int w = 0; w < warp; ++w) wbase += s_warp[w];
     const uint32_t krem = s_krem;
     uint32_t above = (uint32_t)(wbase + incl - local);
-    for (int x = 0; x < per; ++x) {
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      if (x >= per) break;
       uint32_t c = (uint32_t)cnt[x];
       if (above < krem && above + c >= krem) {
         s_prefix |= (uint32_t)(hi - 1 - x) << kShift[p];
@@ -129,25 +132,37 @@ __device__ __forceinline__ void hist_body(const float* __restrict__ scores, int 
   const int64_t n4 = (per_b % 4 == 0) ? per_b / 4 : 0;
   // whole warps iterate together so the lane-aggregated increments stay convergent
   const int64_t n4_round = (n4 + kThreads - 1) / kThreads * kThreads;
+  const bool narrow = per_b <= 0x7fffffff;  // 32-bit index arithmetic suffices
   for (int64_t x = (int64_t)cx * kThreads + threadIdx.x; x < n4_round;
        x += (int64_t)ncx * kThreads) {
     float vals[4] = {0.f, 0.f, 0.f, 0.f};
     const bool in = x < n4;
+    int i = 0, j = 0;  // the first element's query block and key block
     if (in) {
       float4 v = __ldg(reinterpret_cast<const float4*>(base) + x);
       vals[0] = v.x;
       vals[1] = v.y;
       vals[2] = v.z;
       vals[3] = v.w;
+      if (narrow) {
+        const uint32_t e = 4u * (uint32_t)x, r = e / (uint32_t)nb;
+        j = (int)(e - r * (uint32_t)nb);
+        i = (int)(r % (uint32_t)nb);
+      } else {
+        const int64_t e = 4 * x, r = e / nb;
+        j = (int)(e - r * nb);
+        i = (int)(r % nb);
+      }
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int64_t e = 4 * x + u;
-      const int j = (int)(e % nb);
-      const int i = (int)((e / nb) % nb);
       const uint32_t key = __float_as_uint(vals[u]);
       const bool take = in && i != j && (hs >= 32 || (key >> hs) == want);
       hist_add(sh, (int)((key >> shift) & dmask), take);
+      if (++j == nb) {  // the next element starts the next row
+        j = 0;
+        i = i + 1 == nb ? 0 : i + 1;
+      }
     }
   }
   const int64_t tail0 = n4 * 4;

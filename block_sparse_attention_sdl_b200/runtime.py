@@ -27,9 +27,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (anchor_refresh, anchor_workspace_bytes, block_scores, col_budget, col_gather,
-               col_scores, col_scores_workspace_bytes, col_select, col_sparse_attn, dense_attn,
-               make_shape, mask_budget, scores_workspace_bytes, select_mask,
+from . import (anchor_refresh, anchor_step, anchor_workspace_bytes, block_scores, col_budget,
+               col_gather, col_scores, col_scores_workspace_bytes, col_select, col_sparse_attn,
+               dense_attn, make_shape, mask_budget, scores_workspace_bytes, select_mask,
                select_shard_capacity, select_workspace_bytes, sparse_attn, tile_lists,
                tile_lists_bytes, tile_order, tile_plan)
 from .sharded import CudaStages, select_mask_sharded, torch_collectives
@@ -118,8 +118,15 @@ class StepSparseAttention:
                                       dtype=torch.uint8, device=dev) if self.fused else None)
 
     def refresh(self, q, k, step: int, stream=None):
+        if self.fused and self.plan is not None:
+            # the whole step (scores, mask, plan, order, lists) from one C call
+            anchor_step(q, k, self.block, self.sparsity, scores=self.scores,
+                        row_ptr=self.row_ptr, col_idx=self.col_idx, plan=self.plan,
+                        order=self.order, lists=self.lists, want_lists=self.lists is not None,
+                        workspace=self.ws_anchor, stream=stream)
+            self.mask_step = step
+            return
         if self.fused:
-            # the tile plan runs apart: its own kernel is wider than the fused grid's blocks
             anchor_refresh(q, k, self.block, self.sparsity, scores=self.scores,
                            row_ptr=self.row_ptr, col_idx=self.col_idx, want_plan=False,
                            workspace=self.ws_anchor, stream=stream)

@@ -186,6 +186,30 @@ sdl_status sdl_anchor_refresh(const void* q, const void* k, const sdl_shape* sha
                               int32_t* col_idx, int64_t col_capacity, int32_t* plan,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Whole anchor step, one call --------------------------------------------
+ * Everything an anchor step of the Step-dLLM abstract (the mask refresh at
+ * steps 0, K, 2K, ...) produces for the attention calls that follow it, with
+ * every launch issued from here back to back and no return to the caller in
+ * between: the fused block scores and selection of sdl_anchor_refresh, then
+ * sdl_tile_plan, sdl_tile_order and (when `lists` is not NULL)
+ * sdl_tile_lists.  The paper describes the refresh, not this scheduling
+ * aid.  Outputs are bit for bit those of the separate calls: scores fp32
+ * [B,H,nb,nb], row_ptr int32 [B*H*nb + 1], col_idx int32 (col_capacity >=
+ * sdl_mask_budget), plan int32 [B,H,ceil(nb/2),2], order int32
+ * [B*H*ceil(nb/2)], lists (16-byte aligned, lists_bytes >=
+ * sdl_tile_lists_bytes) for sdl_sparse_attn_listed.  64-token blocks only
+ * (else SDL_ERR_UNSUPPORTED); plan and order must not be NULL
+ * (SDL_ERR_INVALID_ARG).  Workspace as sdl_anchor_refresh
+ * (sdl_anchor_workspace_bytes).  All buffers are device memory owned by the
+ * caller.  Arguments are validated before the first launch, so an error
+ * return launches nothing; a launch failure returns SDL_ERR_CUDA and stops
+ * the sequence there. */
+sdl_status sdl_anchor_step(const void* q, const void* k, const sdl_shape* shape, float scale,
+                           double sparsity, float* scores, int32_t* row_ptr, int32_t* col_idx,
+                           int64_t col_capacity, int32_t* plan, int32_t* order, void* lists,
+                           size_t lists_bytes, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
 /* ---- Mask selection with the heads of a sequence split over ranks ----------
  * The global budget of the Step-dLLM abstract (and the rule of sdl_select_mask)
  * when rank r of W holds the contiguous head range [h_r, h_r + H_local) of

@@ -124,6 +124,37 @@ def test_zero_strides_refused_on_axes_with_more_than_one_index():
     assert rc == sdl.SDL_ERR_INVALID_ARG
 
 
+def test_anchor_step_host_checks():
+    """sdl_anchor_step refuses what its header lists before any launch: 128-token
+    blocks, a missing plan or order, a short workspace or lists buffer, a
+    misaligned lists buffer, a column buffer below the budget."""
+    lib = sdl.lib()
+    P = ctypes.c_void_p
+    shp = _shape(H=4, Hkv=4, L=1024)
+    total = sdl.mask_budget(shp, 0.5)
+    ws = sdl.lib().sdl_anchor_workspace_bytes(ctypes.byref(shp))
+    nl = sdl.lib().sdl_tile_lists_bytes(ctypes.byref(shp))
+    assert ws > 0 and nl > 0
+
+    def call(shape=shp, plan=P(256), order=P(256), lists=P(256), lists_bytes=nl, cap=total,
+             ws_bytes=ws):
+        return lib.sdl_anchor_step(P(256), P(256), ctypes.byref(shape), 0.0, 0.5, P(256),
+                                   P(256), P(256), cap, plan, order, lists, lists_bytes, P(256),
+                                   ws_bytes, None)
+
+    big = _shape(H=4, Hkv=4, L=1024, block=128)
+    assert call(shape=big, ws_bytes=1 << 40) == sdl.SDL_ERR_UNSUPPORTED
+    assert call(plan=None) == sdl.SDL_ERR_INVALID_ARG
+    assert call(order=None) == sdl.SDL_ERR_INVALID_ARG
+    assert call(lists=P(264)) == sdl.SDL_ERR_INVALID_ARG
+    assert call(lists_bytes=nl - 1) == sdl.SDL_ERR_WORKSPACE
+    assert call(ws_bytes=ws - 1) == sdl.SDL_ERR_WORKSPACE
+    assert call(cap=total - 1) == sdl.SDL_ERR_CAPACITY
+    rc = lib.sdl_anchor_step(None, P(256), ctypes.byref(shp), 0.0, 0.5, P(256), P(256), P(256),
+                             total, P(256), P(256), None, 0, P(256), ws, None)
+    assert rc == sdl.SDL_ERR_INVALID_ARG
+
+
 def test_status_strings():
     lib = sdl.lib()
     for code in range(9):

@@ -71,3 +71,85 @@ def test_fused_anchor_repeated_launches_on_one_workspace():
         torch.cuda.synchronize()
         assert sdl.last_device_status() == sdl.SDL_OK
         assert torch.equal(sc, sc1) and torch.equal(rp, rp1) and torch.equal(ci, ci1)
+
+
+@pytest.mark.parametrize("dtype,B,L,H,H_kv,d,s", [
+    ("bf16", 2, 1024, 4, 2, 128, 0.7),
+    ("bf16", 1, 576, 3, 3, 64, 0.6),          # nb = 9: a tile with one query block
+    ("fp32", 1, 512, 2, 2, 64, 0.5),          # no tile lists for fp32 layers, still buildable
+    ("bf16", 1, 17408, 2, 2, 64, 0.95),       # nb = 272: adjacent pairs
+    ("bf16", 1, 8192, 32, 32, 128, 0.9),      # the 8K workload's shape
+])
+def test_anchor_step_equals_separate_calls(dtype, B, L, H, H_kv, d, s):
+    """sdl_anchor_step: scores, CSR lists, tile plan, take order and tile lists
+    equal the separate calls bit for bit, over two steps on one set of buffers."""
+    w = synth.small_workload(dtype=dtype, B=B, H=H, H_kv=H_kv, L=L, d=d, bs=64, sparsity=s,
+                             planted=2)
+    bufs = None
+    for step in range(2):
+        x = synth.device_inputs(w, step)
+        q, k = x["q"], x["k"]
+        sc1, rp1, ci1, _ = sdl.anchor_refresh(q, k, 64, s, want_plan=False)
+        plan1 = sdl.tile_plan(rp1, ci1, B, H, L, 64)
+        order1 = sdl.tile_order(rp1, plan1, B, H, L, 64)
+        lists1 = sdl.tile_lists(rp1, ci1, plan1, order1, B, H, L, 64)
+        if bufs is None:
+            bufs = sdl.anchor_step(q, k, 64, s)
+        else:
+            sc, rp, ci, plan, order, lists = bufs
+            bufs = sdl.anchor_step(q, k, 64, s, scores=sc, row_ptr=rp, col_idx=ci, plan=plan,
+                                   order=order, lists=lists)
+        torch.cuda.synchronize()
+        assert sdl.last_device_status() == sdl.SDL_OK
+        sc, rp, ci, plan, order, lists = bufs
+        assert torch.equal(sc, sc1)
+        assert torch.equal(rp, rp1) and torch.equal(ci, ci1[:ci.numel()])
+        assert torch.equal(plan, plan1) and torch.equal(order, order1)
+        assert _lists_used(lists, B, H, L) == _lists_used(lists1, B, H, L)
+
+
+def _lists_used(lists, B, H, L):
+    """The written part of a tile-lists buffer: each record's (item, n_ent, t0, t1)
+    and its first n_ent entries (the slack after them is never written)."""
+    n_items = B * H * ((L + 127) // 128)
+    cap = ((L // 64) + 7) // 8 * 8
+    raw = lists.cpu().numpy()
+    rec = raw[:n_items * 32].view(np.int32).reshape(n_items, 8)
+    ent = raw[n_items * 32:n_items * 32 + n_items * cap * 2].view(np.uint16).reshape(n_items, cap)
+    return [(tuple(rec[r, :4]), tuple(ent[r, :max(rec[r, 1], 0)])) for r in range(n_items)]
+
+
+@pytest.mark.parametrize("B,H,nb,cap", [
+    (1, 100, 1024, 1024),   # 51200 tiles: costs recomputed in the second walk; 13 warps count
+    (2, 64, 128, 128),      # the 8K block count: all 32 warps count
+    (3, 7, 17, 5),          # odd block count, costs in a narrow range (many ties)
+])
+def test_tile_order_exact_at_scale(B, H, nb, cap):
+    """The take order is the stable sort of the tiles by descending cost (a tile's
+    two list lengths), checked entry for entry against numpy's stable sort, with
+    row offsets only (the order reads no column indices)."""
+    rng = np.random.default_rng(B * 1000 + H + nb)
+    # skewed list lengths in [1, cap]: many short rows, a few long ones
+    lens = np.minimum(cap, 1 + rng.geometric(4.0 / cap, size=B * H * nb)).astype(np.int64)
+    rp = np.zeros(B * H * nb + 1, np.int64)
+    rp[1:] = np.cumsum(lens)
+    n_qt = (nb + 1) // 2
+    # a random valid pairing per head
+    pl = np.full((B, H, n_qt, 2), -1, np.int32)
+    for b in range(B):
+        for h in range(H):
+            flat = np.full(2 * n_qt, -1)
+            flat[:nb] = rng.permutation(nb)
+            pl[b, h] = flat.reshape(n_qt, 2)
+    rp_d = torch.from_numpy(rp.astype(np.int32)).cuda()
+    plan_d = torch.from_numpy(pl).cuda()
+    order = sdl.tile_order(rp_d, plan_d, B, H, nb * 64, 64).cpu().numpy()
+    assert sdl.last_device_status() == sdl.SDL_OK
+    flat = pl.reshape(-1, 2)
+    head = np.arange(B * H * n_qt) // n_qt
+    cost = np.zeros(B * H * n_qt, np.int64)
+    for s_ in range(2):
+        qb = flat[:, s_]
+        ok = qb >= 0
+        cost[ok] += lens[head[ok] * nb + qb[ok]]
+    assert np.array_equal(order, np.argsort(-cost, kind="stable"))
