@@ -5,14 +5,15 @@
 // The separate kernels of scores.cu, select.cu and plan.cu take one launch per
 // phase (ten at an anchor); at the 2K and 8K workloads most of their time is
 // launch and ramp latency, not work.  Here one persistent cooperative grid (all
-// blocks resident) runs the same phase bodies back to back, separated by grid
-// barriers:
-//   pooling -> | scores -> | digit pass 0 -> | pass 1 -> | pass 2 -> |
-//   per-row counts -> | tie hand-out and row offsets (block 0) -> |
-//   list compaction -> | tile plan
-// Results are bit for bit those of the separate calls (same bodies, same
-// order of every floating-point operation).  Every barrier wait is bounded: on
-// timeout the grid raises the device status word and every block returns.
+// blocks resident) runs the phases back to back, separated by grid barriers:
+//   pooling -> | scores, each block histogramming the first digit of the rows
+//   it wrote -> | digit pass 1 -> | pass 2 -> | per-row counts over contiguous
+//   row chunks -> | each chunk: offsets from the earlier chunks' totals, tie
+//   quotas, list compaction -> | tile plan
+// Results are bit for bit those of the separate calls (the same scoring
+// bodies and order of every floating-point operation; the same keys and tie
+// rule in the selection).  Every barrier wait is bounded: on timeout the grid
+// raises the device status word and every block returns.
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
@@ -31,16 +32,21 @@ using scimpl::kTI;
 using scimpl::PoolTensor;
 using scimpl::pool_body;
 using scimpl::score_body;
+using scimpl::score_rows_offset;
 using scimpl::score_smem_bytes;
-using selimpl::count_body;
+using selimpl::count_chunk_body;
+using selimpl::finish_chunk_body;
+using selimpl::hist0_rows_body;
 using selimpl::hist_body;
 using selimpl::kBins;
 using selimpl::kPasses;
-using selimpl::scan_body;
 using selimpl::SelWs;
-using selimpl::write_body;
 
 constexpr int kAnchorThreads = 256;  // the selection bodies need exactly 256
+// the first digit's bins sit in the score staging, in front of the kept rows
+static_assert(scimpl::kTI * (64 + 4) * sizeof(float) + scimpl::kTJ * (64 + 4) * sizeof(float) >=
+                  sizeof(int) * selimpl::kBins,
+              "bins overlap the kept score rows");
 constexpr int kBarriers = 8;
 
 struct AnchorArgs {
@@ -103,32 +109,41 @@ __global__ void __launch_bounds__(kAnchorThreads, 1) anchor_kernel(AnchorArgs a)
   pool_body<T, 16, true>(a.tq, a.tk, a.B, a.L, a.d, a.bs, blockIdx.x, nblk);
   if (!grid_barrier(a, 0, &give_up)) return;
 
-  // ---- pooled products and row softmax: items (query-block tile, head, batch)
+  // ---- pooled products and row softmax: items (query-block tile, head, batch);
+  // each block then adds its rows to the first digit's histogram
   const int ntile = (a.nb + kTI - 1) / kTI;
-  for (int v = blockIdx.x; v < ntile * a.H * a.B; v += nblk)
-    score_body(a.qbar, a.kbar, a.scores, a.H, a.Hkv, a.nb, a.d, a.scale, v % ntile,
-               (v / ntile) % a.H, v / (ntile * a.H), reinterpret_cast<float*>(dsm));
+  for (int v = blockIdx.x; v < ntile * a.H * a.B; v += nblk) {
+    const int ti = v % ntile, h = (v / ntile) % a.H, b = v / (ntile * a.H);
+    float* sm = reinterpret_cast<float*>(dsm);
+    score_body<true>(a.qbar, a.kbar, a.scores, a.H, a.Hkv, a.nb, a.d, a.scale, ti, h, b, sm);
+    // the item's rows stay in shared memory; the bins take the staging in front
+    const int i0 = ti * kTI, nrows = a.nb - i0 < kTI ? a.nb - i0 : kTI;
+    hist0_rows_body(sm + score_rows_offset(a.d), nrows, a.nb, i0, a.kfree, a.ws, b,
+                    reinterpret_cast<int*>(dsm));
+  }
   if (!grid_barrier(a, 1, &give_up)) return;
 
-  // ---- radix select: three digit passes over every sequence's scores
+  // ---- radix select: the other two digit passes over every sequence's scores
   const int nck = nblk / a.B > 0 ? nblk / a.B : 1;  // chunks per sequence
-  for (int p = 0; p < kPasses; ++p) {
+  for (int p = 1; p < kPasses; ++p) {
     for (int v = blockIdx.x; v < nck * a.B; v += nblk)
       hist_body(a.scores, a.B, a.H, a.nb, a.kfree, p, a.ws, v % nck, nck, v / nck);
-    if (!grid_barrier(a, 2 + p, &give_up)) return;
+    if (!grid_barrier(a, 1 + p, &give_up)) return;
   }
-  for (int v = blockIdx.x; v < nck * a.B; v += nblk)
-    count_body(a.scores, a.B, a.H, a.nb, a.kfree, a.ws, v % nck, nck, v / nck);
-  if (!grid_barrier(a, 5, &give_up)) return;
-  if (blockIdx.x == 0) scan_body(a.B, a.H, a.nb, a.kfree, a.ws, a.row_ptr, nullptr);
-  if (!grid_barrier(a, 6, &give_up)) return;
-  for (int v = blockIdx.x; v < nck * a.B; v += nblk)
-    write_body(a.scores, a.B, a.H, a.nb, a.ws, a.row_ptr, a.col_idx, nullptr, v % nck, nck,
-               v / nck);
+  // ---- per-row counts over contiguous row chunks, then every chunk's offsets
+  // from the earlier chunks' totals, tie quotas and lists
+  const int rows = a.H * a.nb;
+  const int ncx = nck < rows ? nck : rows;
+  for (int v = blockIdx.x; v < ncx * a.B; v += nblk)
+    count_chunk_body(a.scores, a.B, a.H, a.nb, a.kfree, a.ws, v % ncx, ncx, v / ncx);
+  if (!grid_barrier(a, 4, &give_up)) return;
+  for (int v = blockIdx.x; v < ncx * a.B; v += nblk)
+    finish_chunk_body(a.scores, a.B, a.H, a.nb, a.ws, a.row_ptr, a.col_idx, v % ncx, ncx,
+                      v / ncx);
   if (a.plan == nullptr) return;
 
   // ---- tile plan (needs every list of a head)
-  if (!grid_barrier(a, 7, &give_up)) return;
+  if (!grid_barrier(a, 5, &give_up)) return;
   if (a.nb <= kPlanMaxNb) {
     for (int v = blockIdx.x; v < a.H * a.B; v += nblk)
       plan_body(a.row_ptr, a.col_idx, a.H, a.nb, a.n_qt, a.plan, v % a.H, v / a.H, dsm);

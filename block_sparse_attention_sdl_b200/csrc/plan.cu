@@ -21,13 +21,28 @@ namespace {
 
 using namespace planimpl;
 
-// grid (H, B); dynamic shared memory PlanSmem::bytes(nb)
+// grid (H, B); dynamic shared memory PlanSmem::bytes(nb); nb <= 32 * NW
+template <int NW>
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ row_ptr,
                                                             const int32_t* __restrict__ col_idx,
                                                             int H, int nb, int n_qt,
                                                             int32_t* __restrict__ plan) {
   extern __shared__ __align__(16) uint8_t psm[];
-  plan_body(row_ptr, col_idx, H, nb, n_qt, plan, blockIdx.x, blockIdx.y, psm);
+  plan_body_w<NW>(row_ptr, col_idx, H, nb, n_qt, plan, blockIdx.x, blockIdx.y, psm);
+}
+
+template <int NW>
+cudaError_t launch_plan_w(const int32_t* row_ptr, const int32_t* col_idx, int B, int H, int nb,
+                          int32_t* plan, cudaStream_t st) {
+  static std::atomic<bool> attr_set[64];  // per device; the maximum is constant
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(plan_kernel<NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)PlanSmem::bytes(32 * NW));
+  });
+  if (e != cudaSuccess) return e;
+  plan_kernel<NW><<<dim3(H, B), kPlanThreads, PlanSmem::bytes(nb), st>>>(row_ptr, col_idx, H, nb,
+                                                                       (nb + 1) / 2, plan);
+  return cudaGetLastError();
 }
 
 constexpr int kOrderThreads = 1024;
@@ -149,15 +164,10 @@ cudaError_t launch_plan(const int32_t* row_ptr, const int32_t* col_idx, int B, i
     adjacent_plan_kernel<<<grid, 256, 0, st>>>(n_tiles, nb, n_qt, plan);
     return cudaGetLastError();
   }
-  const size_t smem = PlanSmem::bytes(nb);
-  static std::atomic<bool> attr_set[64];  // per device; the maximum is constant
-  cudaError_t e = once_per_device(attr_set, [] {
-    return cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)PlanSmem::bytes(kPlanMaxNb));
-  });
-  if (e != cudaSuccess) return e;
-  plan_kernel<<<dim3(H, B), kPlanThreads, smem, st>>>(row_ptr, col_idx, H, nb, n_qt, plan);
-  return cudaGetLastError();
+  if (nb <= 32) return launch_plan_w<1>(row_ptr, col_idx, B, H, nb, plan, st);
+  if (nb <= 64) return launch_plan_w<2>(row_ptr, col_idx, B, H, nb, plan, st);
+  if (nb <= 128) return launch_plan_w<4>(row_ptr, col_idx, B, H, nb, plan, st);
+  return launch_plan_w<8>(row_ptr, col_idx, B, H, nb, plan, st);
 }
 
 cudaError_t launch_tile_order(const int32_t* row_ptr, const int32_t* plan, int B, int H, int nb,

@@ -24,11 +24,13 @@ struct PlanSmem {
 };
 
 // Block (head h, batch element b), any multiple of 32 threads; shared memory
-// `psm` of PlanSmem::bytes(nb), 16-byte aligned.
-__device__ __forceinline__ void plan_body(const int32_t* __restrict__ row_ptr,
-                                          const int32_t* __restrict__ col_idx, int H, int nb,
-                                          int n_qt, int32_t* __restrict__ plan, int h, int b,
-                                          uint8_t* psm) {
+// `psm` of PlanSmem::bytes(nb), 16-byte aligned.  NW >= ceil(nb / 32): the
+// bitmap words (and lane chunks) the loops are unrolled for.
+template <int NW>
+__device__ __forceinline__ void plan_body_w(const int32_t* __restrict__ row_ptr,
+                                            const int32_t* __restrict__ col_idx, int H, int nb,
+                                            int n_qt, int32_t* __restrict__ plan, int h, int b,
+                                            uint8_t* psm) {
   const int nthr = blockDim.x;
   const int nw = (nb + 31) / 32;
   uint32_t* bits = reinterpret_cast<uint32_t*>(psm);
@@ -70,13 +72,13 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ row_ptr,
   // intersections, one warp per row i: lanes read consecutive words of the
   // word-major bitmaps and write consecutive entries (no bank conflicts)
   for (int i = warp; i < nb; i += nwarps) {
-    uint32_t bi[kPlanMaxNb / 32];
+    uint32_t bi[NW];
 #pragma unroll
-    for (int w = 0; w < kPlanMaxNb / 32; ++w) bi[w] = w < nw ? bits[w * nb + i] : 0u;
+    for (int w = 0; w < NW; ++w) bi[w] = w < nw ? bits[w * nb + i] : 0u;
     for (int j = lane; j < nb; j += 32) {
       int c = 0;
 #pragma unroll
-      for (int w = 0; w < kPlanMaxNb / 32; ++w)
+      for (int w = 0; w < NW; ++w)
         if (w < nw) c += __popc(bi[w] & bits[w * nb + j]);
       ov[i * nb + j] = (uint16_t)c;
     }
@@ -109,9 +111,9 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ row_ptr,
       // candidate keys of row i, (intersection + 1) << 16 | (0xFFFF - j): the
       // largest is the largest intersection, lowest index on ties.  They do not
       // depend on the pairing so far, so their loads leave the serial chain.
-      uint32_t kj[kPlanMaxNb / 32];
+      uint32_t kj[NW];
 #pragma unroll
-      for (int c = 0; c < kPlanMaxNb / 32; ++c) {
+      for (int c = 0; c < NW; ++c) {
         const int j = lane + 32 * c;
         kj[c] = (c < nc && j < nb)
                     ? ((uint32_t)ov[i * nb + j] + 1u) << 16 | (0xFFFFu - (uint32_t)j)
@@ -122,7 +124,7 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ row_ptr,
       // the unpaired partner with the largest key; 0 when none is left
       uint32_t key = 0;
 #pragma unroll
-      for (int c = 0; c < kPlanMaxNb / 32; ++c)
+      for (int c = 0; c < NW; ++c)
         if ((unpaired >> c) & 1u) key = kj[c] > key ? kj[c] : key;
       key = __reduce_max_sync(0xffffffffu, key);
       const int best = key ? (int)(0xFFFFu - (key & 0xFFFFu)) : -1;
@@ -135,6 +137,21 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ row_ptr,
     }
   }
   __syncthreads();  // shared memory may be reused by the block's next item
+}
+
+__device__ __forceinline__ void plan_body(const int32_t* __restrict__ row_ptr,
+                                          const int32_t* __restrict__ col_idx, int H, int nb,
+                                          int n_qt, int32_t* __restrict__ plan, int h, int b,
+                                          uint8_t* psm) {
+  static_assert(kPlanMaxNb == 256, "unrolled for at most 8 bitmap words");
+  if (nb <= 32)
+    plan_body_w<1>(row_ptr, col_idx, H, nb, n_qt, plan, h, b, psm);
+  else if (nb <= 64)
+    plan_body_w<2>(row_ptr, col_idx, H, nb, n_qt, plan, h, b, psm);
+  else if (nb <= 128)
+    plan_body_w<4>(row_ptr, col_idx, H, nb, n_qt, plan, h, b, psm);
+  else
+    plan_body_w<8>(row_ptr, col_idx, H, nb, n_qt, plan, h, b, psm);
 }
 
 }  // namespace

@@ -170,7 +170,7 @@ __device__ __forceinline__ void stage_wait() {
 // barriers); shared memory `sm` of score_smem_bytes(nb, D):
 //   qs [kTI][D+4], ks [kTJ][D+4], z [kTI][nb] floats.
 // Every score is computed by the same arithmetic for either NT.
-template <int D, int NT = kScoreThreads>
+template <int D, int NT = kScoreThreads, bool kKeep = false>
 __device__ __forceinline__ void score_body_d(const float* __restrict__ qbar,
                                              const float* __restrict__ kbar,
                                              float* __restrict__ scores, int H, int Hkv, int nb,
@@ -279,7 +279,9 @@ __device__ __forceinline__ void score_body_d(const float* __restrict__ qbar,
       float4* dst = reinterpret_cast<float4*>(scores + (((int64_t)b * H + h) * nb + (i0 + r)) * nb);
       for (int j = lane; j < n4; j += 32) {
         const float4 v = zr[j];
-        dst[j] = make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+        const float4 p = make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+        dst[j] = p;
+        if (kKeep) zr[j] = p;
       }
     }
     __syncthreads();  // z may be reused by the block's next item
@@ -302,20 +304,30 @@ __device__ __forceinline__ void score_body_d(const float* __restrict__ qbar,
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     const float inv = 1.0f / s;
     float* dst = scores + (((int64_t)b * H + h) * nb + (i0 + r)) * nb;
-    for (int j = lane; j < nb; j += 32) dst[j] = zr[j] * inv;
+    for (int j = lane; j < nb; j += 32) {
+      const float p = zr[j] * inv;
+      dst[j] = p;
+      if (kKeep) zr[j] = p;
+    }
   }
   __syncthreads();  // z may be reused by the block's next item
 }
 
+// kKeep: the item's normalized rows also stay in shared memory, at
+// score_rows_offset(d) floats into `sm`, row r at r * nb (the values written
+// to `scores`), until the block's next use of `sm`.
+template <bool kKeep = false>
 __device__ __forceinline__ void score_body(const float* __restrict__ qbar,
                                            const float* __restrict__ kbar,
                                            float* __restrict__ scores, int H, int Hkv, int nb,
                                            int d, float scale, int bx, int h, int b, float* sm) {
   if (d == 128)
-    score_body_d<128>(qbar, kbar, scores, H, Hkv, nb, scale, bx, h, b, sm);
+    score_body_d<128, kScoreThreads, kKeep>(qbar, kbar, scores, H, Hkv, nb, scale, bx, h, b, sm);
   else
-    score_body_d<64>(qbar, kbar, scores, H, Hkv, nb, scale, bx, h, b, sm);
+    score_body_d<64, kScoreThreads, kKeep>(qbar, kbar, scores, H, Hkv, nb, scale, bx, h, b, sm);
 }
+
+__host__ __device__ inline size_t score_rows_offset(int d) { return (size_t)(kTI + kTJ) * (d + 4); }
 
 }  // namespace
 }  // namespace scimpl

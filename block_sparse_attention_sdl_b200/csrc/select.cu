@@ -65,9 +65,7 @@ __global__ void __launch_bounds__(kThreads) totals_kernel(int B, int H, int nb, 
 }  // namespace
 
 size_t select_workspace_bytes(int B, int H, int nb) {
-  const size_t R = (size_t)B * H * nb;
-  return align256(sizeof(int) * (size_t)kPasses * B * kBins) + 3 * align256(sizeof(int) * R) +
-         align256(sizeof(uint32_t) * (size_t)B);
+  return selimpl::carve_bytes(B, (size_t)B * H * nb);
 }
 
 cudaError_t launch_select(const float* scores, int B, int H, int nb, int64_t kb, int32_t* row_ptr,

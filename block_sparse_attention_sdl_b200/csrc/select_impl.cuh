@@ -34,6 +34,8 @@ struct SelWs {
   int* eq;        // [R] off-diagonal scores equal to the threshold, per row
   int* take;      // [R] ties this row keeps
   uint32_t* tau;  // [B] threshold bit pattern (0xFFFFFFFF: no free picks)
+  uint32_t* krem; // [B] threshold ties to keep (the chunked count and finish)
+  int2* agg;      // [R] per row chunk: (ties, kept without ties) (chunked count)
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -50,7 +52,17 @@ SelWs carve(void* ws, int B, int R) {
   w.take = reinterpret_cast<int*>(p);
   p += align256(sizeof(int) * (size_t)R);
   w.tau = reinterpret_cast<uint32_t*>(p);
+  p += align256(sizeof(uint32_t) * (size_t)B);
+  w.krem = reinterpret_cast<uint32_t*>(p);
+  p += align256(sizeof(uint32_t) * (size_t)B);
+  w.agg = reinterpret_cast<int2*>(p);
   return w;
+}
+
+// Bytes carve() lays out for B batch elements and R rows in total.
+__host__ inline size_t carve_bytes(int B, size_t R) {
+  return align256(sizeof(int) * (size_t)kPasses * B * kBins) + 3 * align256(sizeof(int) * R) +
+         2 * align256(sizeof(uint32_t) * (size_t)B) + align256(sizeof(int2) * R);
 }
 
 // Block-wide: walk the histograms of passes [0, npass) of batch element b and
@@ -349,6 +361,214 @@ __device__ __forceinline__ void write_body(const float* __restrict__ scores, int
       const uint32_t smask = __ballot_sync(0xffffffffu, sel);
       if (sel) col_idx[pos + __popc(smask & ((1u << lane) - 1u))] = j;
       if (mask && j < nb) mask[row * nb + j] = sel ? 1 : 0;
+      pos += __popc(smask);
+    }
+  }
+}
+
+// ---- chunked variant (one launch; used by the fused anchor kernel)
+//
+// Pass 0 is histogrammed by the blocks that just wrote the scores (rows of one
+// head), and the count, tie hand-out, row offsets and list writing run over
+// contiguous chunks of rows: after the counts, a block takes the kept totals
+// of every earlier chunk instead of waiting for one block's serial scan.  The
+// results are those of hist/count/scan/write above (same keys, same rule).
+
+// Pass-0 histogram of `nrows` rows of scores held in shared memory (`z`, row
+// r at r * nb, query block i0 + r, of batch element b; off-diagonal scores),
+// added into the pass-0 histogram of b.  Requires blockDim.x == kThreads;
+// `sh`: kBins ints of shared memory apart from `z`.  A block barrier must
+// separate the rows' writes from the call.
+__device__ __forceinline__ void hist0_rows_body(const float* z, int nrows, int nb, int i0,
+                                                uint32_t kfree, SelWs ws, int b, int* sh) {
+  if (kfree == 0 || nrows <= 0) return;
+  for (int x = threadIdx.x; x < kBins; x += kThreads) sh[x] = 0;
+  __syncthreads();
+  const int shift = kShift[0];
+  const uint32_t dmask = (1u << kWidth[0]) - 1u;
+  const int lane = threadIdx.x % 32;
+  // one warp per row; every lane of a warp makes the same number of calls
+  for (int r = (int)threadIdx.x / 32; r < nrows; r += kThreads / 32)
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      const bool in = j < nb;
+      const uint32_t key = in ? __float_as_uint(z[r * nb + j]) : 0u;
+      hist_add(sh, (int)((key >> shift) & dmask), in && j != i0 + r);
+    }
+  __syncthreads();
+  int* gh = ws.hist + (size_t)b * kBins;  // pass 0
+  for (int x = threadIdx.x; x <= (int)dmask; x += kThreads)
+    if (sh[x]) atomicAdd(&gh[x], sh[x]);
+  __syncthreads();  // the bins may be reused by the block's next rows
+}
+
+// Rows [r0, r1) of chunk cx of ncx for H*nb rows per batch element.
+__device__ __forceinline__ void chunk_rows(int rows, int cx, int ncx, int& r0, int& r1) {
+  const int per = (rows + ncx - 1) / ncx;
+  r0 = cx * per < rows ? cx * per : rows;
+  r1 = r0 + per < rows ? r0 + per : rows;
+}
+
+// Block (chunk cx of ncx, batch element b), ncx <= H*nb: per-row counts of
+// off-diagonal scores above and at the threshold, and the chunk's totals
+// (ties, rows' kept entries without ties) in ws.agg[b * ncx + cx].  Chunk 0
+// also stores the threshold and the ties to keep.
+__device__ __forceinline__ void count_chunk_body(const float* __restrict__ scores, int B, int H,
+                                                 int nb, uint32_t kfree, SelWs ws, int cx,
+                                                 int ncx, int b) {
+  __shared__ int s_eq, s_g1;
+  uint32_t tau = 0xFFFFFFFFu, krem = 0;
+  if (kfree > 0) resolve(ws.hist, B, b, kPasses, kfree, &tau, &krem);
+  if (threadIdx.x == 0) {
+    s_eq = 0;
+    s_g1 = 0;
+    if (cx == 0) {
+      ws.tau[b] = tau;
+      ws.krem[b] = krem;
+    }
+  }
+  __syncthreads();
+  const int lane = threadIdx.x % 32;
+  const int rows = H * nb;
+  int r0, r1;
+  chunk_rows(rows, cx, ncx, r0, r1);
+  for (int r = r0 + (int)threadIdx.x / 32; r < r1; r += kThreads / 32) {
+    const int i = r % nb;
+    const int64_t row = (int64_t)b * rows + r;
+    const float* pr = scores + row * nb;
+    int gt = 0, eq = 0;
+    for (int j = lane; j < nb; j += 32) {
+      if (j == i) continue;
+      const uint32_t key = __float_as_uint(__ldg(pr + j));
+      gt += key > tau && tau != 0xFFFFFFFFu;
+      eq += key == tau;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      gt += __shfl_xor_sync(0xffffffffu, gt, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (lane == 0) {
+      ws.gt[row] = gt;
+      ws.eq[row] = eq;
+      atomicAdd(&s_eq, eq);
+      atomicAdd(&s_g1, gt + 1);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) ws.agg[(int64_t)b * ncx + cx] = make_int2(s_eq, s_g1);
+}
+
+// Block-wide sums of (x, y) over threads; every thread gets them.
+__device__ __forceinline__ int2 block_sum2(int x, int y, int2* s_part) {
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarp = blockDim.x / 32;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    x += __shfl_xor_sync(0xffffffffu, x, o);
+    y += __shfl_xor_sync(0xffffffffu, y, o);
+  }
+  if (lane == 0) s_part[warp] = make_int2(x, y);
+  __syncthreads();
+  int2 t = make_int2(0, 0);
+  for (int w = 0; w < nwarp; ++w) {
+    t.x += s_part[w].x;
+    t.y += s_part[w].y;
+  }
+  __syncthreads();  // s_part may be reused
+  return t;
+}
+
+// Block (chunk cx of ncx, batch element b), after every count_chunk_body:
+// the chunk's rows' offsets into the lists and tie quotas (ties go to rows in
+// flat order), then their kept blocks in ascending j (as write_body).  The
+// chunk holding the last row of the last batch element writes the end offset.
+__device__ __forceinline__ void finish_chunk_body(const float* __restrict__ scores, int B, int H,
+                                                  int nb, SelWs ws, int32_t* __restrict__ row_ptr,
+                                                  int32_t* __restrict__ col_idx, int cx, int ncx,
+                                                  int b) {
+  __shared__ int2 s_part[kThreads / 32];
+  __shared__ int s_base;
+  const int rows = H * nb;
+  // kept entries of the earlier batch elements, then of the earlier chunks of b
+  int base = 0, eq0 = 0;
+  for (int bb = 0; bb <= b; ++bb) {
+    const int nc = bb < b ? ncx : cx;
+    int x = 0, y = 0;
+    for (int c = threadIdx.x; c < nc; c += kThreads) {
+      const int2 v = ws.agg[(int64_t)bb * ncx + c];
+      x += v.x;
+      y += v.y;
+    }
+    const int2 t = block_sum2(x, y, s_part);
+    // ties go to the earliest rows: min(quota, ties seen) of them are kept
+    const int kr = (int)ws.krem[bb];
+    base += t.y + (t.x < kr ? t.x : kr);
+    if (bb == b) eq0 = t.x;  // ties of the earlier chunks of b
+  }
+  int r0, r1;
+  chunk_rows(rows, cx, ncx, r0, r1);
+  const int krem = (int)ws.krem[b];
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int run_eq = eq0, pos = base;
+    for (int c0 = r0; c0 < r1; c0 += 32) {
+      const int r = c0 + lane;
+      const int64_t row = (int64_t)b * rows + r;
+      const int eqv = r < r1 ? ws.eq[row] : 0;
+      const int gtv = r < r1 ? ws.gt[row] : 0;
+      int ie = eqv;  // inclusive prefix of ties over the lanes
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, ie, o);
+        if (lane >= o) ie += u;
+      }
+      int t = krem - (run_eq + ie - eqv);
+      t = t < 0 ? 0 : (t > eqv ? eqv : t);
+      const int cnt = r < r1 ? gtv + t + 1 : 0;
+      int ic = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, ic, o);
+        if (lane >= o) ic += u;
+      }
+      if (r < r1) {
+        row_ptr[row] = pos + ic - cnt;
+        ws.take[row] = t;
+      }
+      run_eq += __shfl_sync(0xffffffffu, ie, 31);
+      pos += __shfl_sync(0xffffffffu, ic, 31);
+    }
+    if (lane == 0) s_base = pos;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && b == B - 1 && r1 == rows && r0 < r1)
+    row_ptr[(int64_t)B * rows] = s_base;
+  // the chunk's lists (the offsets and quotas above are this block's writes)
+  const uint32_t tau = ws.tau[b];
+  const int lane = threadIdx.x % 32;
+  for (int r = r0 + (int)threadIdx.x / 32; r < r1; r += kThreads / 32) {
+    const int i = r % nb;
+    const int64_t row = (int64_t)b * rows + r;
+    const float* pr = scores + row * nb;
+    int pos = row_ptr[row];
+    int ties_left = ws.take[row];
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      bool sel = false, tie = false;
+      if (j < nb) {
+        const uint32_t key = __float_as_uint(__ldg(pr + j));
+        if (j == i)
+          sel = true;
+        else if (tau != 0xFFFFFFFFu && key > tau)
+          sel = true;
+        else if (key == tau)
+          tie = true;
+      }
+      const uint32_t tmask = __ballot_sync(0xffffffffu, tie);
+      if (tie) sel = __popc(tmask & ((1u << lane) - 1u)) < ties_left;
+      ties_left -= __popc(tmask);
+      const uint32_t smask = __ballot_sync(0xffffffffu, sel);
+      if (sel) col_idx[pos + __popc(smask & ((1u << lane) - 1u))] = j;
       pos += __popc(smask);
     }
   }

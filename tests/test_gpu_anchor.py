@@ -55,6 +55,32 @@ def test_fused_anchor_equals_separate_calls(dtype, B, L, H, H_kv, d, bs, s):
     assert int(rp[-1]) == kept
 
 
+@pytest.mark.parametrize("B,H,L,s", [(2, 4, 1024, 0.6), (3, 8, 2048, 0.85)])
+def test_fused_anchor_hands_out_ties_in_row_order(B, H, L, s):
+    """Q = 0: every row's scores are exactly 1/nb, so every off-diagonal score ties
+    with the threshold and the quota of ties runs through the row chunks and the
+    batch elements in flat row order, as the separate calls and the oracle do."""
+    w = synth.small_workload(B=B, H=H, H_kv=H, L=L, d=128, bs=64, sparsity=s, planted=2)
+    x = synth.device_inputs(w, 0)
+    q = torch.zeros_like(x["q"])
+    sc1 = sdl.block_scores(q, x["k"], 64)
+    rp1, ci1, _ = sdl.select_mask(sc1, s, 64, L)
+    sc2, rp2, ci2, _ = sdl.anchor_refresh(q, x["k"], 64, s, want_plan=False)
+    torch.cuda.synchronize()
+    assert sdl.last_device_status() == sdl.SDL_OK
+    assert torch.equal(sc1, sc2)
+    nb = L // 64
+    assert bool((sc2 == 1.0 / nb).all())
+    assert torch.equal(rp1, rp2) and torch.equal(ci1, ci2)
+    want, _, kept = oracle.select(sc2.cpu().numpy().astype(np.float64), s)
+    rp, ci = rp2.cpu().numpy(), ci2.cpu().numpy()
+    mask = np.zeros((B * H * nb, nb), dtype=np.uint8)
+    for r in range(B * H * nb):
+        mask[r, ci[rp[r]:rp[r + 1]]] = 1
+    assert np.array_equal(mask.reshape(want.shape), want)
+    assert int(rp[-1]) == kept
+
+
 def test_fused_anchor_repeated_launches_on_one_workspace():
     """The barrier counters are reset for every launch: back-to-back refreshes on
     one workspace and distinct inputs stay exact."""
