@@ -472,6 +472,22 @@ def cpu_oracle_sample(w, seed, target_s=20.0):
     return flops(rows) / dt / 1e12, cores, desc, dt, extra
 
 
+def run_config(args, w, world: int) -> dict:
+    """The bench line's `config` for a workload, variant and launch (both arms)."""
+    heads = args.shard == "heads"
+    sparsed = args.variant == "sparsed"
+    return {"workload": args.workload, "global_batch": w.B * (1 if heads else world),
+            "seq_len": w.L, "heads": w.H, "kv_heads": w.H_kv, "head_dim": w.d, "block": w.bs,
+            "sparsity": w.sparsity, "anchor_every": None if sparsed else w.anchor_every,
+            "dense_steps": args.dense_steps if sparsed else 0,
+            "budget": ("key columns per head" if args.variant == "pulsecol" else
+                       "per head" if args.variant == "uniform-head" else
+                       "per sequence, across heads"),
+            "parallelism": (f"heads split over {world} ranks" if heads else
+                            f"independent sequences x{world}"),
+            "l2": "inputs larger than L2 (192 MiB per step, distinct per step)"}
+
+
 def run_reference(args):
     """The reference arm: the fp64 CPU oracle, timed per step on a bounded sample."""
     rank = int(os.environ.get("RANK", "0"))
@@ -492,9 +508,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox, see synth/)",
-        "config": {"workload": args.workload, "global_batch": w.B, "seq_len": w.L,
-                   "heads": w.H, "kv_heads": w.H_kv, "head_dim": w.d, "block": w.bs,
-                   "sparsity": w.sparsity, "parallelism": "cpu oracle"},
+        "config": run_config(args, w, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": desc, **extra},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -680,16 +694,7 @@ def main():
         "dtype": "bf16",
         "data": "synthetic (seeded Philox inputs shaped like the 8K/90% workload, regenerated "
                 "per step)",
-        "config": {"workload": args.workload, "global_batch": w.B * seqs, "seq_len": w.L,
-                   "heads": w.H, "kv_heads": w.H_kv, "head_dim": w.d, "block": w.bs,
-                   "sparsity": w.sparsity, "anchor_every": runner.interval,
-                   "dense_steps": runner.dense_steps,
-                   "budget": ("key columns per head" if runner.pulsecol else
-                              "per head" if runner.att.per_head else
-                              "per sequence, across heads"),
-                   "parallelism": (f"heads split over {world} ranks" if heads else
-                                   f"independent sequences x{world}"),
-                   "l2": "inputs larger than L2 (192 MiB per step, distinct per step)"},
+        "config": run_config(args, w, world),
         "variant": args.variant,
         "sparse_attn_ms": sp_avg, "sparse_attn_tflops": kernel_tflops,
         "sparse_attn_ms_p10_p50_p90": [sp_q[0], statistics.median(sparse_ms), sp_q[-1]],
