@@ -361,14 +361,16 @@ def csr_mask(row_ptr: np.ndarray, col_idx: np.ndarray, B: int, H: int, nb: int) 
     return mask.reshape(B, H, nb, nb)
 
 
-def parity_check(runner, w, seed, step, out, n_random=2, rows_per_block=4):
+def parity_check(runner, w, seed, step, out, n_random=2, rows_per_block=4, mask=None):
     """Outside the timed region: the output of timed step `step` (`out`, on the
     device) on sampled query rows against the fp64 oracle with the GPU's own mask
     (all heads; per head the first and last query block, the block with the
     longest kept list and `n_random` others), and the GPU's mask of that step's
     anchor against the oracle's selection (differences allowed only within 1e-5
     relative of the oracle's threshold, and counted).  Attention under the
-    oracle's own mask on the same rows is reported beside it, not checked."""
+    oracle's own mask on the same rows is reported beside it, not checked.
+    `mask`: (row_ptr, col_idx) as they were at that step, when the layer's own
+    buffers have been refreshed since."""
     import oracle
     import synth
     rt = runner.rt
@@ -383,8 +385,9 @@ def parity_check(runner, w, seed, step, out, n_random=2, rows_per_block=4):
         gpu_mask = None
         lens = np.full((w.B, H, nb), nb)
     else:
-        rp = runner.att.row_ptr.cpu().numpy()
-        ci = runner.att.col_idx.cpu().numpy()
+        rp_t, ci_t = mask if mask is not None else (runner.att.row_ptr, runner.att.col_idx)
+        rp = rp_t.cpu().numpy()
+        ci = ci_t.cpu().numpy()
         gpu_mask = csr_mask(rp, ci, w.B, H, nb)
         lens = np.diff(rp).reshape(w.B, H, nb)
         ha = host if a_step == step else synth.host_inputs(w, a_step, seed)
@@ -602,6 +605,9 @@ def main():
     sdl = runner.sdl
     status_timed = sdl.last_device_status()
     last_out = runner.out.clone()
+    # the mask the last timed step used (the separate timings below refresh it)
+    last_mask = (None if runner.pulsecol else
+                 (runner.att.row_ptr.clone(), runner.att.col_idx.clone()))
 
     pk, pk_kind = peaks()
     budget = runner.att.budget  # kept blocks of the whole sequence
@@ -676,7 +682,7 @@ def main():
 
     parity = None
     if rank == 0 and not heads:
-        parity = parity_check(runner, w, seed, steps[-1], last_out)
+        parity = parity_check(runner, w, seed, steps[-1], last_out, mask=last_mask)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

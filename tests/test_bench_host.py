@@ -96,3 +96,35 @@ def test_parity_check_passes_the_oracle_output_and_catches_a_wrong_one():
     bad = out.clone()
     bad[0, w.L - 1, 1] += 0.05   # the last row of the last query block is always sampled
     assert not bench.parity_check(runner, w, 0, step, bad)["ok"]
+
+
+def test_parity_check_reads_the_mask_snapshot_of_the_checked_step():
+    """The bench refreshes the layer's mask after the timed loop (separate timings on
+    step 0's inputs); the check must judge the mask the checked step used, passed as
+    a snapshot, and a stale mask in the layer's buffers must not be read instead."""
+    import numpy as np
+    import torch
+    import oracle
+    import synth
+    w = synth.small_workload(L=512, H=2, H_kv=1, d=64, sparsity=0.5, planted=1, steps=4,
+                             anchor_every=2)
+    step = 2
+
+    def csr_of(s):
+        h = synth.host_inputs(w, s)
+        m, _, _ = oracle.select(oracle.block_scores(h["q"], h["k"], w.bs), w.sparsity)
+        r = m.reshape(-1, w.nb)
+        rp = np.concatenate([[0], np.cumsum(r.sum(1))]).astype(np.int32)
+        ci = np.concatenate([np.flatnonzero(x) for x in r]).astype(np.int32)
+        return m, torch.as_tensor(rp), torch.as_tensor(ci)
+
+    mask2, rp2, ci2 = csr_of(step)
+    mask0, rp0, ci0 = csr_of(0)
+    assert not np.array_equal(mask0, mask2)
+    host = synth.host_inputs(w, step)
+    O, _ = oracle.attention(host["q"], host["k"], host["v"], w.bs, mask=mask2)
+    out = torch.as_tensor(O.transpose(0, 2, 1, 3).copy()).to(torch.bfloat16)
+    runner = _FakeRunner(_FakeAtt(rp0, ci0), w.anchor_every)  # refreshed since: step 0's
+    assert not bench.parity_check(runner, w, 0, step, out)["ok"]
+    res = bench.parity_check(runner, w, 0, step, out, mask=(rp2, ci2))
+    assert res["ok"] and res["mask_entries_other"] == 0, res
