@@ -591,6 +591,9 @@ def main():
     # timed region.  The timed schedule then builds its own masks.
     runner.prime(inputs[0])
     torch.cuda.synchronize()
+    sdl = runner.sdl
+    status_warm = sdl.last_device_status()  # warm-up and priming (clears the word)
+    detail_warm = sdl.last_device_detail()
 
     sampler = ClockSampler(local)
     for attempt in range(2):
@@ -602,8 +605,8 @@ def main():
     ms_max = max_over_ranks(ms, dist_on, device)
     # outside the timed region: the device status word, and the last timed
     # step's output kept for the parity check (later launches reuse the buffer)
-    sdl = runner.sdl
     status_timed = sdl.last_device_status()
+    detail_timed = sdl.last_device_detail()
     last_out = runner.out.clone()
     # the mask the last timed step used (the separate timings below refresh it)
     last_mask = (None if runner.pulsecol else
@@ -679,6 +682,7 @@ def main():
         e2e = {"value": job_rate(flop_step, len(steps), seqs, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e_ms / len(steps)}
     status_after = sdl.last_device_status()  # the e2e loop and the separate timings
+    detail_after = sdl.last_device_detail()
 
     parity = None
     if rank == 0 and not heads:
@@ -733,7 +737,8 @@ def main():
                              w.bs, runner.att.sharded, runner.att.fused,
                              runner.att.lists is not None)),
         "clocks": sampler.summary(),
-        "device_status": {"timed": status_timed, "after": status_after},
+        "device_status": {"warmup": status_warm, "timed": status_timed, "after": status_after,
+                          "bad_mask_detail": [detail_warm, detail_timed, detail_after]},
         "parity": parity,
     }
     if rank == 0:
@@ -743,7 +748,7 @@ def main():
         dist.destroy_process_group()
     # a kernel that reported a timeout or a rejected list entry, or an output
     # off the oracle, voids the line's numbers
-    if status_timed != sdl.SDL_OK or status_after != sdl.SDL_OK:
+    if any(st != sdl.SDL_OK for st in (status_warm, status_timed, status_after)):
         sys.exit(3)
     if parity is not None and not parity["ok"]:
         sys.exit(4)

@@ -40,7 +40,8 @@ EXPORTS = ("sdl_mask_budget", "sdl_scores_workspace_bytes", "sdl_select_workspac
            "sdl_select_shard_capacity", "sdl_select_shard_pass", "sdl_select_shard_count",
            "sdl_select_shard_finish",
            "sdl_wait_selfcheck",
-           "sdl_last_device_status", "sdl_last_cuda_error", "sdl_status_string")
+           "sdl_last_device_status", "sdl_last_device_detail", "sdl_last_cuda_error",
+           "sdl_status_string")
 SDL_SELECT_PASSES = 3
 
 
@@ -122,6 +123,7 @@ def _lib():
         L.sdl_wait_selfcheck.argtypes = [ctypes.c_uint64, P]
         L.sdl_last_device_status.argtypes = [P]
         L.sdl_last_cuda_error.argtypes = []
+        L.sdl_last_device_detail.argtypes = []
         L.sdl_status_string.argtypes = [ctypes.c_int]
         L.sdl_status_string.restype = ctypes.c_char_p
         for f in ("sdl_block_scores", "sdl_select_mask", "sdl_select_mask_scoped",
@@ -134,7 +136,7 @@ def _lib():
                   "sdl_sparse_attn_planned", "sdl_tile_order", "sdl_sparse_attn_scheduled",
                   "sdl_tile_lists", "sdl_sparse_attn_listed",
                   "sdl_dense_attn",
-                  "sdl_last_device_status", "sdl_last_cuda_error"):
+                  "sdl_last_device_status", "sdl_last_device_detail", "sdl_last_cuda_error"):
             getattr(L, f).restype = ctypes.c_int
         _L = L
     return _L
@@ -692,3 +694,18 @@ def wait_selfcheck(limit_ns: int = 1_000_000, stream=None):
 def last_device_status(stream=None) -> int:
     """Synchronizes the stream and returns (and clears) the kernels' status code."""
     return int(_lib().sdl_last_device_status(_stream(stream)))
+
+
+BAD_MASK_SITES = {1: "tile plan entry", 2: "CSR entry", 3: "tile-lists record",
+                  4: "tile-lists record rows", 5: "tile-lists entry",
+                  6: "take-order entry (attention)", 7: "take-order entry (tile lists)",
+                  8: "CSR entry (fp32 kernel)"}
+
+
+def last_device_detail():
+    """(site name, offending value) of the bad-mask report behind the last
+    :func:`last_device_status` of this thread, or None (``sdl_last_device_detail``)."""
+    d = int(_lib().sdl_last_device_detail())
+    if d == 0:
+        return None
+    return BAD_MASK_SITES.get(d >> 24, f"site {d >> 24}"), d & 0xFFFFFF

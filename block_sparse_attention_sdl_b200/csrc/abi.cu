@@ -11,11 +11,13 @@
 
 namespace sdl {
 
-__device__ int g_device_status;
+// [0]: status bits; [1]: the first bad-mask report's site and value
+__device__ int g_device_status[2];
 
 namespace {
 
 thread_local int t_last_cuda_error = 0;
+thread_local int t_last_device_detail = 0;
 
 sdl_status cuda_fail(cudaError_t e) {
   t_last_cuda_error = (int)e;
@@ -719,12 +721,14 @@ sdl_status sdl_wait_selfcheck(uint64_t limit_ns, void* stream) {
 sdl_status sdl_last_device_status(void* stream) {
   cudaError_t ce = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (ce != cudaSuccess) return cuda_fail(ce);
-  int v = 0;
-  ce = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+  int w[2] = {0, 0};
+  ce = cudaMemcpyFromSymbol(w, g_device_status, sizeof(w));
   if (ce != cudaSuccess) return cuda_fail(ce);
-  const int zero = 0;
-  ce = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  const int zero[2] = {0, 0};
+  ce = cudaMemcpyToSymbol(g_device_status, zero, sizeof(zero));
   if (ce != cudaSuccess) return cuda_fail(ce);
+  const int v = w[0];
+  t_last_device_detail = (v & kDevBadMask) ? w[1] : 0;
   if (v & kDevTimeout) return SDL_ERR_TIMEOUT;
   if (v & kDevBadMask) return SDL_ERR_BAD_MASK;
   if (v & kDevOverlap) return SDL_ERR_OVERLAP;
@@ -732,6 +736,8 @@ sdl_status sdl_last_device_status(void* stream) {
 }
 
 int sdl_last_cuda_error(void) { return t_last_cuda_error; }
+
+int sdl_last_device_detail(void) { return t_last_device_detail; }
 
 const char* sdl_status_string(sdl_status status) {
   switch (status) {

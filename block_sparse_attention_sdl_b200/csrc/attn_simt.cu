@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
     for (int x = beg + tid; x < end; x += kThreads) {
       const int j = a.col_idx[x];
       if (j < 0 || j >= a.nb || (x > beg && a.col_idx[x - 1] >= j)) {
-        atomicOr(a.status, kDevBadMask);
+        report_bad_mask(a.status, kBadSimtEntry, j);
         if (j < 0 || j >= a.nb) continue;
       }
       for (int u = 0; u < per; ++u) {

@@ -177,7 +177,8 @@ __device__ __forceinline__ void tile_of(const AttnArgs& a, int item, int n_qt, i
   if (a.plan != nullptr) {
     // the tile's two query blocks from the plan (64-token blocks)
     const int qb0 = a.plan[2 * (int64_t)item], qb1 = a.plan[2 * (int64_t)item + 1];
-    if (qb0 >= a.nb || qb0 < -1 || qb1 >= a.nb || qb1 < -1) atomicOr(a.status, kDevBadMask);
+    if (qb0 >= a.nb || qb0 < -1 || qb1 >= a.nb || qb1 < -1)
+      report_bad_mask(a.status, kBadPlanEntry, item);
     t0 = (qb0 >= 0 && qb0 < a.nb) ? qb0 * 64 : a.L;
     t1 = (qb1 >= 0 && qb1 < a.nb) ? qb1 * 64 : a.L;
   } else {
@@ -212,7 +213,8 @@ __device__ int union_list(const AttnArgs& a, int b, int h, int t0, int t1,
       for (int x = beg + lane; x < end; x += 32) {
         const int jb = a.col_idx[x];
         const bool bad_range = jb < 0 || jb >= a.nb;
-        if (bad_range || (x > beg && a.col_idx[x - 1] >= jb)) atomicOr(a.status, kDevBadMask);
+        if (bad_range || (x > beg && a.col_idx[x - 1] >= jb))
+          report_bad_mask(a.status, kBadListEntry, jb);
         if (bad_range) continue;
         for (int u = 0; u < per; ++u) {
           const int s = jb * per + u;
@@ -303,7 +305,7 @@ __device__ bool build_item(const AttnArgs& a, const CUtensorMap* tmq, Slot& S,
       item = rec.x;
       n_ent = rec.y;
       if (item < 0 || item >= n_items || n_ent < 0 || n_ent > nsub) {
-        if (lane == 0) atomicOr(a.status, kDevBadMask);
+        if (lane == 0) report_bad_mask(a.status, kBadRecord, item);
         continue;
       }
       b = item / (a.H * n_qt);
@@ -311,7 +313,7 @@ __device__ bool build_item(const AttnArgs& a, const CUtensorMap* tmq, Slot& S,
       t0 = rec.z;
       t1 = rec.w;
       if (t0 < 0 || t0 > a.L || t1 < 0 || t1 > a.L) {
-        if (lane == 0) atomicOr(a.status, kDevBadMask);
+        if (lane == 0) report_bad_mask(a.status, kBadRecordRows, t0);
         continue;
       }
       const uint16_t* src = reinterpret_cast<const uint16_t*>(a.lists + (int64_t)n_items *
@@ -320,7 +322,7 @@ __device__ bool build_item(const AttnArgs& a, const CUtensorMap* tmq, Slot& S,
       for (int x = lane; x < n_ent; x += 32) {
         uint16_t e = src[x];
         if ((int)(e & kSubMask) >= nsub) {
-          atomicOr(a.status, kDevBadMask);
+          report_bad_mask(a.status, kBadRecordEntry, e);
           e = 0;
         }
         S.ent[x] = e;
@@ -331,7 +333,7 @@ __device__ bool build_item(const AttnArgs& a, const CUtensorMap* tmq, Slot& S,
         // costliest tiles first (the order is a permutation of the items)
         const int o = a.order[item];
         if (o < 0 || o >= n_items) {
-          if (lane == 0) atomicOr(a.status, kDevBadMask);
+          if (lane == 0) report_bad_mask(a.status, kBadOrderEntry, o);
           continue;
         }
         item = o;
@@ -382,7 +384,7 @@ __global__ void __launch_bounds__(kListWarps * 32) tile_lists_kernel(AttnArgs a,
     item = a.order[r];
     if (item < 0 || item >= n_items) {
       if (lane == 0) {
-        atomicOr(a.status, kDevBadMask);
+        report_bad_mask(a.status, kBadListsOrder, item);
         *reinterpret_cast<int4*>(lists + (int64_t)r * kListRecInts) = make_int4(-1, 0, 0, 0);
       }
       return;

@@ -14,10 +14,28 @@ namespace sdl {
 // kDevOverlap: two attention launches in flight shared one tile counter.
 enum : int { kDevTimeout = 1, kDevBadMask = 2, kDevOverlap = 4 };
 
+// Sites of bad-mask reports.  The word after the status word records the first
+// report since the last read: site << 24 | the low 24 bits of the offending value.
+enum : int {
+  kBadPlanEntry = 1,    // a tile plan entry outside [-1, nb)
+  kBadListEntry = 2,    // a CSR entry out of range or not ascending (value: the entry)
+  kBadRecord = 3,       // a tile-lists record's tile or length (value: the tile)
+  kBadRecordRows = 4,   // a tile-lists record's first tokens (value: t0)
+  kBadRecordEntry = 5,  // a tile-lists entry's key sub-block (value: the entry)
+  kBadOrderEntry = 6,   // a take-order entry, attention kernel (value: the entry)
+  kBadListsOrder = 7,   // a take-order entry, tile-lists kernel (value: the entry)
+  kBadSimtEntry = 8,    // a CSR entry, fp32 kernel (value: the entry)
+};
+
+__device__ __forceinline__ void report_bad_mask(int* status, int site, int value) {
+  atomicOr(status, kDevBadMask);
+  atomicCAS(status + 1, 0, (site << 24) | (value & 0xFFFFFF));
+}
+
 // Wall-time bound for every spin wait inside a kernel.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-int* device_status_ptr();  // address of the library's device status word
+int* device_status_ptr();  // the library's device status word and its detail word
 
 // List entries handed to the attention kernels: 64-token key sub-block index
 // in the low 16 bits, and in bits 16..17 which halves (query rows 0..63,

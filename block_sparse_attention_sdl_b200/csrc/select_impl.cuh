@@ -69,10 +69,18 @@ __host__ inline size_t carve_bytes(int B, size_t R) {
 // return the digit prefix of the k-th largest key and how many of the keys
 // sharing that prefix still have to be taken.  All threads of the block get
 // the result.  Requires blockDim.x == kThreads.
+//
+// Every thread compares against its own copy of the prefix and the count
+// left; the one thread whose bins hold the k-th key publishes the new values
+// in shared memory, and all threads take them only after the next barrier.
+// (Reading the shared count in the same barrier interval as its update let a
+// late thread see the updated count, match one of its own bins as well and
+// corrupt the prefix.)
 __device__ void resolve(const int* hist, int B, int b, int npass, uint32_t kfree,
                         uint32_t* prefix_out, uint32_t* krem_out) {
   __shared__ uint32_t s_prefix, s_krem;
   __shared__ int s_warp[kThreads / 32];
+  uint32_t prefix = 0, krem = kfree;
   if (threadIdx.x == 0) {
     s_prefix = 0;
     s_krem = kfree;
@@ -102,23 +110,24 @@ __device__ void resolve(const int* hist, int B, int b, int npass, uint32_t kfree
     __syncthreads();
     int wbase = 0;
     for (int w = 0; w < warp; ++w) wbase += s_warp[w];
-    const uint32_t krem = s_krem;
     uint32_t above = (uint32_t)(wbase + incl - local);
 #pragma unroll
     for (int x = 0; x < 8; ++x) {
       if (x >= per) break;
       uint32_t c = (uint32_t)cnt[x];
       if (above < krem && above + c >= krem) {
-        s_prefix |= (uint32_t)(hi - 1 - x) << kShift[p];
+        s_prefix = prefix | (uint32_t)(hi - 1 - x) << kShift[p];
         s_krem = krem - above;
       }
       above += c;
     }
     __syncthreads();
+    prefix = s_prefix;
+    krem = s_krem;
   }
-  *prefix_out = s_prefix;
-  *krem_out = s_krem;
-  __syncthreads();
+  *prefix_out = prefix;
+  *krem_out = krem;
+  __syncthreads();  // the shared values may be rewritten by the block's next call
 }
 
 

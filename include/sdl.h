@@ -380,6 +380,17 @@ sdl_status sdl_dense_attn(const void* q, const void* k, const void* v, const sdl
  * these in that order when several bits are set. */
 sdl_status sdl_last_device_status(void* stream);
 
+/* Where the bad-mask report behind the last sdl_last_device_status of this
+ * thread came from: 0 if it reported none, else site << 24 | the low 24 bits
+ * of the offending value, for the first report since the read before it.
+ * Sites: 1 a tile-plan entry outside [-1, nb) (value: the tile); 2 a CSR
+ * entry out of range or not ascending (the entry); 3 a tile-lists record's
+ * tile or length (the tile); 4 a record's first tokens (t0); 5 a list entry's
+ * key sub-block (the entry); 6 a take-order entry read by the attention kernel
+ * (the entry); 7 one read by sdl_tile_lists (the entry); 8 a CSR entry in the
+ * fp32 kernel (the entry).  A diagnostic: the pages describe no such word. */
+int sdl_last_device_detail(void);
+
 /* Self-check of the failure path: launches one warp that waits, through the
  * same bounded wait every kernel of the library uses, on an mbarrier phase
  * that nothing completes, giving up after `limit_ns` (1 us .. 1 s, else

@@ -179,3 +179,45 @@ def test_tile_order_exact_at_scale(B, H, nb, cap):
         ok = qb >= 0
         cost[ok] += lens[head[ok] * nb + qb[ok]]
     assert np.array_equal(order, np.argsort(-cost, kind="stable"))
+
+
+@pytest.mark.parametrize("per_head", [False, True])
+def test_selection_is_the_same_over_many_back_to_back_calls(per_head):
+    """The radix resolution is shared by every block of the count and digit-pass
+    kernels; a race there (a thread reading the count left after another thread had
+    updated it) made a few selections of long runs write rows out of order.  On the
+    8K workload's block scores at four anchors, 40 calls each, queued back to back,
+    must all give the oracle's CSR."""
+    w = synth.WORKLOADS["bf16-L8192-H32-s90"]
+    nb, s = w.nb, w.sparsity
+    for step in (0, 32, 64, 96):
+        x = synth.device_inputs(w, step)
+        scores = sdl.block_scores(x["q"], x["k"], w.bs)
+        want, _, kept = oracle.select(scores.cpu().numpy().astype(np.float64), s,
+                                      per_head=per_head)
+        outs = [sdl.select_mask(scores, s, w.bs, w.L, per_head=per_head)[:2]
+                for _ in range(40)]
+        torch.cuda.synchronize()
+        assert sdl.last_device_status() == sdl.SDL_OK, (step, sdl.last_device_detail())
+        rp0, ci0 = outs[0][0].cpu().numpy(), outs[0][1].cpu().numpy()
+        mask = np.zeros((w.B * w.H * nb, nb), dtype=np.uint8)
+        for r in range(w.B * w.H * nb):
+            mask[r, ci0[rp0[r]:rp0[r + 1]]] = 1
+        assert np.array_equal(mask.reshape(want.shape), want) and int(rp0[-1]) == kept, step
+        for k, (rp, ci) in enumerate(outs[1:]):
+            assert torch.equal(rp, outs[0][0]) and torch.equal(ci, outs[0][1]), (step, k)
+
+
+def test_fused_anchor_is_the_same_over_many_back_to_back_calls():
+    """The fused kernel resolves the threshold in its digit-pass and count phases
+    with the same shared routine: at four anchors of the 8K workload, 30 queued
+    calls each give one result."""
+    w = synth.WORKLOADS["bf16-L8192-H32-s90"]
+    for step in (0, 32, 64, 96):
+        x = synth.device_inputs(w, step)
+        outs = [sdl.anchor_refresh(x["q"], x["k"], w.bs, w.sparsity, want_plan=False)[1:3]
+                for _ in range(30)]
+        torch.cuda.synchronize()
+        assert sdl.last_device_status() == sdl.SDL_OK, (step, sdl.last_device_detail())
+        for k, (rp, ci) in enumerate(outs[1:]):
+            assert torch.equal(rp, outs[0][0]) and torch.equal(ci, outs[0][1]), (step, k)

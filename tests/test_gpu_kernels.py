@@ -415,6 +415,8 @@ def test_bad_tile_order_entry_is_reported():
     order = torch.tensor([1, 5], dtype=torch.int32, device="cuda")  # 5: no such tile
     sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, plan=plan, order=order)
     assert sdl.last_device_status() == sdl.SDL_ERR_BAD_MASK
+    assert sdl.last_device_detail() == ("take-order entry (attention)", 5)
+    assert sdl.last_device_status() == sdl.SDL_OK and sdl.last_device_detail() is None
 
 
 def test_bad_tile_plan_entry_is_reported():
@@ -425,6 +427,7 @@ def test_bad_tile_plan_entry_is_reported():
     plan = torch.tensor([[[[0, 1], [2, 77]]]], dtype=torch.int32, device="cuda")  # 77 >= nb
     sdl.sparse_attn(dev["q"], dev["k"], dev["v"], rp, ci, 64, plan=plan)
     assert sdl.last_device_status() == sdl.SDL_ERR_BAD_MASK
+    assert sdl.last_device_detail() == ("tile plan entry", 1)  # tile 1 holds the 77
 
 
 def test_repeated_launches_on_two_streams_are_identical():
