@@ -727,6 +727,10 @@ def main():
         "sparse_attn_ms_p10_p50_p90": [sp_q[0], statistics.median(sparse_ms), sp_q[-1]],
         "dense_steps_timed": n_dense_steps,
         "pct_bf16_peak": kernel_tflops / peak,
+        # against the measured sustained figure (a GEMM back to back under the power
+        # cap): the fair denominator when long tensor-bound launches settle at the cap
+        "pct_bf16_peak_sustained": kernel_tflops / pk.get(
+            "bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]),
         "dense_attn_ms": dense_ms, "dense_attn_tflops": dense_flop / (dense_ms * 1e-3) / 1e12,
         "speedup_vs_dense": dense_ms / sp_avg,
         "speedup_vs_dense_amortized": dense_ms / (ms_max / len(steps)),
