@@ -24,6 +24,8 @@ CASES = [
     ("bf16", 1, 512, 4, 4, 64, 64, 1 - 1 / 8),  # diagonal only
     ("bf16", 1, 17408, 2, 2, 64, 64, 0.95),     # nb = 272: adjacent pairs
     ("bf16", 1, 8192, 32, 32, 128, 64, 0.9),    # the 8K workload's shape
+    ("bf16", 1, 1024, 4, 4, 64, 64, 0.0),       # keep everything: the threshold is the minimum
+    ("bf16", 3, 576, 3, 1, 64, 64, 0.5),        # three sequences, nb = 9: one row per chunk
 ]
 
 
