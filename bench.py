@@ -247,6 +247,16 @@ def job_rate(flop_per_step: float, n_steps: int, world: int, ms_max: float) -> f
     return flop_per_step * n_steps * world / (ms_max * 1e-3) / 1e12
 
 
+def any_rank(flag: bool, dist_on, device) -> bool:
+    """True on every rank if `flag` is true on any of them."""
+    if not dist_on:
+        return bool(flag)
+    import torch.distributed as dist
+    t = torch.tensor([1 if flag else 0], dtype=torch.int32, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return bool(t.item())
+
+
 def max_over_ranks(x, dist_on, device):
     if not dist_on:
         return x
@@ -616,7 +626,8 @@ def main():
     for attempt in range(2):
         with sampler:
             ms, ev = time_steps(runner, inputs, steps, dist_on, device)
-        if not sampler.rejected():
+        # every rank takes the same decision (a retry runs the timed loop's barriers)
+        if not any_rank(sampler.rejected(), dist_on, device):
             break
         sampler = ClockSampler(local)
     ms_max = max_over_ranks(ms, dist_on, device)

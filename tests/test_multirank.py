@@ -47,10 +47,13 @@ def _rank_main(rank, world, port, out_dir):
         all_d = [torch.zeros(1, dtype=torch.float64) for _ in range(world)]
         dist.all_gather(all_d, digest)
         rate = bench.job_rate(2.0e9, 4, world, ms)
+        # a clock rejection on one rank makes every rank retry the timed loop
+        retry = bench.any_rank(rank == 1, True, cpu)
+        keep = bench.any_rank(False, True, cpu)
         bench.barrier(True)
         np.save(os.path.join(out_dir, f"rank{rank}.npy"),
                 np.array([ms, rate, float(np.array_equal(np.asarray(q), np.asarray(q2)))] +
-                         [float(d.item()) for d in all_d]))
+                         [float(d.item()) for d in all_d] + [float(retry), float(keep)]))
     finally:
         dist.destroy_process_group()
 
@@ -71,6 +74,7 @@ def test_two_rank_gloo_timing_and_seeds(tmp_path):
     assert r0[2] == r1[2] == 1.0                       # a rank's inputs are reproducible
     assert r0[3] == r1[3] and r0[4] == r1[4]           # every rank saw the same digests
     assert r0[3] != r0[4]                              # and the two sequences differ
+    assert r0[5] == r1[5] == 1.0 and r0[6] == r1[6] == 0.0  # one decision on every rank
 
 
 def test_reference_arm_runs_on_rank_zero_only():
