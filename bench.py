@@ -73,9 +73,10 @@ def parse():
                         "exchanges (strong scaling)")
     p.add_argument("--dense-steps", type=int, default=32,
                    help="dense warm-up steps of the sparsed variant")
-    p.add_argument("--profile", choices=["sparse", "dense"], default=None,
-                   help="launch only this attention kernel (warmup + steps times, one input) "
-                        "and print its event-timed average; for profiler captures")
+    p.add_argument("--profile", choices=["sparse", "dense", "scores"], default=None,
+                   help="launch only this attention kernel, or (scores) the separate block-"
+                        "score and selection calls (warmup + steps times, one input), and "
+                        "print the event-timed average; for profiler captures")
     return p.parse_args()
 
 
@@ -552,7 +553,14 @@ def profile_kernel(runner, args):
     x = runner.make_inputs([0])[0]
     runner.att.refresh(x["q"], x["k"], 0)
     torch.cuda.synchronize()
-    if args.profile == "sparse":
+    if args.profile == "scores":
+        # the anchor's parts as separate calls: block scores (pool + score kernels),
+        # then the selection kernels on those scores
+        att = runner.att
+        fn = lambda: (sdl.block_scores(x["q"], x["k"], w.bs, scores=att.scores,
+                                       workspace=att.ws_scores), att.select())
+        flop = 0.0
+    elif args.profile == "sparse":
         fn = lambda: sdl.sparse_attn(x["q"], x["k"], x["v"], runner.att.row_ptr,
                                      runner.att.col_idx, w.bs, out=runner.out,
                                      plan=runner.att.plan, order=runner.att.order,
